@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the frozen-NF4 QLoRA linear layer on B200.
+
+One step = one pass of the whole hot path over one batch, on inputs already
+resident in HBM:
+    quantize W (fp32 -> NF4 + double quant) -> dequantize to bf16
+    -> forward (Y, sT) -> backward (dX, dA, dB)
+Workload: the LLaMA-7B attention projection, W 4096 x 4096 (0.1% outliers),
+M = 4096 tokens (8 x 512), r = 16, alpha = 32, synthetic seeded inputs.
+Two input sets alternate between steps; one step touches ~0.26 GB, more than
+the 126 MB L2.
+
+Metric value: fwd+bwd algorithmic TFLOP/s = (4MNK + 6Mr(N+K)) / step time,
+whole job (all ranks). Under torchrun every rank runs an independent replica
+(weak scaling, no collective on the data path); timing is the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+_CORES = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+for _v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+    os.environ.setdefault(_v, str(_CORES))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and tokens/s; NF4 dequant GB/s (% of roofline)"
+CFG = synth.ATTN7B
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def fwd_bwd_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (N + K)
+
+
+def workload_config(cfg, extra=None):
+    c = {"workload": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "r": cfg.r, "alpha": cfg.alpha,
+         "step": "quantize(W fp32) + dequantize(bf16) + forward + backward",
+         "l2": "inputs larger than L2: two alternating input sets, ~0.26 GB touched per step"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------- clocks ------
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            target = str(device)
+            try:
+                bus = torch.cuda.get_device_properties(device).pci_bus_id
+                if bus:
+                    target = bus
+            except AttributeError:
+                pass
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", target], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------- CPU oracle leg ----
+
+class OracleSample:
+    """The CPU oracle on a proportional slice of the workload: m_s tokens
+    forward+backward in fp64 against the oracle's dequantised W, plus the
+    quantisation and dequantisation of m_s rows of W (the share of the
+    one-per-step weight work that m_s of the M tokens carry)."""
+
+    def __init__(self, cfg):
+        import oracle
+        self.o = oracle
+        self.cfg = cfg
+        W = synth.weight(cfg).numpy()
+        z = oracle.quantize_nf4(W)
+        self.W = W
+        self.What = oracle.bf16_bits_to_f64(
+            oracle.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], cfg.N, cfg.K))
+        self.X = synth.activations(cfg).float().numpy().astype(np.float64)
+        self.dY = synth.grad_output(cfg).float().numpy().astype(np.float64)
+        self.A = synth.lora_a(cfg).float().numpy().astype(np.float64)
+        self.B = synth.lora_b(cfg).float().numpy().astype(np.float64)
+        self.threads = oracle.num_threads()
+
+    def step(self, m_s: int, offset: int = 0):
+        c = self.cfg
+        lo = offset % (c.M - m_s + 1)
+        rows = slice(lo, lo + m_s)
+        wrows = slice(lo % (c.N - m_s + 1), lo % (c.N - m_s + 1) + m_s) if m_s <= c.N else slice(0, c.N)
+        z = self.o.quantize_nf4(self.W[wrows])
+        self.o.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], z["N"], z["K"])
+        X, dY = self.X[rows], self.dY[rows]
+        self.o.forward(X, self.What, self.A, self.B, c.alpha, c.r)
+        self.o.backward(dY, X, self.What, self.A, self.B, c.alpha, c.r)
+
+    def flops(self, m_s):
+        return fwd_bwd_flops(m_s, self.cfg.N, self.cfg.K, self.cfg.r)
+
+    def calibrate(self, target_s: float) -> int:
+        t0 = time.perf_counter()
+        self.step(16)
+        dt = max(time.perf_counter() - t0, 1e-4)
+        m = int(16 * target_s / dt)
+        m_s = 1
+        while m_s * 2 <= max(m, 1) and m_s * 2 <= self.cfg.M:
+            m_s *= 2
+        return m_s
+
+    def sample_line(self, seconds: float = 10.0):
+        m_s = self.calibrate(1.0)
+        n = 0
+        t0 = time.perf_counter()
+        while True:
+            self.step(m_s, offset=n * m_s)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+        value = self.flops(m_s) * n / el / 1e12
+        return {"value": value, "unit": "TFLOP/s", "cores": self.threads, "kind": "oracle",
+                "sample": f"{n} slices of {m_s} tokens fwd+bwd (fp64 numpy) + quantize/dequantize of {m_s} "
+                          f"rows of W (C oracle), {el:.1f} s on {self.threads} host threads"}
+
+
+# ------------------------------------------------------------ reference ----
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    s = OracleSample(CFG)
+    budget = 150.0 / max(args.steps + args.warmup, 1)  # whole run within ~2.5 minutes
+    m_s = s.calibrate(budget)
+    for i in range(args.warmup):
+        s.step(m_s, offset=i * m_s)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        s.step(m_s, offset=(args.warmup + i) * m_s)
+    el = time.perf_counter() - t0
+    value = s.flops(m_s) * args.steps / el / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": workload_config(CFG, {"sample_tokens_per_step": m_s,
+                                            "reference": "CPU oracle (C + numpy fp64), no GPU"}),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle",
+                             "sample": f"per step: {m_s} tokens fwd+bwd + quantize/dequantize of {m_s} rows of W"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ours ---
+
+def run_ours(args, rank, world, local_rank):
+    import bit_nf4_quantized_09_b200 as q
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    cfg = CFG
+    M, N, K, r, alpha = cfg.M, cfg.N, cfg.K, cfg.r, cfg.alpha
+    host = [dict(W=synth.weight(cfg), X=synth.activations(cfg), A=synth.lora_a(cfg), B=synth.lora_b(cfg),
+                 dY=synth.grad_output(cfg))]
+    # second input set: the same distributions, other seeds
+    cfg2 = synth.custom(N=N, K=K, M=M, r=r, alpha=alpha, seed_base=77, outliers=True)
+    host.append(dict(W=synth.weight(cfg2), X=synth.activations(cfg2), A=synth.lora_a(cfg2),
+                     B=synth.lora_b(cfg2), dY=synth.grad_output(cfg2)))
+    sets = [{k: v.to(dev) for k, v in h.items()} for h in host]
+
+    w = q.NF4Weight.empty(N, K, dev)
+    Wbf = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+    ws_q = torch.empty(q.workspace_bytes(q.OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
+    ws_f = torch.empty(q.workspace_bytes(q.OP_FWD, M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.workspace_bytes(q.OP_BWD, M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step(i, prof=None):
+        s = sets[i % 2]
+        q.quantize_nf4(s["W"], out=w, ws=ws_q)
+        q.dequantize_nf4(w, out=Wbf)
+        if prof is not None:
+            q.profile_next_launch(q.KERNEL_FUSED_FWD, *prof[0])
+            q.profile_next_launch(q.KERNEL_FUSED_DX, *prof[1])
+        q.linear_fwd(s["X"], w, s["A"], s["B"], alpha, Y=Y, sT=sT, ws=ws_f)
+        q.linear_bwd(s["dY"], s["X"], w, s["A"], s["B"], alpha, sT=sT, dX=dX, dA=dA, dB=dB, ws=ws_b)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K whole steps, events around each fused matmul too
+    prof = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+            for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = q.launch_count()
+    sampler = ClockSampler(local_rank)
+    time.sleep(0.15)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        step(i, prof[i])
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    launches = q.launch_count() - launches0
+    ms = start.elapsed_time(stop) / args.steps
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    fwd_ms = statistics.mean(p[0][0].elapsed_time(p[0][1]) for p in prof)
+    dx_ms = statistics.mean(p[1][0].elapsed_time(p[1][1]) for p in prof)
+
+    # ---- per-row breakdown (outside the timed region, same inputs)
+    def timed(fn, n=20):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn(0)
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    rows_ms = {
+        "quantize": timed(lambda i: q.quantize_nf4(sets[i % 2]["W"], out=w, ws=ws_q)),
+        "dequantize": timed(lambda i: q.dequantize_nf4(w, out=Wbf)),
+        "forward": timed(lambda i: q.linear_fwd(sets[i % 2]["X"], w, sets[i % 2]["A"], sets[i % 2]["B"], alpha,
+                                                Y=Y, sT=sT, ws=ws_f)),
+        "backward": timed(lambda i: q.linear_bwd(sets[i % 2]["dY"], sets[i % 2]["X"], w, sets[i % 2]["A"],
+                                                 sets[i % 2]["B"], alpha, sT=sT, dX=dX, dA=dA, dB=dB, ws=ws_b)),
+    }
+
+    # ---- end to end through the public API with host buffers
+    pin = [{k: v.pin_memory() for k, v in h.items()} for h in host]
+    out_host = dict(Y=torch.empty_like(Y, device="cpu").pin_memory(), dX=torch.empty_like(dX, device="cpu").pin_memory(),
+                    dA=torch.empty_like(dA, device="cpu").pin_memory(), dB=torch.empty_like(dB, device="cpu").pin_memory(),
+                    Wbf=torch.empty_like(Wbf, device="cpu").pin_memory())
+    h2d = sum(v.numel() * v.element_size() for v in pin[0].values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+
+    def e2e_step(i):
+        s, p = sets[i % 2], pin[i % 2]
+        for k in s:
+            s[k].copy_(p[k], non_blocking=True)
+        step(i)
+        out_host["Y"].copy_(Y, non_blocking=True)
+        out_host["dX"].copy_(dX, non_blocking=True)
+        out_host["dA"].copy_(dA, non_blocking=True)
+        out_host["dB"].copy_(dB, non_blocking=True)
+        out_host["Wbf"].copy_(Wbf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 30))
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if pg is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flops = fwd_bwd_flops(M, N, K, r)
+    value = flops * world / (ms * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    # dominant kernel: the fused matmul with the larger time per step
+    kern = {"fused_forward": (fwd_ms, 2 * M * N * (K + r)), "fused_dx": (dx_ms, 2 * M * K * (N + r))}
+    dom = max(kern, key=lambda k: kern[k][0])
+    d_ms, d_flops = kern[dom]
+    achieved = d_flops / (d_ms * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    deq_bytes = N * K * (0.5 + 1 / 64 + 4 / 16384 + 2)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg),
+        "tokens_per_s": M * world / (ms * 1e-3),
+        "dequant_gbs": deq_bytes / (rows_ms["dequantize"] * 1e-3) / 1e9,
+        "rows_ms": rows_ms,
+        "kernels_ms": {"fused_forward": fwd_ms, "fused_dx": dx_ms},
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_kind": f"bf16 sustained ({pk_kind})"},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = OracleSample(cfg).sample_line(args.cpu_seconds)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,600 @@
+// C ABI of libqlora_nf4.so: argument checks, workspace layout, TMA tensor
+// maps and the launch sequence of each call. All compute happens in the
+// kernels of quantize.cu, gemm_fused.cu and gemm_skinny.cu.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/qlora_nf4.h"
+#include "kernels.h"
+
+using namespace qlora;
+
+namespace {
+
+// ------------------------------------------------------------ options ----
+std::atomic<int64_t> g_small_m_max{-1};
+std::atomic<int64_t> g_fail_launches{0};
+std::atomic<int64_t> g_timeout_us{1000000};
+std::atomic<int64_t> g_stall_producer{0};
+std::atomic<int64_t> g_launch_count{0};
+thread_local std::string g_last_error;
+
+// One-shot event requests of qlora_profile_next_launch, per kernel id.
+std::mutex g_prof_mu;
+cudaEvent_t g_prof_events[3][2] = {};
+
+void take_profile_events(int kernel, cudaEvent_t* start, cudaEvent_t* stop) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    *start = g_prof_events[kernel][0];
+    *stop = g_prof_events[kernel][1];
+    g_prof_events[kernel][0] = g_prof_events[kernel][1] = nullptr;
+}
+
+qlora_status cuda_fail(cudaError_t e, const char* where) {
+    g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+    return QLORA_ERR_CUDA;
+}
+
+#define QLORA_TRY(expr, where)                          \
+    do {                                                \
+        cudaError_t e_ = (expr);                        \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+// A launch of `nkernels` kernels of this library.
+#define QLORA_LAUNCH(expr, nkernels, where)             \
+    do {                                                \
+        cudaError_t e_ = (expr);                        \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+        g_launch_count += (nkernels);                   \
+    } while (0)
+
+int tree_passes(int64_t nb) {
+    int passes = 1;
+    int64_t n = (nb + 1023) / 1024;
+    if (n == 1) return 2;
+    while (n > 1) {
+        n = (n + 1023) / 1024;
+        ++passes;
+    }
+    return passes;
+}
+
+// Host-side fault injection: consumes one "launch" and reports a failure
+// before anything reaches the GPU.
+bool injected_failure() {
+    int64_t n = g_fail_launches.load();
+    while (n > 0) {
+        if (g_fail_launches.compare_exchange_weak(n, n - 1)) {
+            g_last_error = "injected launch failure";
+            return true;
+        }
+    }
+    return false;
+}
+
+// ------------------------------------------------------------ NF4 tables --
+// Independent host computation of the levels (normal quantiles by Newton's
+// method on Phi) and of the decision thresholds: for each neighbour pair the
+// exact midpoint rounded toward -infinity to fp32, so that "v > threshold"
+// means "v is strictly nearer the upper level" and an exact tie stays below.
+double std_normal_quantile(double p) {
+    // Phi is concave on x >= 0, so Newton's method from x = 0 climbs
+    // monotonically to the root for p > 1/2.
+    double x = 0.0;
+    for (int i = 0; i < 200; ++i) {
+        const double f = 0.5 * std::erfc(-x / std::sqrt(2.0)) - p;
+        const double d = std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI);
+        const double nx = x - f / d;
+        if (nx == x) break;
+        x = nx;
+    }
+    return x;
+}
+
+Nf4Tables build_tables() {
+    Nf4Tables t{};
+    const double top = 0.9677083;
+    double v[16];
+    int n = 0;
+    for (int k = 0; k < 8; ++k) v[n++] = std_normal_quantile(top - k * ((top - 0.5) / 8.0));   // 8 positive
+    for (int k = 0; k < 7; ++k) v[n++] = -std_normal_quantile(top - k * ((top - 0.5) / 7.0));  // 7 negative
+    v[n++] = 0.0;                                                                           // exact zero
+    std::sort(v, v + 16);
+    for (int k = 0; k < 16; ++k) t.level[k] = static_cast<float>(v[k] / v[15]);
+    for (int k = 0; k < 15; ++k) {
+        const double mid = (static_cast<double>(t.level[k]) + static_cast<double>(t.level[k + 1])) * 0.5;
+        float f = static_cast<float>(mid);
+        if (static_cast<double>(f) > mid) f = std::nextafter(f, -INFINITY);
+        t.thresh[k] = f;
+    }
+    return t;
+}
+
+const Nf4Tables& tables() {
+    static const Nf4Tables t = build_tables();
+    return t;
+}
+
+// ------------------------------------------------------------- devices ----
+struct DeviceState {
+    bool ready = false;
+    qlora_status status = QLORA_OK;
+    int sms = 0;
+};
+std::mutex g_dev_mu;
+DeviceState g_dev[64];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Checks the current device once (sm_100, 148-SM class) and opts the big
+// kernels in to their shared-memory sizes.
+qlora_status device_ready(int* sms_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceState& d = g_dev[dev];
+    if (!d.ready) {
+        d.ready = true;
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
+            d.status = cuda_fail(e, "cudaDeviceGetAttribute");
+        } else if (major != 10 || minor != 0) {
+            g_last_error = "device is not sm_100 (compute capability " + std::to_string(major) + "." +
+                           std::to_string(minor) + ")";
+            d.status = QLORA_ERR_UNSUPPORTED_DEVICE;
+        } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess) {
+            d.status = cuda_fail(e, "cudaFuncSetAttribute");
+        } else if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+                d.status = cuda_fail(e == cudaSuccess ? cudaErrorSymbolNotFound : e, "cuTensorMapEncodeTiled");
+            else
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    if (sms_out) *sms_out = d.sms;
+    return d.status;
+}
+
+// 2-D tiled tensor map over a row-major [d1, d0] array (d0 contiguous).
+qlora_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                      uint64_t row_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw, const char* what) {
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {b0, b1};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_error = std::string("cuTensorMapEncodeTiled(") + what + ") failed: " + std::to_string(r);
+        return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+}
+
+#define QLORA_MAP(...)                            \
+    do {                                          \
+        qlora_status s_ = make_map(__VA_ARGS__);  \
+        if (s_ != QLORA_OK) return s_;            \
+    } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
+int rank_pad(int r) { return r < 16 ? 16 : r; }
+
+// Reduction splits of a skinny matmul: enough CTAs for two per SM of a
+// 148-SM B200 (fixed so workspace sizes do not depend on the device).
+constexpr int64_t kTargetCtas = 296;
+struct Split {
+    int splits;
+    int steps;
+};
+Split split_for(int64_t tiles, int64_t red) {
+    const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
+    int64_t s = std::max<int64_t>(1, std::min<int64_t>(cdiv(kTargetCtas, std::max<int64_t>(tiles, 1)), KT));
+    const int64_t steps = cdiv(KT, s);
+    s = cdiv(KT, steps);
+    return Split{static_cast<int>(s), static_cast<int>(steps)};
+}
+
+// ------------------------------------------------------- workspace layout --
+struct Layout {
+    size_t status = 0, cT = 0, partT = 0, sT = 0;         // forward
+    size_t Bt = 0, partU = 0, sU = 0, sUt = 0, sTt = 0;    // backward
+    size_t partA = 0, partB = 0;
+    size_t total = 0;
+    int64_t ldc = 0, ldt = 0;
+    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1};
+};
+
+Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
+    Layout L;
+    const int NR = rank_pad(r);
+    L.ldc = (N + 3) / 4 * 4;   // constants row pitch: a multiple of 16 bytes
+    L.ldt = (M + 7) / 8 * 8;   // pitch of the [r, M] transposed copies: a multiple of 16 bytes
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += up256(bytes);
+        return at;
+    };
+    L.status = take(256);
+    L.cT = take(static_cast<size_t>(K / kBlock) * L.ldc * 4);
+    const int64_t mtiles = std::max<int64_t>(1, cdiv(M, 128));
+    L.sT_split = split_for(mtiles, K);
+    if (op == QLORA_OP_FWD) {
+        L.partT = take(static_cast<size_t>(L.sT_split.splits) * M * NR * 4);
+        L.sT = take(static_cast<size_t>(M) * r * 2);
+    } else {
+        L.sU_split = split_for(mtiles, N);
+        L.grad_split = split_for(cdiv(K, 128) + cdiv(N, 128), M);
+        L.Bt = take(static_cast<size_t>(r) * N * 2);
+        const int64_t part_down = std::max(L.sU_split.splits, L.sT_split.splits);
+        L.partU = take(static_cast<size_t>(part_down) * M * NR * 4);
+        L.sU = take(static_cast<size_t>(M) * r * 2);
+        L.sUt = take(static_cast<size_t>(L.ldt) * r * 2);
+        L.sT = take(static_cast<size_t>(M) * r * 2);
+        L.sTt = take(static_cast<size_t>(L.ldt) * r * 2);
+        L.partA = take(static_cast<size_t>(L.grad_split.splits) * K * NR * 4);
+        L.partB = take(static_cast<size_t>(L.grad_split.splits) * N * NR * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+qlora_status check_weight(const qlora_nf4_weight* w) {
+    if (!w || !w->codes || !w->qabsmax || !w->s2 || !w->mean) return QLORA_ERR_INVALID_ARG;
+    if (w->N <= 0 || w->K <= 0 || w->K % kBlock != 0 || w->N % 8 != 0) return QLORA_ERR_BAD_SHAPE;
+    if (!aligned16(w->codes) || !aligned16(w->qabsmax) || !aligned16(w->s2) || (reinterpret_cast<uintptr_t>(w->mean) & 3u))
+        return QLORA_ERR_MISALIGNED;
+    return QLORA_OK;
+}
+
+uint64_t timeout_ns() { return static_cast<uint64_t>(std::max<int64_t>(1, g_timeout_us.load())) * 1000ull; }
+
+// T-side skinny matmul: part = act[M, red] . wt[r, red]^T, then
+// out = bf16(scale * sum of partials) as [M, r] (and [r, M] when out_t).
+qlora_status lora_down(const uint16_t* act, int64_t M, int64_t red, const uint16_t* wt, int r, float scale,
+                       const Split& sp, float* part, uint16_t* out, uint16_t* out_t, int64_t ldt, int* status,
+                       cudaStream_t st) {
+    const int NR = rank_pad(r);
+    CUtensorMap ta, tb;
+    QLORA_MAP(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, red, M, red * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "act");
+    QLORA_MAP(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, red, r, red * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "lora");
+    SkinnyArgs a{};
+    a.NR = NR;
+    a.a_mn_major = 0;
+    a.p[0] = SkinnyProblem{M, red, sp.splits, sp.steps, part};
+    a.p[1] = a.p[0];
+    a.status = status;
+    a.timeout_ns = timeout_ns();
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_skinny(ta, tb, ta, tb, a, 1, st), 1, "skinny(lora down)");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_reduce_lora_down(part, sp.splits, M, NR, r, scale, out, out_t, ldt, st), 1, "reduce(lora down)");
+    return QLORA_OK;
+}
+
+}  // namespace
+
+// =================================================================== ABI ==
+
+extern "C" {
+
+int64_t qlora_nf4_bytes(int64_t N, int64_t K, size_t* codes, size_t* qabsmax, size_t* s2, size_t* mean) {
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return -1;
+    const int64_t nb = N * K / kBlock, ng = cdiv(nb, kGroup);
+    const size_t c = static_cast<size_t>(N * K / 2), q = static_cast<size_t>(nb), s = static_cast<size_t>(ng) * 4, m = 4;
+    if (codes) *codes = c;
+    if (qabsmax) *qabsmax = q;
+    if (s2) *s2 = s;
+    if (mean) *mean = m;
+    return static_cast<int64_t>(c + q + s + m);
+}
+
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return 0;
+    if (op == QLORA_OP_QUANTIZE) {
+        const int64_t nb = N * K / kBlock;
+        return up256(static_cast<size_t>(nb) * 4) + up256(dq_tree_scratch_doubles(nb) * 8);
+    }
+    if (op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
+    if (M < 0 || !rank_ok(r)) return 0;
+    return layout_for(op, M, N, K, r).total;
+}
+
+const char* qlora_status_string(qlora_status s) {
+    switch (s) {
+        case QLORA_OK: return "QLORA_OK";
+        case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+        case QLORA_ERR_BAD_SHAPE: return "QLORA_ERR_BAD_SHAPE";
+        case QLORA_ERR_MISALIGNED: return "QLORA_ERR_MISALIGNED";
+        case QLORA_ERR_UNSUPPORTED_RANK: return "QLORA_ERR_UNSUPPORTED_RANK";
+        case QLORA_ERR_WORKSPACE_TOO_SMALL: return "QLORA_ERR_WORKSPACE_TOO_SMALL";
+        case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+        case QLORA_ERR_DEVICE_TIMEOUT: return "QLORA_ERR_DEVICE_TIMEOUT";
+        case QLORA_ERR_UNSUPPORTED_DEVICE: return "QLORA_ERR_UNSUPPORTED_DEVICE";
+        default: return "QLORA_ERR_UNKNOWN";
+    }
+}
+
+const char* qlora_last_error(void) { return g_last_error.c_str(); }
+
+qlora_status qlora_set_option(int option, int64_t value) {
+    switch (option) {
+        case QLORA_OPT_SMALL_M_MAX: g_small_m_max = value; return QLORA_OK;
+        case QLORA_OPT_FAIL_LAUNCHES: g_fail_launches = std::max<int64_t>(0, value); return QLORA_OK;
+        case QLORA_OPT_WAIT_TIMEOUT_US:
+            if (value <= 0) return QLORA_ERR_INVALID_ARG;
+            g_timeout_us = value;
+            return QLORA_OK;
+        case QLORA_OPT_STALL_PRODUCER: g_stall_producer = value ? 1 : 0; return QLORA_OK;
+        case QLORA_OPT_LAUNCH_COUNT: g_launch_count = value; return QLORA_OK;
+        default: return QLORA_ERR_INVALID_ARG;
+    }
+}
+
+int64_t qlora_get_option(int option) {
+    switch (option) {
+        case QLORA_OPT_SMALL_M_MAX: return g_small_m_max.load();
+        case QLORA_OPT_FAIL_LAUNCHES: return g_fail_launches.load();
+        case QLORA_OPT_WAIT_TIMEOUT_US: return g_timeout_us.load();
+        case QLORA_OPT_STALL_PRODUCER: return g_stall_producer.load();
+        case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
+        default: return -1;
+    }
+}
+
+qlora_status qlora_nf4_tables(float* levels_host, float* thresholds_host) {
+    if (!levels_host || !thresholds_host) return QLORA_ERR_INVALID_ARG;
+    const Nf4Tables& t = tables();
+    std::memcpy(levels_host, t.level, sizeof(t.level));
+    std::memcpy(thresholds_host, t.thresh, sizeof(t.thresh));
+    return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
+                                float* mean, void* ws, size_t ws_bytes, void* stream) {
+    if (!W || !codes || !qabsmax || !s2 || !mean || !ws) return QLORA_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return QLORA_ERR_BAD_SHAPE;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(qabsmax) || !aligned16(s2) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(mean) & 3u))
+        return QLORA_ERR_MISALIGNED;
+    if (ws_bytes < qlora_workspace_bytes(QLORA_OP_QUANTIZE, 0, N, K, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    qlora_status s = device_ready(&sms);
+    if (s != QLORA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t nb = N * K / kBlock;
+    float* absmax = static_cast<float*>(ws);
+    double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + up256(static_cast<size_t>(nb) * 4));
+    QLORA_LAUNCH(launch_nf4_encode(W, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
+    return QLORA_OK;
+}
+
+qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
+    if (!W_out) return QLORA_ERR_INVALID_ARG;
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
+    QLORA_LAUNCH(launch_nf4_dequant(w->codes, w->qabsmax, w->s2, w->mean, w->N, w->K, W_out, tables(), sms,
+                                    static_cast<cudaStream_t>(stream)),
+                 1, "nf4_dequant");
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
+                              const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* sT_save, void* ws,
+                              size_t ws_bytes, void* stream) {
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    if (M < 0) return QLORA_ERR_BAD_SHAPE;
+    if (!rank_ok(r)) return QLORA_ERR_UNSUPPORTED_RANK;
+    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    if (M == 0) return QLORA_OK;
+    if (!X || !A || !B || !Y || !ws) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(ws) ||
+        (sT_save && !aligned16(sT_save)))
+        return QLORA_ERR_MISALIGNED;
+    const int64_t N = w->N, K = w->K;
+    const Layout L = layout_for(QLORA_OP_FWD, M, N, K, r);
+    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(base + L.status);
+    float* cT = reinterpret_cast<float*>(base + L.cT);
+    float* partT = reinterpret_cast<float*>(base + L.partT);
+    uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
+    const float scale = alpha / static_cast<float>(r);
+
+    QLORA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st), "clear status");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
+    if ((s = lora_down(X, M, K, A, r, scale, L.sT_split, partT, sT, nullptr, 0, status, st)) != QLORA_OK) return s;
+
+    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
+    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");
+    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 32, 256, CU_TENSOR_MAP_SWIZZLE_32B,
+              "codes");
+    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+              "constants");
+    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sT, r, M, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sT");
+    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, r, N, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "B");
+    FusedArgs fa{};
+    fa.M = M;
+    fa.out_cols = N;
+    fa.red = K;
+    fa.r = r;
+    fa.out = Y;
+    fa.status = status;
+    fa.timeout_ns = timeout_ns();
+    fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+    if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused forward");
+    if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+    return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                              const uint16_t* A, const uint16_t* B, int r, float alpha, const uint16_t* sT_in,
+                              uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    if (M < 0) return QLORA_ERR_BAD_SHAPE;
+    if (!rank_ok(r)) return QLORA_ERR_UNSUPPORTED_RANK;
+    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    if (!dA || !dB || !A || !B || !ws) return QLORA_ERR_INVALID_ARG;
+    if (M > 0 && (!dY || !X || !dX)) return QLORA_ERR_INVALID_ARG;
+    if ((M > 0 && (!aligned16(dY) || !aligned16(X) || !aligned16(dX))) || !aligned16(A) || !aligned16(B) ||
+        !aligned16(dA) || !aligned16(dB) || !aligned16(ws) || (sT_in && !aligned16(sT_in)))
+        return QLORA_ERR_MISALIGNED;
+    const int64_t N = w->N, K = w->K;
+    const Layout L = layout_for(QLORA_OP_BWD, M, N, K, r);
+    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0) {  // an empty batch: the adapter gradients are exactly zero
+        QLORA_TRY(cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 4, st), "zero dA");
+        QLORA_TRY(cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 4, st), "zero dB");
+        return QLORA_OK;
+    }
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(base + L.status);
+    float* cT = reinterpret_cast<float*>(base + L.cT);
+    uint16_t* Bt = reinterpret_cast<uint16_t*>(base + L.Bt);
+    float* partU = reinterpret_cast<float*>(base + L.partU);
+    uint16_t* sU = reinterpret_cast<uint16_t*>(base + L.sU);
+    uint16_t* sUt = reinterpret_cast<uint16_t*>(base + L.sUt);
+    uint16_t* sT = reinterpret_cast<uint16_t*>(base + L.sT);
+    uint16_t* sTt = reinterpret_cast<uint16_t*>(base + L.sTt);
+    float* partA = reinterpret_cast<float*>(base + L.partA);
+    float* partB = reinterpret_cast<float*>(base + L.partB);
+    const float scale = alpha / static_cast<float>(r);
+    const int NR = rank_pad(r);
+
+    QLORA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st), "clear status");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_transpose_bf16(B, N, r, Bt, N, st), 1, "transpose B");
+    // sU = s dY B  ([M, r] and [r, M])
+    if ((s = lora_down(dY, M, N, Bt, r, scale, L.sU_split, partU, sU, sUt, L.ldt, status, st)) != QLORA_OK) return s;
+    // sT^T from the forward's sT, or sT recomputed
+    if (sT_in) {
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        QLORA_LAUNCH(launch_transpose_bf16(sT_in, M, r, sTt, L.ldt, st), 1, "transpose sT");
+    } else {
+        if ((s = lora_down(X, M, K, A, r, scale, L.sT_split, partU, sT, sTt, L.ldt, status, st)) != QLORA_OK)
+            return s;
+    }
+
+    // dX = dY deq(W) + sU A
+    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
+    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "dY");
+    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+              "codes");
+    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 4, CU_TENSOR_MAP_SWIZZLE_NONE,
+              "constants");
+    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sU, r, M, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sU");
+    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, r, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+    FusedArgs fa{};
+    fa.M = M;
+    fa.out_cols = K;
+    fa.red = N;
+    fa.r = r;
+    fa.out = dX;
+    fa.status = status;
+    fa.timeout_ns = timeout_ns();
+    fa.stall_producer = 0;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
+    if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused dX");
+    if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+
+    // dA^T[K, NR] = X^T sU  and  dB[N, NR] = dY^T sT, split over tokens
+    CUtensorMap ta0, tb0, ta1, tb1;
+    QLORA_MAP(&ta0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
+    QLORA_MAP(&tb0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sUt, M, r, L.ldt * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "sU^T");
+    QLORA_MAP(&ta1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
+    QLORA_MAP(&tb1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sTt, M, r, L.ldt * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "sT^T");
+    SkinnyArgs ga{};
+    ga.NR = NR;
+    ga.a_mn_major = 1;
+    ga.p[0] = SkinnyProblem{K, M, L.grad_split.splits, L.grad_split.steps, partA};
+    ga.p[1] = SkinnyProblem{N, M, L.grad_split.splits, L.grad_split.steps, partB};
+    ga.status = status;
+    ga.timeout_ns = timeout_ns();
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_skinny(ta0, tb0, ta1, tb1, ga, 2, st), 1, "skinny(grads)");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_reduce_lora_grads(partA, L.grad_split.splits, K, partB, L.grad_split.splits, N, NR, r, dA,
+                                          dB, st),
+                 1, "reduce(grads)");
+    return QLORA_OK;
+}
+
+qlora_status qlora_device_status(const void* ws, int* status_host, void* stream) {
+    if (!ws || !status_host) return QLORA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    QLORA_TRY(cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st), "read status");
+    QLORA_TRY(cudaStreamSynchronize(st), "sync");
+    *status_host = (v & kStatusTimeout) ? QLORA_ERR_DEVICE_TIMEOUT : (v ? QLORA_ERR_CUDA : QLORA_OK);
+    return QLORA_OK;
+}
+
+qlora_status qlora_profile_next_launch(int kernel, void* ev_start, void* ev_stop) {
+    if (kernel != QLORA_KERNEL_FUSED_FWD && kernel != QLORA_KERNEL_FUSED_DX) return QLORA_ERR_INVALID_ARG;
+    if ((ev_start == nullptr) != (ev_stop == nullptr)) return QLORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_events[kernel][0] = static_cast<cudaEvent_t>(ev_start);
+    g_prof_events[kernel][1] = static_cast<cudaEvent_t>(ev_stop);
+    return QLORA_OK;
+}
+
+qlora_status qlora_e4m3_encode(const float* x, uint8_t* q, int64_t n, void* stream) {
+    if (!x || !q) return QLORA_ERR_INVALID_ARG;
+    if (n < 0) return QLORA_ERR_BAD_SHAPE;
+    if (n == 0) return QLORA_OK;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    qlora_status s = device_ready(nullptr);
+    if (s != QLORA_OK) return s;
+    QLORA_LAUNCH(launch_e4m3_encode(x, q, n, static_cast<cudaStream_t>(stream)), 1, "e4m3_encode");
+    return QLORA_OK;
+}
+
+}  // extern "C"

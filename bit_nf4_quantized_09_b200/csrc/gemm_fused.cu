@@ -1,0 +1,294 @@
+// Dequant-fused NF4 matmuls on the sm_100 tensor core (tcgen05 + TMEM + TMA).
+//
+//   forward:  out[M, N] = X[M, K] . deq(W)[N, K]^T + sT[M, r] . B[N, r]^T
+//   dX:       out[M, K] = dY[M, N] . deq(W)[N, K]   + sU[M, r] . A[r, K]
+//
+// "ta-paperlens QLoRA explainer", section 勾配は実際どこへ行くのか: W is stored
+// in NF4 and every matmul restores the 4-bit blocks it needs to BF16 on the
+// spot; the input gradient passes through deq(W)^T. "waylandz ch.26" 26.2.4:
+// the LoRA path adds (alpha/r) B (A x); here (alpha/r) A x arrives precomputed
+// in bf16 (sT, sU) and the rank-r product runs as one extra reduction step.
+//
+// One CTA computes a 256 x 256 output tile (two M=128 UMMAs sharing each
+// dequantised weight tile, 512 TMEM columns of fp32 accumulators).
+//   warp 8      TMA producer: activation tile, packed codes, decoded constants
+//   warps 0-7   dequantisers: one 64-weight block per thread per step, written
+//               as bf16 straight into the 128-byte-swizzled UMMA operand layout
+//               (K-major for the forward, MN-major for dX); then epilogue
+//   warp 9      TMEM owner; lane 0 issues the UMMAs and commits
+// Pipelined over 3 shared-memory stages with mbarriers; every wait is bounded.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr uint32_t kActBytes = kFusedBM * kFusedBK * 2;   // 32 KB bf16
+constexpr uint32_t kWBytes = kFusedBN * kFusedBK * 2;     // 32 KB bf16
+constexpr uint32_t kCodeBytes = kFusedBN * kFusedBK / 2;  // 8 KB packed nibbles
+constexpr uint32_t kCBytes = 1024;                        // 256 decoded constants
+constexpr uint32_t kOffW = kActBytes;
+constexpr uint32_t kOffCodes = kOffW + kWBytes;
+constexpr uint32_t kOffC = kOffCodes + kCodeBytes;
+constexpr uint32_t kStageBytes = kOffC + kCBytes;  // 73 KB, a multiple of 1024
+constexpr uint32_t kBarOffset = kFusedStages * kStageBytes;
+constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;  // + barriers, + alignment slack
+constexpr uint32_t kTmemCols = 512;
+constexpr int kDequantThreads = 256;
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&v)[4]) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+
+// Dequantise one 64-weight block: 32 code bytes (two 16-byte chunks at c0, c1)
+// into eight 16-byte bf16 chunks at dst + chunk_off(j).
+template <typename ChunkOff>
+__device__ __forceinline__ void dequant_block(const Nf4Tables& tab, float cprime, uint32_t c0, uint32_t c1,
+                                              ChunkOff chunk_off) {
+    const Nf4BlockLut lut = make_block_lut(tab.level, cprime);
+    const uint4 a = lds128(c0), b = lds128(c1);
+    const uint32_t words[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+        lut_decode8(lut, words[j], o);
+        sts128(chunk_off(j), o);
+    }
+}
+
+template <bool kTransW>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+                   const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_lact,
+                   const __grid_constant__ CUtensorMap tm_lw, const FusedArgs args, const Nf4Tables tab) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+    uint64_t* deq = full + kFusedStages;
+    uint64_t* empty = deq + kFusedStages;
+    uint64_t* acc = empty + kFusedStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kFusedBM;  // first token of the tile
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kFusedBN;  // first output column
+    const int KT = static_cast<int>((args.red + kFusedBK - 1) / kFusedBK);
+    const bool has_lora = args.r > 0;
+    const int steps = KT + (has_lora ? 1 : 0);
+    const uint64_t tmo = args.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kFusedStages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(deq + s, kDequantThreads);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(acc, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tm_act);
+        tma_prefetch_desc(&tm_codes);
+        tma_prefetch_desc(&tm_c);
+        tma_prefetch_desc(&tm_lact);
+        tma_prefetch_desc(&tm_lw);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0) {
+            int last_use[kFusedStages];
+            for (int s = 0; s < kFusedStages; ++s) last_use[s] = -1;
+            if (!args.stall_producer) {
+                for (int kt = 0; kt < steps; ++kt) {
+                    const int s = kt % kFusedStages;
+                    const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
+                    if (kt >= kFusedStages && !mbar_wait(empty + s, (u - 1) & 1u, tmo, args.status)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    uint8_t* st = smem + s * kStageBytes;
+                    if (kt < KT) {
+                        mbar_arrive_expect_tx(full + s, kActBytes + kCodeBytes + kCBytes);
+                        tma_load_2d(st, &tm_act, full + s, kt * kFusedBK, static_cast<int>(m0));
+                        if (!kTransW) {
+                            // codes rows n0.., bytes of k-block kt; constants of k-block kt, rows n0..
+                            tma_load_2d(st + kOffCodes, &tm_codes, full + s, kt * (kFusedBK / 2), static_cast<int>(n0));
+                            tma_load_2d(st + kOffC, &tm_c, full + s, static_cast<int>(n0), kt);
+                        } else {
+                            // codes rows kt*64.. (reduction), bytes of columns n0..n0+255
+                            tma_load_2d(st + kOffCodes, &tm_codes, full + s, static_cast<int>(n0 / 2), kt * kFusedBK);
+                            tma_load_2d(st + kOffC, &tm_c, full + s, kt * kFusedBK, static_cast<int>(n0 / kBlock));
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(full + s, kActBytes + kWBytes);
+                        tma_load_2d(st, &tm_lact, full + s, 0, static_cast<int>(m0));
+                        if (!kTransW) {
+                            tma_load_2d(st + kOffW, &tm_lw, full + s, 0, static_cast<int>(n0));
+                        } else {
+                            for (int a = 0; a < 4; ++a)
+                                tma_load_2d(st + kOffW + a * 8192, &tm_lw, full + s, static_cast<int>(n0) + 64 * a, 0);
+                        }
+                    }
+                    last_use[s] = static_cast<int>(u);
+                }
+            }
+            // make sure no copy is still landing in shared memory at exit
+            for (int s = 0; s < kFusedStages; ++s)
+                if (last_use[s] >= 0) mbar_wait(full + s, static_cast<uint32_t>(last_use[s]) & 1u, tmo, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ----------------------------------------------------------- MMA --
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, kFusedBN, false, kTransW);
+            bool ok = true;
+            for (int kt = 0; kt < steps; ++kt) {
+                const int s = kt % kFusedStages;
+                const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
+                if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
+                if (kt < KT && !mbar_wait(deq + s, u & 1u, tmo, args.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t act = smem_u32(smem + s * kStageBytes);
+                const uint32_t wt = act + kOffW;
+                const int ksub = (kt < KT) ? (kFusedBK / 16) : (args.r + 15) / 16;
+                for (int kk = 0; kk < ksub; ++kk) {
+                    const uint64_t bdesc = kTransW ? sw128_desc(wt + kk * 2048, 8192, 1024)
+                                                   : sw128_desc(wt + kk * 32, 16, 1024);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t adesc = sw128_desc(act + h * 16384 + kk * 32, 16, 1024);
+                        umma_f16(tmem + h * 256, adesc, bdesc, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(empty + s);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                __threadfence_block();
+            }
+            umma_commit(acc);  // arrives once every issued UMMA has completed
+            mbar_wait(acc, 0, tmo, args.status);
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------- dequantise --
+        const int t = threadIdx.x;  // 0..255
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % kFusedStages;
+            const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
+            if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
+            uint8_t* st = smem + s * kStageBytes;
+            const uint32_t codes = smem_u32(st + kOffCodes);
+            const uint32_t wt = smem_u32(st + kOffW);
+            const float* cs = reinterpret_cast<const float*>(st + kOffC);
+            if (!kTransW) {
+                // row t of the weight tile, k-block kt; codes rows are 32 B, 32-byte swizzled
+                const uint32_t crow = codes + t * 32;
+                const uint32_t sw = (t >> 2) & 1;
+                const uint32_t wrow = wt + t * 128;
+                dequant_block(tab, cs[t], crow + ((0 ^ sw) << 4), crow + ((1 ^ sw) << 4),
+                              [&](int j) { return wrow + ((static_cast<uint32_t>(j) ^ (t & 7)) << 4); });
+            } else {
+                // weight row nl (reduction index), k-block a of the 4 in the tile
+                const int nl = t & 63, a = t >> 6;
+                const uint32_t crow = codes + nl * 128;
+                const uint32_t sw = nl & 7;
+                const uint32_t dst = wt + a * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+                dequant_block(tab, cs[a * 64 + nl], crow + (((2 * a) ^ sw) << 4), crow + (((2 * a + 1) ^ sw) << 4),
+                              [&](int j) { return dst + ((static_cast<uint32_t>(j) ^ sw) << 4); });
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(deq + s);
+        }
+        if (!ok) *abort_flag = 1;
+
+        // ------------------------------------------------------- epilogue --
+        const bool acc_ok = mbar_wait(acc, 0, tmo, args.status);
+        tc_fence_after();
+        if (acc_ok && !*abort_flag) {
+            const int q = warp & 3, h = warp >> 2;
+            const int64_t row = m0 + h * 128 + q * 32 + lane;
+            for (int c0 = 0; c0 < kFusedBN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c0, r);
+                tmem_ld_wait();
+                const int64_t col = n0 + c0;
+                if (row < args.M && col < args.out_cols) {
+                    uint32_t p[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        p[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                    uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.out_cols + col);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (col + 8 * i < args.out_cols)
+                            dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <bool kTransW>
+cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                         const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
+                         cudaStream_t st) {
+    dim3 grid(static_cast<unsigned>((a.out_cols + kFusedBN - 1) / kFusedBN),
+              static_cast<unsigned>((a.M + kFusedBM - 1) / kFusedBM));
+    fused_nf4_gemm<kTransW><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fused_smem_bytes() { return kSmemBytes; }
+
+cudaError_t fused_init_device() {
+    cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(fused_nf4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kSmemBytes));
+}
+
+cudaError_t launch_fused_fwd(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                             const Nf4Tables& tab, cudaStream_t st) {
+    return launch_fused<false>(act, codes, cT, lora_act, lora_w, a, tab, st);
+}
+
+cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                            const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                            const Nf4Tables& tab, cudaStream_t st) {
+    return launch_fused<true>(act, codes, cT, lora_act, lora_w, a, tab, st);
+}
+
+}  // namespace qlora

@@ -1,0 +1,101 @@
+// Host-side launchers of the library's kernels (internal to libqlora_nf4.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qlora {
+
+// ----------------------------------------------------------- quantisation --
+cudaError_t launch_nf4_encode(const float* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+                              const Nf4Tables& tab, int num_sms, cudaStream_t st);
+size_t dq_tree_scratch_doubles(int64_t nb);
+cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,
+                                float* mean, cudaStream_t st);
+cudaError_t launch_nf4_dequant(const uint8_t* codes, const uint8_t* q, const float* s2, const float* mean,
+                               int64_t N, int64_t K, uint16_t* out, const Nf4Tables& tab, int num_sms,
+                               cudaStream_t st);
+cudaError_t launch_decode_constants_t(const uint8_t* q, const float* s2, const float* mean, int64_t N, int64_t K,
+                                      int64_t ldc, float* cT, cudaStream_t st);
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* q, int64_t n, cudaStream_t st);
+
+// ------------------------------------------------------ fused NF4 GEMMs --
+// Tile of the fused kernels: 256 output rows (two M=128 MMAs) x 256 columns,
+// 64-deep reduction steps, 3 pipeline stages.
+constexpr int kFusedBM = 256;
+constexpr int kFusedBN = 256;
+constexpr int kFusedBK = 64;
+constexpr int kFusedStages = 3;
+constexpr int kFusedThreads = 320;  // 8 dequant/epilogue warps, 1 TMA warp, 1 MMA warp
+size_t fused_smem_bytes();
+cudaError_t fused_init_device();  // opt in to the large shared-memory carve-out
+
+struct FusedArgs {
+    int64_t M;          // tokens
+    int64_t out_cols;   // N (forward) or K (dX)
+    int64_t red;        // reduction length: K (forward) or N (dX)
+    int r;              // LoRA rank (extra reduction columns of the last step)
+    uint16_t* out;      // bf16 [M, out_cols]
+    int* status;        // device status word
+    uint64_t timeout_ns;
+    int stall_producer; // test hook: load nothing
+};
+
+// Forward: out = A_op . deq(W)^T + lora_a . lora_b^T, A_op = X [M, K].
+// Maps: act {K, M} box {64, 256} SW128; codes {K/2, N} box {32, 256} SW32;
+// cT {ldc, K/64} box {256, 1}; lora_act = sT {r, M} box {64, 256} SW128;
+// lora_w = B {r, N} box {64, 256} SW128.
+cudaError_t launch_fused_fwd(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                             const Nf4Tables& tab, cudaStream_t st);
+// dX: out = dY . deq(W) + sU . A.
+// Maps: act = dY {N, M} box {64, 256} SW128; codes {K/2, N} box {128, 64} SW128;
+// cT {ldc, K/64} box {64, 4}; lora_act = sU {r, M} box {64, 256} SW128;
+// lora_w = A {K, r} box {64, 64} SW128 (four boxes per step).
+cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                            const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                            const Nf4Tables& tab, cudaStream_t st);
+
+// ---------------------------------------------------------- skinny GEMMs --
+// D[rows, NR] = sum over a reduction range of A_op[rows, red] * B_op[NR, red]^T,
+// written as fp32 partials part[split][rows][NR]. Two independent problems
+// may share one launch (blockIdx.z).
+constexpr int kSkinnyStages = 4;
+constexpr int kSkinnyThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
+size_t skinny_smem_bytes();
+cudaError_t skinny_init_device();
+
+struct SkinnyProblem {
+    int64_t rows;       // output rows (tiles of 128)
+    int64_t red;        // reduction length (steps of 64)
+    int splits;         // reduction splits (grid.y)
+    int steps_per_split;
+    float* part;        // fp32 [splits][rows][NR]
+};
+
+struct SkinnyArgs {
+    int NR;             // 16, 32 or 64
+    int a_mn_major;     // A_op stored rows-contiguous (MN-major) instead of red-contiguous
+    SkinnyProblem p[2];
+    int* status;
+    uint64_t timeout_ns;
+};
+
+cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+                          const CUtensorMap& b1, const SkinnyArgs& args, int nproblems, cudaStream_t st);
+
+// out_rm[m][j] = bf16(scale * sum_s part[s][m][j]) for j < r (row-major [M, r]);
+// out_t[j * ldt + m] likewise transposed ([r, M], row pitch ldt) when out_t is not NULL.
+cudaError_t launch_reduce_lora_down(const float* part, int splits, int64_t M, int NR, int r, float scale,
+                                    uint16_t* out_rm, uint16_t* out_t, int64_t ldt, cudaStream_t st);
+// dA[j][k] = sum_s partA[s][k][j] (fp32 [r, K]); dB[n][j] = sum_s partB[s][n][j] (fp32 [N, r]).
+cudaError_t launch_reduce_lora_grads(const float* partA, int splitsA, int64_t K, const float* partB, int splitsB,
+                                     int64_t N, int NR, int r, float* dA, float* dB, cudaStream_t st);
+// out[j * ldo + n] = in[n][j]: bf16 [rows, cols] -> [cols, rows] with row pitch ldo >= rows.
+cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ldo,
+                                  cudaStream_t st);
+
+}  // namespace qlora

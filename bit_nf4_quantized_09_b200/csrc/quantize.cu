@@ -1,0 +1,309 @@
+// NF4 quantiser (blockwise absmax + nearest-level codes + nibble packing),
+// double quantisation of the absmax constants, and dequantisation.
+//
+// Sources: "ta-paperlens QLoRA explainer", sections 量子化を1段落で (c = max|x|
+// over blocks of 64; store the index of the nearest level of x/c), NF4
+// (16 normal-quantile levels, exact zero, ends +-1) and 二重量子化 (constants
+// centred by their mean, 8-bit floats in groups of 256, one fp32 per group);
+// "QLoRA" glossary (ultralytics), NF4 construction and nearest-level argmin.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+// ---------------------------------------------------------------------------
+// K1: absmax + encode + pack. Eight threads per 64-weight block, eight
+// consecutive weights per thread (two 16-byte loads), four packed bytes out.
+// Nearest level = number of decision thresholds strictly below v = w / c,
+// found by a 4-step binary search over the 15 thresholds in shared memory.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restrict__ W, int64_t nblocks,
+                                                         uint32_t* __restrict__ codes, float* __restrict__ absmax,
+                                                         Nf4Tables tab) {
+    __shared__ float sM[16];
+    if (threadIdx.x < 15) sM[threadIdx.x] = tab.thresh[threadIdx.x];
+    __syncthreads();
+
+    const int sub = threadIdx.x & 7;  // position inside the block
+    const int lane_blk = (threadIdx.x & 31) >> 3;  // which of the warp's 4 blocks
+    const int64_t warps_per_grid = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // warp-uniform loop: every lane takes part in the shuffles of every pass
+    for (int64_t bw = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * 4; bw < nblocks;
+         bw += warps_per_grid * 4) {
+        const int64_t b = bw + lane_blk;
+        const bool valid = b < nblocks;
+        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+        if (valid) {
+            x0 = __ldcs(W + b * 16 + sub * 2);
+            x1 = __ldcs(W + b * 16 + sub * 2 + 1);
+        }
+        float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float c = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c = fmaxf(c, fabsf(v[i]));
+        c = fmaxf(c, __shfl_xor_sync(0xFFFFFFFFu, c, 1));
+        c = fmaxf(c, __shfl_xor_sync(0xFFFFFFFFu, c, 2));
+        c = fmaxf(c, __shfl_xor_sync(0xFFFFFFFFu, c, 4));
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t code;
+            if (c == 0.0f) {
+                code = 7u;  // all-zero block: every element is the exact-zero level
+            } else {
+                const float q = __fdiv_rn(v[i], c);
+                int k = (q > sM[7]) ? 8 : 0;
+                k += (q > sM[k + 3]) ? 4 : 0;
+                k += (q > sM[k + 1]) ? 2 : 0;
+                k += (q > sM[k]) ? 1 : 0;
+                code = static_cast<uint32_t>(k);
+            }
+            // element 2j -> high nibble of byte j; bytes little-endian in the word
+            const int byte = i >> 1;
+            const int shift = 8 * byte + ((i & 1) ? 0 : 4);
+            word |= code << shift;
+        }
+        if (valid) {
+            __stcs(codes + b * 8 + sub, word);
+            if (sub == 0) absmax[b] = c;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K2a: fp64 sum of the constants by the stride-doubling pairwise tree.
+// Each CTA of 1024 threads reduces one aligned run of 1024 values; lane l
+// holds value l of its warp and `x += shfl_down(x, s)` for s = 1, 2, 4, 8, 16
+// leaves in lane 0 exactly the tree ((x0 + x1) + (x2 + x3)) + ...; the same
+// step then runs over the 32 warp sums. Runs of a power-of-two length nest, so
+// repeating the pass over the run sums reproduces the tree over all values
+// (zero-padded to a power of two).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double tree_sum_1024(double x, double* warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) x += __shfl_down_sync(0xFFFFFFFFu, x, s);
+    if (lane == 0) warp_sums[warp] = x;
+    __syncthreads();
+    double y = 0.0;
+    if (warp == 0) {
+        y = warp_sums[lane];
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) y += __shfl_down_sync(0xFFFFFFFFu, y, s);
+    }
+    return y;  // valid in thread 0
+}
+
+__global__ void __launch_bounds__(1024) dq_tree_pass_f32(const float* __restrict__ in, int64_t n,
+                                                          double* __restrict__ out) {
+    __shared__ double ws[32];
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
+    const double x = (i < n) ? static_cast<double>(in[i]) : 0.0;
+    const double s = tree_sum_1024(x, ws);
+    if (threadIdx.x == 0) out[blockIdx.x] = s;
+}
+
+__global__ void __launch_bounds__(1024) dq_tree_pass_f64(const double* __restrict__ in, int64_t n,
+                                                          double* __restrict__ out, int64_t count_for_mean,
+                                                          float* __restrict__ mean_out) {
+    __shared__ double ws[32];
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
+    const double x = (i < n) ? in[i] : 0.0;
+    const double s = tree_sum_1024(x, ws);
+    if (threadIdx.x == 0) {
+        out[blockIdx.x] = s;
+        if (mean_out) *mean_out = __double2float_rn(__ddiv_rn(s, static_cast<double>(count_for_mean)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K2b: one warp per group of 256 constants, eight per lane.
+// d = c - mean, s2 = max|d| / 448, code = E4M3_rn_satfinite(d / s2).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dq_groups_kernel(const float* __restrict__ c, int64_t nb,
+                                                         const float* __restrict__ mean, uint8_t* __restrict__ q,
+                                                         float* __restrict__ s2) {
+    const int lane = threadIdx.x & 31;
+    const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t ng = (nb + kGroup - 1) / kGroup;
+    if (g >= ng) return;
+    const float mu = *mean;
+    const int64_t b0 = g * kGroup + lane * 8;
+    float d[8];
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t b = b0 + i;
+        d[i] = (b < nb) ? __fsub_rn(c[b], mu) : 0.0f;
+        m = fmaxf(m, fabsf(d[i]));
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+    const float sg = __fdiv_rn(m, 448.0f);
+    if (lane == 0) s2[g] = sg;
+    uint8_t out[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        uint32_t pair = 0;
+        if (sg != 0.0f) pair = f32x2_to_e4m3x2(__fdiv_rn(d[i], sg), __fdiv_rn(d[i + 1], sg));
+        out[i] = static_cast<uint8_t>(pair & 0xFFu);
+        out[i + 1] = static_cast<uint8_t>((pair >> 8) & 0xFFu);
+    }
+    if (b0 + 8 <= nb) {
+        uint2 w;
+        w.x = out[0] | (out[1] << 8) | (out[2] << 16) | (static_cast<uint32_t>(out[3]) << 24);
+        w.y = out[4] | (out[5] << 8) | (out[6] << 16) | (static_cast<uint32_t>(out[7]) << 24);
+        *reinterpret_cast<uint2*>(q + b0) = w;
+    } else {
+        for (int i = 0; i < 8; ++i)
+            if (b0 + i < nb) q[b0 + i] = out[i];
+    }
+}
+
+// Decoded first-level constant of block b: c' = E4M3(q_b) * s2_g + mean, one
+// fp32 rounding.
+__device__ __forceinline__ float decode_constant(const uint8_t* q, const float* s2, float mu, int64_t b) {
+    return __fmaf_rn(e4m3_to_f32(q[b]), s2[b / kGroup], mu);
+}
+
+// ---------------------------------------------------------------------------
+// K3: standalone dequantisation to bf16, one 64-weight block per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4* __restrict__ codes,
+                                                           const uint8_t* __restrict__ q,
+                                                           const float* __restrict__ s2,
+                                                           const float* __restrict__ mean, int64_t nblocks,
+                                                           uint4* __restrict__ out, Nf4Tables tab) {
+    const float mu = *mean;
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
+         b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 p0 = __ldcs(codes + 2 * b);
+        const uint4 p1 = __ldcs(codes + 2 * b + 1);
+        const Nf4BlockLut lut = make_block_lut(tab.level, decode_constant(q, s2, mu, b));
+        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint32_t o[4];
+            lut_decode8(lut, words[j], o);
+            __stcs(out + 8 * b + j, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Decoded constants transposed for the matmul kernels: cT[kb * ldc + n] =
+// c' of block (n, kb), so a run of consecutive output rows n for one k-block
+// is contiguous (one TMA box). 32 x 32 tiles through shared memory.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_constants_t_kernel(const uint8_t* __restrict__ q,
+                                                                  const float* __restrict__ s2,
+                                                                  const float* __restrict__ mean, int64_t N,
+                                                                  int64_t KB, int64_t ldc,
+                                                                  float* __restrict__ cT) {
+    __shared__ float tile[32][33];
+    const float mu = *mean;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 32, kb0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    for (int i = ty; i < 32; i += 8) {
+        const int64_t n = n0 + i, kb = kb0 + tx;
+        tile[i][tx] = (n < N && kb < KB) ? decode_constant(q, s2, mu, n * KB + kb) : 0.0f;
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int64_t kb = kb0 + i, n = n0 + tx;
+        if (kb < KB && n < ldc) cT[kb * ldc + n] = (n < N) ? tile[tx][i] : 0.0f;
+    }
+}
+
+// Test hook: the double quantisation's E4M3 conversion on arbitrary floats.
+__global__ void e4m3_encode_kernel(const float* __restrict__ x, uint8_t* __restrict__ q, int64_t n) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        q[i] = static_cast<uint8_t>(f32x2_to_e4m3x2(x[i], 0.0f) & 0xFFu);
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+
+static int grid_for(int64_t work_items, int threads, int max_ctas) {
+    int64_t g = (work_items + threads - 1) / threads;
+    if (g > max_ctas) g = max_ctas;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_nf4_encode(const float* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+                              const Nf4Tables& tab, int num_sms, cudaStream_t st) {
+    const int64_t nb = N * K / kBlock;
+    const int grid = grid_for(nb * 8, 256, num_sms * 8);
+    nf4_encode_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(W), nb,
+                                            reinterpret_cast<uint32_t*>(codes), absmax, tab);
+    return cudaGetLastError();
+}
+
+size_t dq_tree_scratch_doubles(int64_t nb) {
+    // pass outputs, ping-ponged: ceil(nb/1024) + ceil(nb/1024^2) + ...
+    size_t total = 0;
+    int64_t n = nb;
+    do {
+        n = (n + 1023) / 1024;
+        total += static_cast<size_t>(n);
+    } while (n > 1);
+    return total + 1;  // + the slot of the final single-value pass
+}
+
+cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,
+                                float* mean, cudaStream_t st) {
+    // pass 1 over the fp32 constants, further passes over fp64 run sums
+    int64_t n = (nb + 1023) / 1024;
+    double* cur = tree_scratch;
+    dq_tree_pass_f32<<<static_cast<unsigned>(n), 1024, 0, st>>>(absmax, nb, cur);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (n == 1) {
+        dq_tree_pass_f64<<<1, 1024, 0, st>>>(cur, 1, cur + 1, nb, mean);
+    } else {
+        while (n > 1) {
+            const int64_t m = (n + 1023) / 1024;
+            double* nxt = cur + n;
+            dq_tree_pass_f64<<<static_cast<unsigned>(m), 1024, 0, st>>>(cur, n, nxt, nb,
+                                                                          m == 1 ? mean : nullptr);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            cur = nxt;
+            n = m;
+        }
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t ng = (nb + kGroup - 1) / kGroup;
+    dq_groups_kernel<<<static_cast<unsigned>((ng * 32 + 255) / 256), 256, 0, st>>>(absmax, nb, mean, q, s2);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nf4_dequant(const uint8_t* codes, const uint8_t* q, const float* s2, const float* mean,
+                               int64_t N, int64_t K, uint16_t* out, const Nf4Tables& tab, int num_sms,
+                               cudaStream_t st) {
+    const int64_t nb = N * K / kBlock;
+    const int grid = grid_for(nb, 256, num_sms * 8);
+    nf4_dequant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), q, s2, mean, nb,
+                                             reinterpret_cast<uint4*>(out), tab);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_constants_t(const uint8_t* q, const float* s2, const float* mean, int64_t N, int64_t K,
+                                      int64_t ldc, float* cT, cudaStream_t st) {
+    const int64_t KB = K / kBlock;
+    dim3 grid(static_cast<unsigned>((KB + 31) / 32), static_cast<unsigned>((ldc + 31) / 32));
+    decode_constants_t_kernel<<<grid, 256, 0, st>>>(q, s2, mean, N, KB, ldc, cT);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* q, int64_t n, cudaStream_t st) {
+    e4m3_encode_kernel<<<grid_for(n, 256, 4096), 256, 0, st>>>(x, q, n);
+    return cudaGetLastError();
+}
+
+}  // namespace qlora

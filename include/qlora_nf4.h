@@ -1,0 +1,186 @@
+/*
+ * qlora_nf4.h - C ABI of libqlora_nf4.so, the frozen-NF4 QLoRA linear layer
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources: the pages on QLoRA):
+ *   - "ta-paperlens QLoRA explainer" (QLoRA - 650億パラメータのモデルをGPU 1枚で
+ *     微調整する), sections 量子化を1段落で (blockwise absmax over 64 weights,
+ *     nearest of 16 levels), NF4 (normal-quantile levels, exact zero, ends +-1),
+ *     二重量子化 (absmax constants centred by their mean, stored as 8-bit floats
+ *     in groups of 256 with one fp32 constant per group), 勾配は実際どこへ行くのか
+ *     (stored NF4, computed BF16; the gradient flows through deq(W) but W gets
+ *     none; only A and B are trained);
+ *   - "QLoRA" glossary (ultralytics), the NF4 level construction and the
+ *     nearest-level argmin;
+ *   - "waylandz LLM book ch.26", 26.2.4: y = W x + (alpha/r) B (A x).
+ *
+ * Conventions
+ *   W is N x K row-major fp32 (N = out features, K = in features), K % 64 == 0.
+ *   X is M x K, Y is M x N, A is r x K, B is N x r, dY is M x N, all row-major.
+ *   bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   s = alpha / r.
+ *   Every pointer argument is a DEVICE pointer unless it says "host".
+ *   The caller allocates and frees every buffer (the library never allocates
+ *   device memory); `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   Calls are asynchronous and stream-ordered. A return value of QLORA_OK means
+ *   the arguments were valid and every kernel was launched; errors found by
+ *   the device itself (a pipeline wait that ran out) are recorded in the
+ *   workspace's status word, read back with qlora_device_status().
+ *   Device buffers must be 16-byte aligned.
+ *
+ * Quantised weight format (qlora_nf4_weight), for nb = N*K/64 blocks and
+ * ng = ceil(nb/256) groups:
+ *   codes   uint8[N*K/2]  flat row-major element 2j in the HIGH nibble of byte j,
+ *                         element 2j+1 in the low nibble; code = index of the
+ *                         nearest NF4 level (0 = -1, 7 = 0, 15 = +1)
+ *   qabsmax uint8[nb]     OCP FP8 E4M3 code of (absmax_b - mean) / s2_g
+ *   s2      float[ng]     second-level constant of group g (blocks 256g..256g+255)
+ *   mean    float[1]      mean of all first-level absmax constants
+ *   Dequantised weight: c'_b = fmaf(E4M3(qabsmax_b), s2_g, mean) (one fp32
+ *   rounding), w_hat = bf16_rn(fp32_rn(level[code] * c'_b)).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int qlora_status;
+
+#define QLORA_OK                        0
+#define QLORA_ERR_INVALID_ARG          -1  /* NULL pointer, alpha not finite, bad op   */
+#define QLORA_ERR_BAD_SHAPE            -2  /* K % 64 != 0, N*K == 0, N % 8 != 0, M < 0 */
+#define QLORA_ERR_MISALIGNED           -3  /* a device pointer not 16-byte aligned     */
+#define QLORA_ERR_UNSUPPORTED_RANK     -4  /* r not in {8, 16, 32, 64}                 */
+#define QLORA_ERR_WORKSPACE_TOO_SMALL  -5  /* ws_bytes < qlora_workspace_bytes(...)    */
+#define QLORA_ERR_CUDA                 -6  /* a CUDA call or launch failed; see
+                                              qlora_last_error()                        */
+#define QLORA_ERR_DEVICE_TIMEOUT       -7  /* device status: a pipeline wait ran out   */
+#define QLORA_ERR_UNSUPPORTED_DEVICE   -8  /* current device is not sm_100             */
+
+/* Read-only view of a quantised weight. All five pointers are device
+ * pointers owned by the caller; the library never writes through them. */
+typedef struct {
+    const uint8_t* codes;
+    const uint8_t* qabsmax;
+    const float*   s2;
+    const float*   mean;
+    int64_t        N;
+    int64_t        K;
+} qlora_nf4_weight;
+
+/* Sizes in bytes of the four buffers of an N x K quantised weight. Host only;
+ * any out-pointer may be NULL. Returns their sum, or -1 for a bad shape.
+ * 8 * sum / (N*K) = 4 + 8/64 + 32/(64*256) + 32/(N*K) bits per weight, the
+ * 4.127 of the explainer's 二重量子化 section. */
+int64_t qlora_nf4_bytes(int64_t N, int64_t K, size_t* codes, size_t* qabsmax,
+                        size_t* s2, size_t* mean);
+
+/* Workspace (device scratch, caller-allocated) needed by one call. */
+#define QLORA_OP_QUANTIZE 0
+#define QLORA_OP_FWD      1
+#define QLORA_OP_BWD      2
+/* Returns the byte count, or 0 for an invalid op/shape. Host only. */
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
+
+/* Quantise W (fp32 [N, K], device) to NF4 with double quantisation.
+ * [explainer 量子化を1段落で + NF4 + 二重量子化; glossary NF4 snippet]
+ * Per 64-block: absmax c (fp32), v = w / c (IEEE fp32 division), code = number
+ * of decision thresholds below v (exactly the nearest level, ties to the lower
+ * index; a block with c == 0 codes every element 7). Then mean = fp32 of the
+ * fp64 pairwise-tree sum of all c divided by nb; per group of 256 blocks
+ * d = c - mean, s2 = max|d| / 448, qabsmax = E4M3_rn_satfinite(d / s2)
+ * (0x00 when s2 == 0).
+ * Outputs codes/qabsmax/s2/mean are device buffers sized by qlora_nf4_bytes;
+ * ws needs qlora_workspace_bytes(QLORA_OP_QUANTIZE, 0, N, K, 0) bytes.
+ * Deterministic: the same W always gives the same bits. */
+qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K,
+                                uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Dequantise to bf16 [N, K] (device W_out), bit-exact with the format's
+ * definition above. [explainer 量子化を1段落で: x_hat = c * level[code]] */
+qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream);
+
+/* Forward of the QLoRA linear layer [waylandz 26.2.4; explainer 勾配は...]:
+ *   sT = bf16( s * X A^T )                    (M x r, written to sT_save if not NULL)
+ *   Y  = bf16( X deq(W)^T + sT B^T )           (M x N)
+ * The NF4 weight is dequantised tile by tile inside the matmul (no bf16 copy
+ * of W is ever written to memory). X: bf16 [M, K]; A: bf16 [r, K];
+ * B: bf16 [N, r]; r in {8, 16, 32, 64}; M >= 0 (M == 0 is a no-op).
+ * ws needs qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r) bytes. */
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                              const uint16_t* A, const uint16_t* B, int r, float alpha,
+                              uint16_t* Y, uint16_t* sT_save,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of the layer, gradients of <dY, Y> [explainer 勾配は実際どこへ行くのか:
+ * the input gradient needs deq(W)^T; W itself gets no gradient]:
+ *   sU = bf16( s * dY B )                      (M x r)
+ *   dX = bf16( dY deq(W) + sU A )               (M x K)
+ *   dA = fp32( sU^T X )      = s (dY B)^T X     (r x K, overwritten)
+ *   dB = fp32( dY^T sT )     = s dY^T (X A^T)   (N x r, overwritten)
+ * sT is the forward's sT_save (bf16 [M, r]) or NULL to recompute it.
+ * ws needs qlora_workspace_bytes(QLORA_OP_BWD, M, N, K, r) bytes. */
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M,
+                              const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
+                              int r, float alpha, const uint16_t* sT,
+                              uint16_t* dX, float* dA, float* dB,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* Host copies of the library's own NF4 tables: levels[16] (fp32, ascending)
+ * and thresholds[15] (the fp32 decision points between neighbouring levels).
+ * Computed on the host at load time, independently of any test code. */
+qlora_status qlora_nf4_tables(float* levels_host, float* thresholds_host);
+
+/* Read the device status word at the head of a fwd/bwd workspace (0 = ok,
+ * otherwise a QLORA_ERR_DEVICE_* code). Synchronises `stream`. */
+qlora_status qlora_device_status(const void* ws, int* status_host, void* stream);
+
+/* Human-readable name of a status code, and the text of the last CUDA error
+ * seen by this thread (empty if none). Host only; static strings. */
+const char* qlora_status_string(qlora_status s);
+const char* qlora_last_error(void);
+
+/* Test and tuning hooks (not needed for normal use).
+ *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses the
+ *                           small-batch dequant-GEMV kernel (default 64;
+ *                           -1 forces the tiled GEMM for every M)
+ *   QLORA_OPT_FAIL_LAUNCHES the next `value` kernel launches report
+ *                           QLORA_ERR_CUDA without launching (host-side fault
+ *                           injection; nothing reaches the GPU)
+ *   QLORA_OPT_WAIT_TIMEOUT_US per-wait limit of the pipelined kernels' barrier
+ *                           waits in microseconds (default 1000000)
+ *   QLORA_OPT_STALL_PRODUCER 1 = the next forward's tiled GEMM loads nothing,
+ *                           so its consumers' waits run out and the device
+ *                           status reports QLORA_ERR_DEVICE_TIMEOUT */
+#define QLORA_OPT_SMALL_M_MAX     1
+#define QLORA_OPT_FAIL_LAUNCHES   2
+#define QLORA_OPT_WAIT_TIMEOUT_US 3
+#define QLORA_OPT_STALL_PRODUCER  4
+#define QLORA_OPT_LAUNCH_COUNT    5  /* read: kernels launched by this library so
+                                        far in this process; set: reset to value */
+qlora_status qlora_set_option(int option, int64_t value);
+int64_t qlora_get_option(int option);
+
+/* Profiling hook: record the CUDA events ev_start / ev_stop (cudaEvent_t,
+ * owned by the caller) on the launch stream immediately before and after the
+ * next launch of the named kernel; the request is consumed by that launch. */
+#define QLORA_KERNEL_FUSED_FWD 1   /* the dequant-fused forward matmul       */
+#define QLORA_KERNEL_FUSED_DX  2   /* the transposed-dequant dX matmul       */
+qlora_status qlora_profile_next_launch(int kernel, void* ev_start, void* ev_stop);
+
+/* Test hook: E4M3 round-to-nearest-even with saturation, exactly as the
+ * double quantisation stores constants (the sm_100 cvt instruction), on n
+ * device floats. */
+qlora_status qlora_e4m3_encode(const float* x, uint8_t* q, int64_t n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

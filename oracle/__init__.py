@@ -48,6 +48,7 @@ def lib():
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
         L.oracle_dq_mean.restype = ctypes.c_float
         L.oracle_dq_mean.argtypes = [_f32p, _i64, _f64p]
         L.oracle_double_quant.argtypes = [_f32p, _i64, _u8p, _f32p, _f32p]
@@ -136,6 +137,13 @@ def e4m3_decode(q: int) -> float:
 
 def e4m3_encode(x: float) -> int:
     return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def e4m3_encode_array(x) -> np.ndarray:
+    x = _f32(x).reshape(-1)
+    q = np.zeros(x.size, np.uint8)
+    lib().oracle_e4m3_encode_array(_p(x, _f32p), x.size, _p(q, _u8p))
+    return q
 
 
 # --------------------------------------------------------- double quant ----

@@ -367,3 +367,12 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* The E4M3 encoder above, applied to an array (for wide sweeps in tests). */
+void oracle_e4m3_encode_array(const float* x, int64_t n, uint8_t* q)
+{
+    double vals[127];
+    e4m3_values(vals);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) q[i] = e4m3_nearest(x[i], vals);
+}

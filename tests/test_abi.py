@@ -1,0 +1,142 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, sizes its buffers as the format says, and rejects bad
+arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def q():
+    from bit_nf4_quantized_09_b200 import build
+    build.build()
+    import bit_nf4_quantized_09_b200 as q
+    return q
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(q):
+    L = ctypes.CDLL(q.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(L, name), name
+    # and the binding knows every one of them under the same name
+    assert set(names) == set(q._SIGNATURES)
+
+
+def test_nf4_bytes_match_oracle_storage(q):
+    for N, K in [(512, 512), (4096, 4096), (11008, 4096), (8192, 22016), (8, 64)]:
+        sz = q.nf4_bytes(N, K)
+        assert sz["codes"] == N * K // 2
+        assert sz["qabsmax"] == N * K // 64
+        assert sz["s2"] == 4 * ((N * K // 64 + 255) // 256)
+        assert sz["mean"] == 4
+        assert sz["total"] == oracle.storage_bytes(N, K, True)
+    with pytest.raises(q.QLoraError):
+        q.nf4_bytes(4, 100)
+
+
+def test_library_tables_equal_oracle_bit_for_bit(q):
+    """The library computes the NF4 levels and thresholds on its own (Newton
+    on the normal CDF); the oracle by bisection. Same fp32 bits."""
+    lv, th = q.nf4_tables()
+    _, L = oracle.nf4_levels()
+    M = oracle.midpoints(L)
+    assert np.array_equal(np.array(lv, np.float32).view(np.uint32), L.view(np.uint32))
+    assert np.array_equal(np.array(th, np.float32).view(np.uint32), M.view(np.uint32))
+
+
+def test_workspace_sizes(q):
+    assert q.workspace_bytes(q.OP_QUANTIZE, 0, 512, 512, 0) >= 512 * 512 // 64 * 4
+    assert q.workspace_bytes(q.OP_FWD, 64, 512, 512, 8) > 0
+    assert q.workspace_bytes(q.OP_BWD, 4096, 4096, 4096, 16) > q.workspace_bytes(q.OP_FWD, 4096, 4096, 4096, 16)
+    assert q.workspace_bytes(q.OP_FWD, 64, 512, 500, 8) == 0      # K % 64
+    assert q.workspace_bytes(q.OP_FWD, 64, 512, 512, 12) == 0     # rank
+    assert q.workspace_bytes(7, 64, 512, 512, 8) == 0             # op
+
+
+def _weight(q, N=512, K=512, base=0x10000):
+    return q.Nf4WeightC(base, base + 0x100000, base + 0x200000, base + 0x300000, N, K)
+
+
+def test_host_validation_without_gpu(q):
+    L = q.lib()
+    w = _weight(q)
+    P = 0x7000000  # fake, 16-byte aligned; never dereferenced on these paths
+    ws_ok = q.workspace_bytes(q.OP_FWD, 64, 512, 512, 8)
+    fwd = lambda **kw: L.qlora_linear_fwd(kw.get("X", P), kw.get("M", 64), ctypes.byref(kw.get("w", w)),
+                                          kw.get("A", P), kw.get("B", P), kw.get("r", 8), kw.get("alpha", 16.0),
+                                          kw.get("Y", P), None, kw.get("ws", P), kw.get("wsb", 0), None)
+    assert fwd(r=12) == -4
+    assert fwd(r=0) == -4
+    assert fwd(X=None) == -1
+    assert fwd(alpha=float("nan")) == -1
+    assert fwd(X=P + 2) == -3
+    assert fwd(M=-1) == -2
+    assert fwd(M=0) == 0                       # empty batch: valid no-op, nothing launched
+    assert fwd(w=_weight(q, K=500)) == -2       # K % 64 != 0
+    assert fwd(w=_weight(q, N=12)) == -2        # N % 8 != 0
+    assert fwd(w=_weight(q, base=0x10004)) == -3
+    assert fwd(wsb=ws_ok - 1) == -5
+    # quantize
+    assert L.qlora_quantize_nf4(P, 512, 500, P, P, P, P, P, 1 << 30, None) == -2
+    assert L.qlora_quantize_nf4(P, 0, 512, P, P, P, P, P, 1 << 30, None) == -2
+    assert L.qlora_quantize_nf4(None, 512, 512, P, P, P, P, P, 1 << 30, None) == -1
+    assert L.qlora_quantize_nf4(P, 512, 512, P, P, P, P, P, 16, None) == -5
+    # dequantize
+    assert L.qlora_dequantize_nf4(ctypes.byref(w), None, None) == -1
+    assert L.qlora_dequantize_nf4(ctypes.byref(w), P + 8, None) == -3
+    # backward
+    bws = q.workspace_bytes(q.OP_BWD, 64, 512, 512, 8)
+    bwd = lambda **kw: L.qlora_linear_bwd(P, P, kw.get("M", 64), ctypes.byref(w), P, P, kw.get("r", 8), 16.0,
+                                          None, P, kw.get("dA", P), P, P, kw.get("wsb", bws), None)
+    assert bwd(r=24) == -4
+    assert bwd(dA=None) == -1
+    assert bwd(dA=P + 4) == -3
+    assert bwd(wsb=bws - 256) == -5
+
+
+def test_host_fault_injection(q):
+    """An injected launch failure is reported as QLORA_ERR_CUDA with its text,
+    and nothing reaches a GPU (none is needed for this test)."""
+    L = q.lib()
+    w = _weight(q)
+    P = 0x7000000
+    ws = q.workspace_bytes(q.OP_FWD, 64, 512, 512, 8)
+    q.set_option(q.OPT_FAIL_LAUNCHES, 1)
+    try:
+        s = L.qlora_linear_fwd(P, 64, ctypes.byref(w), P, P, 8, 16.0, P, None, P, ws, None)
+        assert s == -6
+        assert b"injected" in L.qlora_last_error()
+        assert q.get_option(q.OPT_FAIL_LAUNCHES) == 0
+    finally:
+        q.set_option(q.OPT_FAIL_LAUNCHES, 0)
+
+
+def test_status_strings_and_options(q):
+    L = q.lib()
+    for code, name in q.STATUS.items():
+        assert L.qlora_status_string(code).decode() == name
+    assert L.qlora_status_string(-99).decode() == "QLORA_ERR_UNKNOWN"
+    old = q.get_option(q.OPT_WAIT_TIMEOUT_US)
+    q.set_option(q.OPT_WAIT_TIMEOUT_US, 5000)
+    assert q.get_option(q.OPT_WAIT_TIMEOUT_US) == 5000
+    q.set_option(q.OPT_WAIT_TIMEOUT_US, old)
+    with pytest.raises(q.QLoraError):
+        q.set_option(q.OPT_WAIT_TIMEOUT_US, 0)
+    with pytest.raises(q.QLoraError):
+        q.set_option(99, 1)

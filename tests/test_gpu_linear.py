@@ -1,0 +1,170 @@
+"""GPU forward/backward of the QLoRA linear layer vs the fp64 CPU oracle.
+
+Tolerance (the stated bar for forward/backward outputs): for each output
+tensor, max |gpu - ref| / max |ref| <= 1e-2, where ref is computed in fp64
+from the oracle's own dequantised weight and the same bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def q():
+    from bit_nf4_quantized_09_b200 import build
+    build.build()
+    import bit_nf4_quantized_09_b200 as q
+    assert torch.cuda.is_available()
+    return q
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def inputs(cfg):
+    return dict(W=synth.weight(cfg), X=synth.activations(cfg), A=synth.lora_a(cfg), B=synth.lora_b(cfg),
+                dY=synth.grad_output(cfg))
+
+
+def gpu_run(q, cfg, t, alpha=None, sT_saved=True):
+    alpha = cfg.alpha if alpha is None else alpha
+    w = q.quantize_nf4(t["W"].cuda())
+    X, A, B, dY = (t[k].cuda() for k in ("X", "A", "B", "dY"))
+    Y, sT = q.linear_fwd(X, w, A, B, alpha)
+    dX, dA, dB = q.linear_bwd(dY, X, w, A, B, alpha, sT if sT_saved else None)
+    torch.cuda.synchronize()
+    return dict(Y=Y, sT=sT, dX=dX, dA=dA, dB=dB, w=w)
+
+
+def oracle_what(W: torch.Tensor) -> np.ndarray:
+    z = oracle.quantize_nf4(W.numpy())
+    bits = oracle.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], z["N"], z["K"])
+    return oracle.bf16_bits_to_f64(bits)
+
+
+def check(name, got, ref, tol=TOL):
+    e = oracle.rel_err(got, ref)
+    print(f"{name}: max|err|/max|ref| = {e:.3e}")
+    assert e <= tol, (name, e)
+    return e
+
+
+def full_compare(q, cfg, t=None, alpha=None):
+    t = t or inputs(cfg)
+    alpha = cfg.alpha if alpha is None else alpha
+    g = gpu_run(q, cfg, t, alpha)
+    What = oracle_what(t["W"])
+    X, A, B, dY = (f64(t[k]) for k in ("X", "A", "B", "dY"))
+    Y, T = oracle.forward(X, What, A, B, alpha, cfg.r)
+    dX, dA, dB = oracle.backward(dY, X, What, A, B, alpha, cfg.r)
+    errs = dict(Y=check("Y", f64(g["Y"]), Y), sT=check("sT", f64(g["sT"]), (alpha / cfg.r) * T),
+                dX=check("dX", f64(g["dX"]), dX), dA=check("dA", f64(g["dA"]), dA),
+                dB=check("dB", f64(g["dB"]), dB))
+    return g, errs
+
+
+def test_tiny_config(q):
+    full_compare(q, synth.TINY)
+
+
+RAGGED = [synth.custom(N=520, K=320, M=100, r=8), synth.custom(N=264, K=640, M=300, r=16),
+          synth.custom(N=512, K=512, M=1, r=32), synth.custom(N=1024, K=256, M=257, r=64),
+          synth.custom(N=776, K=1088, M=513, r=16, outliers=True), synth.custom(N=8, K=64, M=3, r=8)]
+
+
+@pytest.mark.parametrize("cfg", RAGGED, ids=lambda c: c.name)
+def test_ragged_shapes(q, cfg):
+    full_compare(q, cfg)
+
+
+FULL = [synth.ATTN7B, synth.MLP7B[0], synth.MLP7B[2], synth.L65B[0], synth.L65B[1], synth.L65B[2]]
+
+
+@pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
+def test_full_size_sampled(q, cfg):
+    """Full-size run in the benchmark's launch configuration; Y and dX are
+    checked on 48 sampled tokens (first, last and random), dA and dB in full
+    (they need every token but not the weight)."""
+    t = inputs(cfg)
+    g = gpu_run(q, cfg, t)
+    rng = np.random.default_rng(cfg.config_index * 31 + cfg.layer_id)
+    rows = np.unique(np.concatenate([[0, cfg.M - 1], rng.choice(cfg.M, 46, replace=False)]))
+    What = oracle_what(t["W"])
+    X, A, B, dY = (f64(t[k]) for k in ("X", "A", "B", "dY"))
+    Ys, _ = oracle.forward(X[rows], What, A, B, cfg.alpha, cfg.r)
+    dXs, _, _ = oracle.backward(dY[rows], X[rows], What, A, B, cfg.alpha, cfg.r)
+    del What
+    s = cfg.alpha / cfg.r
+    U = dY @ B
+    dA = s * (U.T @ X)
+    dB = s * (dY.T @ (X @ A.T))
+    check("Y[rows]", f64(g["Y"])[rows], Ys)
+    check("dX[rows]", f64(g["dX"])[rows], dXs)
+    check("dA", f64(g["dA"]), dA)
+    check("dB", f64(g["dB"]), dB)
+
+
+def test_zero_b_is_the_base_layer(q):
+    """waylandz 26.2.3: with B = 0 the layer is exactly W. The LoRA step then
+    adds exact zeros, so Y does not depend on A bit for bit, dA is exactly 0,
+    and Y matches X deq(W)^T."""
+    cfg = synth.custom(N=512, K=512, M=200, r=16)
+    t = inputs(cfg)
+    t["B"] = torch.zeros_like(t["B"])
+    g1 = gpu_run(q, cfg, t)
+    t2 = dict(t, A=synth.lora_a(synth.custom(N=512, K=512, M=200, r=16, seed_base=91)))
+    g2 = gpu_run(q, cfg, t2)
+    assert torch.equal(g1["Y"].view(torch.int16), g2["Y"].view(torch.int16))
+    assert torch.count_nonzero(g1["dA"]) == 0
+    What = oracle_what(t["W"])
+    check("Y", f64(g1["Y"]), f64(t["X"]) @ What.T)
+    check("dX", f64(g1["dX"]), f64(t["dY"]) @ What)
+
+
+def test_alpha_zero_equals_zero_b(q):
+    cfg = synth.custom(N=264, K=320, M=77, r=8)
+    t = inputs(cfg)
+    a = gpu_run(q, cfg, t, alpha=0.0)
+    t0 = dict(t, B=torch.zeros_like(t["B"]))
+    b = gpu_run(q, cfg, t0)
+    assert torch.equal(a["Y"].view(torch.int16), b["Y"].view(torch.int16))
+
+
+def test_backward_recomputes_sT(q):
+    cfg = synth.custom(N=512, K=448, M=130, r=32)
+    t = inputs(cfg)
+    a = gpu_run(q, cfg, t, sT_saved=True)
+    b = gpu_run(q, cfg, t, sT_saved=False)
+    for k in ("dX", "dA", "dB"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_empty_batch(q):
+    cfg = synth.custom(N=512, K=512, M=4, r=8)
+    t = inputs(cfg)
+    w = q.quantize_nf4(t["W"].cuda())
+    X = torch.empty(0, 512, dtype=torch.bfloat16, device="cuda")
+    Y, sT = q.linear_fwd(X, w, t["A"].cuda(), t["B"].cuda(), 16.0)
+    assert Y.shape == (0, 512)
+    dA = torch.full((8, 512), 7.0, device="cuda")
+    dB = torch.full((512, 8), 7.0, device="cuda")
+    q.linear_bwd(torch.empty(0, 512, dtype=torch.bfloat16, device="cuda"), X, w, t["A"].cuda(), t["B"].cuda(),
+                 16.0, None, dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
+
+
+def test_forward_backward_deterministic(q):
+    cfg = synth.custom(N=1024, K=1024, M=600, r=16)
+    t = inputs(cfg)
+    a = gpu_run(q, cfg, t)
+    b = gpu_run(q, cfg, t)
+    for k in ("Y", "dX", "dA", "dB"):
+        assert torch.equal(a[k], b[k]), k
