@@ -76,18 +76,18 @@ class ClockSampler:
 
     def __init__(self, device: int):
         self.proc = None
+        target = str(device)
         try:
-            target = str(device)
-            try:
-                bus = torch.cuda.get_device_properties(device).pci_bus_id
-                if bus:
-                    target = bus
-            except AttributeError:
-                pass
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if uuid:
+                target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:  # noqa: BLE001 - fall back to the ordinal
+            pass
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "100", "-i", target], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
-        except (OSError, RuntimeError):
+        except (OSError, ValueError, TypeError):
             self.proc = None
 
     def stop(self):
@@ -265,6 +265,10 @@ def run_ours(args, rank, world, local_rank):
     # ---- timed region: K whole steps, events around each fused matmul too
     prof = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
             for _ in range(args.steps)]
+    for pair in prof:  # torch creates events lazily: make them exist before the library records them
+        for a, b in pair:
+            a.record()
+            b.record()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = q.launch_count()
     sampler = ClockSampler(local_rank)

@@ -19,7 +19,7 @@ using namespace qlora;
 namespace {
 
 // ------------------------------------------------------------ options ----
-std::atomic<int64_t> g_small_m_max{-1};
+std::atomic<int64_t> g_small_m_max{kGemvMaxM};
 std::atomic<int64_t> g_fail_launches{0};
 std::atomic<int64_t> g_timeout_us{1000000};
 std::atomic<int64_t> g_stall_producer{0};
@@ -154,7 +154,8 @@ qlora_status device_ready(int* sms_out) {
             g_last_error = "device is not sm_100 (compute capability " + std::to_string(major) + "." +
                            std::to_string(minor) + ")";
             d.status = QLORA_ERR_UNSUPPORTED_DEVICE;
-        } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess) {
+        } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess ||
+                   (e = gemv_init_device()) != cudaSuccess) {
             d.status = cuda_fail(e, "cudaFuncSetAttribute");
         } else if (!g_encode) {
             void* fn = nullptr;
@@ -215,14 +216,35 @@ Split split_for(int64_t tiles, int64_t red) {
     return Split{static_cast<int>(s), static_cast<int>(steps)};
 }
 
+// K splits of the small-batch kernel: at most two waves of two CTAs per SM
+// (on 148 SMs), the best wave fill, and fp32 partials no larger than a
+// quarter of the packed weight.
+Split gemv_split(int64_t M, int64_t N, int64_t K) {
+    const int64_t KT = K / 64, tiles = cdiv(N, 128), slots = kTargetCtas;
+    const int64_t smax = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(KT, 64), K / (32 * std::max<int64_t>(M, 1))));
+    int64_t best = 1;
+    double best_eff = -1.0;
+    for (int64_t s = 1; s <= smax; ++s) {
+        const int64_t units = tiles * s;
+        if (s > 1 && units > 2 * slots) break;
+        const double eff = static_cast<double>(units) / static_cast<double>(cdiv(units, slots) * slots);
+        if (eff > best_eff + 1e-9) {
+            best = s;
+            best_eff = eff;
+        }
+    }
+    const int64_t steps = cdiv(KT, best);
+    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
+}
+
 // ------------------------------------------------------- workspace layout --
 struct Layout {
     size_t status = 0, cT = 0, partT = 0, sT = 0;         // forward
     size_t Bt = 0, partU = 0, sU = 0, sUt = 0, sTt = 0;    // backward
-    size_t partA = 0, partB = 0;
+    size_t partA = 0, partB = 0, partY = 0;
     size_t total = 0;
     int64_t ldc = 0, ldt = 0;
-    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1};
+    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1}, gemv{1, 1};
 };
 
 Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
@@ -243,6 +265,10 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     if (op == QLORA_OP_FWD) {
         L.partT = take(static_cast<size_t>(L.sT_split.splits) * M * NR * 4);
         L.sT = take(static_cast<size_t>(M) * r * 2);
+        if (M <= kGemvMaxM) {
+            L.gemv = gemv_split(M, N, K);
+            L.partY = take(static_cast<size_t>(L.gemv.splits) * M * N * 4);
+        }
     } else {
         L.sU_split = split_for(mtiles, N);
         L.grad_split = split_for(cdiv(K, 128) + cdiv(N, 128), M);
@@ -438,6 +464,37 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
     if ((s = lora_down(X, M, K, A, r, scale, L.sT_split, partT, sT, nullptr, 0, status, st)) != QLORA_OK) return s;
+
+    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
+    if (M <= small) {
+        // few tokens: weight-streaming swap-AB kernel, split over K
+        const int Mp = static_cast<int>((M + 15) / 16 * 16);
+        CUtensorMap t_x, t_codes, t_c;
+        QLORA_MAP(&t_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, Mp, CU_TENSOR_MAP_SWIZZLE_128B, "X");
+        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_32B, "codes");
+        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
+        GemvArgs ga{};
+        ga.M = M;
+        ga.N = N;
+        ga.K = K;
+        ga.Mp = Mp;
+        ga.splits = L.gemv.splits;
+        ga.steps_per_split = L.gemv.steps;
+        ga.part = reinterpret_cast<float*>(base + L.partY);
+        ga.status = status;
+        ga.timeout_ns = timeout_ns();
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        cudaEvent_t ev0, ev1;
+        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+        if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+        QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
+        if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        QLORA_LAUNCH(launch_gemv_reduce(ga.part, ga.splits, M, N, sT, B, r, Y, st), 1, "gemv reduce");
+        return QLORA_OK;
+    }
 
     CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
     QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");

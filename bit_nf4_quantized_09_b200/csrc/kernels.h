@@ -59,6 +59,31 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
                             const Nf4Tables& tab, cudaStream_t st);
 
+// ------------------------------------------------ small-batch dequant GEMV --
+constexpr int kGemvStages = 3;
+constexpr int kGemvThreads = 192;  // 4 dequant/epilogue warps, TMA warp, MMA warp
+constexpr int kGemvMaxM = 64;      // tokens that fit the UMMA N side of one tile
+size_t gemv_smem_bytes();
+cudaError_t gemv_init_device();
+
+struct GemvArgs {
+    int64_t M, N, K;
+    int Mp;              // M rounded up to a multiple of 16
+    int splits;          // K splits (grid.y)
+    int steps_per_split;
+    float* part;         // fp32 [splits][M][N]
+    int* status;
+    uint64_t timeout_ns;
+};
+
+// Maps: x = X {K, M} box {64, Mp} SW128; codes {K/2, N} box {32, 128} SW32;
+// cT {ldc, K/64} box {128, 1}.
+cudaError_t launch_gemv(const CUtensorMap& x, const CUtensorMap& codes, const CUtensorMap& cT, const GemvArgs& a,
+                        const Nf4Tables& tab, cudaStream_t st);
+// Y[m][n] = bf16(sum_s part[s][m][n] + sum_j sT[m][j] B[n][j]).
+cudaError_t launch_gemv_reduce(const float* part, int splits, int64_t M, int64_t N, const uint16_t* sT,
+                               const uint16_t* B, int r, uint16_t* Y, cudaStream_t st);
+
 // ---------------------------------------------------------- skinny GEMMs --
 // D[rows, NR] = sum over a reduction range of A_op[rows, red] * B_op[NR, red]^T,
 // written as fp32 partials part[split][rows][NR]. Two independent problems

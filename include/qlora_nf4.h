@@ -148,8 +148,8 @@ const char* qlora_last_error(void);
 
 /* Test and tuning hooks (not needed for normal use).
  *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses the
- *                           small-batch dequant-GEMV kernel (default 64;
- *                           -1 forces the tiled GEMM for every M)
+ *                           small-batch dequant-GEMV kernel (default and
+ *                           maximum 64; 0 forces the tiled GEMM for every M)
  *   QLORA_OPT_FAIL_LAUNCHES the next `value` kernel launches report
  *                           QLORA_ERR_CUDA without launching (host-side fault
  *                           injection; nothing reaches the GPU)
@@ -170,7 +170,8 @@ int64_t qlora_get_option(int option);
 /* Profiling hook: record the CUDA events ev_start / ev_stop (cudaEvent_t,
  * owned by the caller) on the launch stream immediately before and after the
  * next launch of the named kernel; the request is consumed by that launch. */
-#define QLORA_KERNEL_FUSED_FWD 1   /* the dequant-fused forward matmul       */
+#define QLORA_KERNEL_FUSED_FWD 1   /* the dequant-fused forward matmul (the
+                                      small-batch kernel when M <= 64)        */
 #define QLORA_KERNEL_FUSED_DX  2   /* the transposed-dequant dX matmul       */
 qlora_status qlora_profile_next_launch(int kernel, void* ev_start, void* ev_stop);
 

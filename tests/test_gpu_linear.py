@@ -168,3 +168,48 @@ def test_forward_backward_deterministic(q):
     b = gpu_run(q, cfg, t)
     for k in ("Y", "dX", "dA", "dB"):
         assert torch.equal(a[k], b[k]), k
+
+
+# ------------------------------------------------- small-batch (M <= 64) ---
+
+@pytest.mark.parametrize("cfg", synth.SWEEP, ids=lambda c: c.name)
+def test_small_batch_sweep_forward(q, cfg):
+    """The memory-bound sweep (M in {1, 4, 16, 64}), forward only: every
+    output row against the fp64 oracle."""
+    t = inputs(cfg)
+    w = q.quantize_nf4(t["W"].cuda())
+    Y, sT = q.linear_fwd(t["X"].cuda(), w, t["A"].cuda(), t["B"].cuda(), cfg.alpha)
+    torch.cuda.synchronize()
+    What = oracle_what(t["W"])
+    Yr, T = oracle.forward(f64(t["X"]), What, f64(t["A"]), f64(t["B"]), cfg.alpha, cfg.r)
+    check("Y", f64(Y), Yr)
+    check("sT", f64(sT), (cfg.alpha / cfg.r) * T)
+
+
+SMALL = [synth.custom(N=520, K=320, M=3, r=8), synth.custom(N=1024, K=576, M=17, r=64),
+         synth.custom(N=264, K=64, M=64, r=32), synth.custom(N=2048, K=1024, M=1, r=16, outliers=True)]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_batch_ragged(q, cfg):
+    full_compare(q, cfg)
+
+
+def test_small_batch_matches_tiled_path(q):
+    """The same forward through the small-batch kernel and through the tiled
+    256 x 256 kernel (forced by QLORA_OPT_SMALL_M_MAX = 0)."""
+    cfg = synth.custom(N=4096, K=2048, M=48, r=16)
+    t = inputs(cfg)
+    w = q.quantize_nf4(t["W"].cuda())
+    args = (t["X"].cuda(), w, t["A"].cuda(), t["B"].cuda(), cfg.alpha)
+    Ys, _ = q.linear_fwd(*args)
+    old = q.get_option(q.OPT_SMALL_M_MAX)
+    try:
+        q.set_option(q.OPT_SMALL_M_MAX, 0)
+        Yt, _ = q.linear_fwd(*args)
+    finally:
+        q.set_option(q.OPT_SMALL_M_MAX, old)
+    torch.cuda.synchronize()
+    e = oracle.rel_err(f64(Ys), f64(Yt))
+    print(f"small-batch vs tiled: {e:.3e}")
+    assert e <= 2 ** -7
