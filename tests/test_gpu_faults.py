@@ -18,7 +18,7 @@ def q():
 
 
 def test_stalled_producer_times_out_and_context_survives(q):
-    cfg = synth.TINY
+    cfg = synth.custom(N=512, K=512, M=256, r=8)   # M > 64: the tiled fused kernel
     W = synth.weight(cfg).cuda()
     X, A, B = synth.activations(cfg).cuda(), synth.lora_a(cfg).cuda(), synth.lora_b(cfg).cuda()
     w = q.quantize_nf4(W)
