@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 QLORA_OK = 0
 STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_BAD_SHAPE", -3: "QLORA_ERR_MISALIGNED",
           -4: "QLORA_ERR_UNSUPPORTED_RANK", -5: "QLORA_ERR_WORKSPACE_TOO_SMALL", -6: "QLORA_ERR_CUDA",
-          -7: "QLORA_ERR_DEVICE_TIMEOUT", -8: "QLORA_ERR_UNSUPPORTED_DEVICE"}
+          -7: "QLORA_ERR_DEVICE_TIMEOUT", -8: "QLORA_ERR_UNSUPPORTED_DEVICE", -9: "QLORA_ERR_EXCEEDS_STATIC_SCRATCH"}
 OP_QUANTIZE, OP_FWD, OP_BWD = 0, 1, 2
 OPT_SMALL_M_MAX, OPT_FAIL_LAUNCHES, OPT_WAIT_TIMEOUT_US, OPT_STALL_PRODUCER, OPT_LAUNCH_COUNT = 1, 2, 3, 4, 5
 KERNEL_FUSED_FWD, KERNEL_FUSED_DX = 1, 2
@@ -48,6 +48,7 @@ _SIGNATURES = {
                                ctypes.POINTER(_sz)]),
     "qlora_workspace_bytes": (_sz, [_int, _i64, _i64, _i64, _int]),
     "qlora_quantize_nf4": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_quantize_nf4_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "qlora_dequantize_nf4": (_int, [_wp, _vp, _vp]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -169,6 +170,17 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, ws: torch.Tensor
     _check(lib().qlora_quantize_nf4(_ptr(W), N, K, _ptr(w.codes), _ptr(w.qabsmax), _ptr(w.s2), _ptr(w.mean),
                                     _ptr(ws), ws.numel(), _stream(W.device)), "qlora_quantize_nf4")
     return w
+
+
+def quantize_nf4_noalloc(W: torch.Tensor, out: NF4Weight) -> NF4Weight:
+    """Quantise without any workspace: for callers that cannot allocate device
+    memory at call time. The library keeps its scratch in one static device
+    array (N*K up to 67,108,864 weights); `out` must be allocated beforehand."""
+    assert W.dtype == torch.float32 and W.is_cuda and W.dim() == 2
+    N, K = W.shape
+    _check(lib().qlora_quantize_nf4_noalloc(_ptr(W), N, K, _ptr(out.codes), _ptr(out.qabsmax), _ptr(out.s2),
+                                            _ptr(out.mean), _stream(W.device)), "qlora_quantize_nf4_noalloc")
+    return out
 
 
 def dequantize_nf4(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:

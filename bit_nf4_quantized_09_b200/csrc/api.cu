@@ -358,6 +358,7 @@ const char* qlora_status_string(qlora_status s) {
         case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
         case QLORA_ERR_DEVICE_TIMEOUT: return "QLORA_ERR_DEVICE_TIMEOUT";
         case QLORA_ERR_UNSUPPORTED_DEVICE: return "QLORA_ERR_UNSUPPORTED_DEVICE";
+        case QLORA_ERR_EXCEEDS_STATIC_SCRATCH: return "QLORA_ERR_EXCEEDS_STATIC_SCRATCH";
         default: return "QLORA_ERR_UNKNOWN";
     }
 }
@@ -655,3 +656,70 @@ qlora_status qlora_e4m3_encode(const float* x, uint8_t* q, int64_t n, void* stre
 }
 
 }  // extern "C"
+
+// ======================================================== no allocation ==
+// Quantiser scratch for callers that cannot allocate: one file-scope device
+// array, 4 MiB of fp32 block absmax followed by 16 KiB of fp64 partial sums.
+// Host code never touches `g_noalloc_scratch` directly (on the host its name
+// is only a stand-in); each device's real address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+namespace {
+
+constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 20;  // 64M weights
+constexpr size_t kNoAllocAbsmaxBytes = static_cast<size_t>(kNoAllocMaxBlocks) * 4;
+constexpr size_t kNoAllocTreeBytes = 16 * 1024;
+constexpr size_t kNoAllocBytes = kNoAllocAbsmaxBytes + kNoAllocTreeBytes;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+qlora_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        if (!p) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress(static scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, int64_t K, uint8_t* codes,
+                                                   uint8_t* qabsmax, float* s2, float* mean, void* stream) {
+    if (!W || !codes || !qabsmax || !s2 || !mean) return QLORA_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return QLORA_ERR_BAD_SHAPE;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(qabsmax) || !aligned16(s2) ||
+        (reinterpret_cast<uintptr_t>(mean) & 3u))
+        return QLORA_ERR_MISALIGNED;
+    if (N > kNoAllocMaxBlocks * kBlock / K) {
+        g_last_error = "qlora_quantize_nf4_noalloc: N*K = " + std::to_string(N) + "*" + std::to_string(K) +
+                       " exceeds the static scratch limit of " + std::to_string(kNoAllocMaxBlocks * kBlock) +
+                       " weights; use qlora_quantize_nf4 with a workspace";
+        return QLORA_ERR_EXCEEDS_STATIC_SCRATCH;
+    }
+    const int64_t nb = N * K / kBlock;
+    if (dq_tree_scratch_doubles(nb) * 8 > kNoAllocTreeBytes) return QLORA_ERR_EXCEEDS_STATIC_SCRATCH;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    qlora_status s = device_ready(&sms);
+    if (s != QLORA_OK) return s;
+    void* scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != QLORA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* absmax = static_cast<float*>(scratch);
+    double* tree = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocAbsmaxBytes);
+    QLORA_LAUNCH(launch_nf4_encode(W, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
+    return QLORA_OK;
+}

@@ -61,6 +61,7 @@ typedef int qlora_status;
                                               qlora_last_error()                        */
 #define QLORA_ERR_DEVICE_TIMEOUT       -7  /* device status: a pipeline wait ran out   */
 #define QLORA_ERR_UNSUPPORTED_DEVICE   -8  /* current device is not sm_100             */
+#define QLORA_ERR_EXCEEDS_STATIC_SCRATCH -9 /* N*K above the no-allocation limit        */
 
 /* Read-only view of a quantised weight. All five pointers are device
  * pointers owned by the caller; the library never writes through them. */
@@ -101,6 +102,32 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
 qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K,
                                 uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
                                 void* ws, size_t ws_bytes, void* stream);
+
+/* The same quantisation as qlora_quantize_nf4, for callers that cannot
+ * allocate device memory at the point of the call: inference-runtime plugin
+ * interfaces that hand over only input and output buffers and no workspace,
+ * and latency-critical code that must not call cudaMalloc because it can
+ * block or synchronise the device in the middle of a step. The pages about
+ * QLoRA have no counterpart to this call; it exists only for such callers.
+ *   - It takes no workspace and allocates nothing. Its scratch (the fp32
+ *     per-block absmax and the fp64 partial sums of the mean) lives in one
+ *     static device array of 4 MiB + 16 KiB that every GPU which loads the
+ *     library keeps until the process exits.
+ *   - Limit: N*K <= 67,108,864 weights (at most 1,048,576 blocks of 64, e.g.
+ *     8192 x 8192). Larger weights return QLORA_ERR_EXCEEDS_STATIC_SCRATCH
+ *     and launch nothing; use qlora_quantize_nf4 with a workspace instead.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array: calls that overlap on the GPU (for
+ *     example on two streams at once) race and corrupt each other's results.
+ *     Calls in one stream are ordered and safe; nothing in the array has to
+ *     start at zero, every byte read is written earlier in the same call.
+ *   - Outputs, argument checks and determinism are those of
+ *     qlora_quantize_nf4. */
+qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, int64_t K,
+                                        uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
+                                        void* stream);
 
 /* Dequantise to bf16 [N, K] (device W_out), bit-exact with the format's
  * definition above. [explainer 量子化を1段落で: x_hat = c * level[code]] */
