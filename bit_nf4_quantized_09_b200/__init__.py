@@ -24,6 +24,7 @@ STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_BAD_SHAPE",
           -7: "QLORA_ERR_DEVICE_TIMEOUT", -8: "QLORA_ERR_UNSUPPORTED_DEVICE", -9: "QLORA_ERR_EXCEEDS_STATIC_SCRATCH"}
 OP_QUANTIZE, OP_FWD, OP_BWD = 0, 1, 2
 OPT_SMALL_M_MAX, OPT_FAIL_LAUNCHES, OPT_WAIT_TIMEOUT_US, OPT_STALL_PRODUCER, OPT_LAUNCH_COUNT = 1, 2, 3, 4, 5
+OPT_SKINNY_MAX_SPLITS = 6
 KERNEL_FUSED_FWD, KERNEL_FUSED_DX = 1, 2
 
 
@@ -85,7 +86,18 @@ def _check(status: int, where: str):
         raise QLoraError(status, where, detail)
 
 
+try:
+    _raw_stream = torch._C._cuda_getCurrentRawStream  # fast path: the handle without a Stream object
+except AttributeError:  # pragma: no cover
+    _raw_stream = None
+
+
 def _stream(device=None) -> int:
+    if _raw_stream is not None:
+        idx = torch.cuda.current_device() if device is None else (device.index if isinstance(device, torch.device)
+                                                                  and device.index is not None else
+                                                                  torch.cuda.current_device())
+        return _raw_stream(idx)
     return torch.cuda.current_stream(device).cuda_stream
 
 
@@ -106,8 +118,15 @@ def nf4_bytes(N: int, K: int) -> dict:
     return dict(codes=c.value, qabsmax=q.value, s2=s.value, mean=m.value, total=total)
 
 
+_ws_cache: dict = {}
+
+
 def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
-    return int(lib().qlora_workspace_bytes(op, M, N, K, r))
+    key = (op, M, N, K, r)
+    v = _ws_cache.get(key)
+    if v is None:
+        v = _ws_cache[key] = int(lib().qlora_workspace_bytes(op, M, N, K, r))
+    return v
 
 
 def nf4_tables():
@@ -139,7 +158,14 @@ class NF4Weight:
     K: int
 
     def c_view(self) -> Nf4WeightC:
-        return Nf4WeightC(_ptr(self.codes), _ptr(self.qabsmax), _ptr(self.s2), _ptr(self.mean), self.N, self.K)
+        key = (self.codes.data_ptr(), self.qabsmax.data_ptr(), self.s2.data_ptr(), self.mean.data_ptr(),
+               self.N, self.K)
+        cached = self.__dict__.get("_c_view")
+        if cached is None or cached[0] != key:
+            cached = (key, Nf4WeightC(_ptr(self.codes), _ptr(self.qabsmax), _ptr(self.s2), _ptr(self.mean),
+                                      self.N, self.K))
+            self.__dict__["_c_view"] = cached
+        return cached[1]
 
     @staticmethod
     def empty(N: int, K: int, device) -> "NF4Weight":

@@ -24,6 +24,7 @@ std::atomic<int64_t> g_fail_launches{0};
 std::atomic<int64_t> g_timeout_us{1000000};
 std::atomic<int64_t> g_stall_producer{0};
 std::atomic<int64_t> g_launch_count{0};
+std::atomic<int64_t> g_skinny_max_splits{0};
 thread_local std::string g_last_error;
 
 // One-shot event requests of qlora_profile_next_launch, per kernel id.
@@ -171,9 +172,37 @@ qlora_status device_ready(int* sms_out) {
     return d.status;
 }
 
+// Recently encoded tensor maps, keyed by everything that goes into one, so a
+// caller that reuses its buffers pays for cuTensorMapEncodeTiled once.
+struct MapKey {
+    const void* base;
+    uint64_t d0, d1, row_bytes;
+    uint32_t b0, b1;
+    int dt, sw;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && row_bytes == o.row_bytes && b0 == o.b0 && b1 == o.b1 &&
+               dt == o.dt && sw == o.sw;
+    }
+};
+constexpr int kMapCacheSize = 64;
+std::mutex g_map_mu;
+MapKey g_map_keys[kMapCacheSize];
+CUtensorMap g_map_vals[kMapCacheSize];
+bool g_map_used[kMapCacheSize] = {};
+int g_map_next = 0;
+
 // 2-D tiled tensor map over a row-major [d1, d0] array (d0 contiguous).
 qlora_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
                       uint64_t row_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw, const char* what) {
+    const MapKey key{base, d0, d1, row_bytes, b0, b1, static_cast<int>(dt), static_cast<int>(sw)};
+    {
+        std::lock_guard<std::mutex> lk(g_map_mu);
+        for (int i = 0; i < kMapCacheSize; ++i)
+            if (g_map_used[i] && g_map_keys[i] == key) {
+                *m = g_map_vals[i];
+                return QLORA_OK;
+            }
+    }
     const cuuint64_t dims[2] = {d0, d1};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {b0, b1};
@@ -185,6 +214,11 @@ qlora_status make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, 
         g_last_error = std::string("cuTensorMapEncodeTiled(") + what + ") failed: " + std::to_string(r);
         return QLORA_ERR_CUDA;
     }
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    g_map_keys[g_map_next] = key;
+    g_map_vals[g_map_next] = *m;
+    g_map_used[g_map_next] = true;
+    g_map_next = (g_map_next + 1) % kMapCacheSize;
     return QLORA_OK;
 }
 
@@ -210,7 +244,9 @@ struct Split {
 };
 Split split_for(int64_t tiles, int64_t red) {
     const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
-    int64_t s = std::max<int64_t>(1, std::min<int64_t>(cdiv(kTargetCtas, std::max<int64_t>(tiles, 1)), KT));
+    // as many splits as fit in one wave of two CTAs per SM, at most 32
+    int64_t s = std::max<int64_t>(
+        1, std::min<int64_t>(std::min<int64_t>(kTargetCtas / std::max<int64_t>(tiles, 1), KT), 32));
     const int64_t steps = cdiv(KT, s);
     s = cdiv(KT, steps);
     return Split{static_cast<int>(s), static_cast<int>(steps)};
@@ -238,49 +274,55 @@ Split gemv_split(int64_t M, int64_t N, int64_t K) {
 }
 
 // ------------------------------------------------------- workspace layout --
+// Head of every fwd/bwd workspace: the device status word, then the split
+// tickets of the skinny matmuls; cleared by one memset at the start of each
+// call (the kernels also leave their tickets at zero).
 struct Layout {
-    size_t status = 0, cT = 0, partT = 0, sT = 0;         // forward
-    size_t Bt = 0, partU = 0, sU = 0, sUt = 0, sTt = 0;    // backward
-    size_t partA = 0, partB = 0, partY = 0;
+    size_t header = 0;                                   // bytes cleared per call
+    size_t status = 0, ctrT = 0, ctrU = 0, ctrA = 0, ctrB = 0, ctrY = 0;
+    size_t cT = 0, partT = 0, sT = 0, partY = 0;          // forward
+    size_t partU = 0, sU = 0, partA = 0;                  // backward (partA holds dA and dB partials)
     size_t total = 0;
-    int64_t ldc = 0, ldt = 0;
+    int64_t ldc = 0;
     Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1}, gemv{1, 1};
 };
 
 Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     Layout L;
     const int NR = rank_pad(r);
-    L.ldc = (N + 3) / 4 * 4;   // constants row pitch: a multiple of 16 bytes
-    L.ldt = (M + 7) / 8 * 8;   // pitch of the [r, M] transposed copies: a multiple of 16 bytes
-    size_t off = 0;
+    L.ldc = (N + 3) / 4 * 4;  // constants row pitch: a multiple of 16 bytes
+    const int64_t mtiles = std::max<int64_t>(1, cdiv(M, 128));
+    const int64_t ktiles = cdiv(K, 128), ntiles = cdiv(N, 128);
+    L.status = 0;
+    L.ctrT = 256;
+    L.ctrU = L.ctrT + 4 * static_cast<size_t>(mtiles);
+    L.ctrA = L.ctrU + 4 * static_cast<size_t>(mtiles);
+    L.ctrB = L.ctrA + 4 * static_cast<size_t>(ktiles);
+    L.ctrY = L.ctrB + 4 * static_cast<size_t>(ntiles);
+    L.header = up256(L.ctrY + 4 * static_cast<size_t>(ntiles));
+    size_t off = L.header;
     auto take = [&](size_t bytes) {
         const size_t at = off;
         off += up256(bytes);
         return at;
     };
-    L.status = take(256);
     L.cT = take(static_cast<size_t>(K / kBlock) * L.ldc * 4);
-    const int64_t mtiles = std::max<int64_t>(1, cdiv(M, 128));
     L.sT_split = split_for(mtiles, K);
+    L.sT = take(static_cast<size_t>(M) * r * 2);
     if (op == QLORA_OP_FWD) {
         L.partT = take(static_cast<size_t>(L.sT_split.splits) * M * NR * 4);
-        L.sT = take(static_cast<size_t>(M) * r * 2);
         if (M <= kGemvMaxM) {
             L.gemv = gemv_split(M, N, K);
             L.partY = take(static_cast<size_t>(L.gemv.splits) * M * N * 4);
         }
     } else {
         L.sU_split = split_for(mtiles, N);
-        L.grad_split = split_for(cdiv(K, 128) + cdiv(N, 128), M);
-        L.Bt = take(static_cast<size_t>(r) * N * 2);
+        L.grad_split = split_for(ktiles + ntiles, M);
         const int64_t part_down = std::max(L.sU_split.splits, L.sT_split.splits);
         L.partU = take(static_cast<size_t>(part_down) * M * NR * 4);
+        L.partT = L.partU;
         L.sU = take(static_cast<size_t>(M) * r * 2);
-        L.sUt = take(static_cast<size_t>(L.ldt) * r * 2);
-        L.sT = take(static_cast<size_t>(M) * r * 2);
-        L.sTt = take(static_cast<size_t>(L.ldt) * r * 2);
-        L.partA = take(static_cast<size_t>(L.grad_split.splits) * K * NR * 4);
-        L.partB = take(static_cast<size_t>(L.grad_split.splits) * N * NR * 4);
+        L.partA = take(static_cast<size_t>(L.grad_split.splits) * (K + N) * NR * 4);
     }
     L.total = off;
     return L;
@@ -296,26 +338,63 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
 
 uint64_t timeout_ns() { return static_cast<uint64_t>(std::max<int64_t>(1, g_timeout_us.load())) * 1000ull; }
 
-// T-side skinny matmul: part = act[M, red] . wt[r, red]^T, then
-// out = bf16(scale * sum of partials) as [M, r] (and [r, M] when out_t).
-qlora_status lora_down(const uint16_t* act, int64_t M, int64_t red, const uint16_t* wt, int r, float scale,
-                       const Split& sp, float* part, uint16_t* out, uint16_t* out_t, int64_t ldt, int* status,
+CUtensorMapSwizzle swizzle_for_rank(int NR) {
+    return NR == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : (NR == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Map of a row-major [rows, r] bf16 matrix read as an MN-major [64, NR] tile
+// per 64 rows (B, sU, sT).
+qlora_status make_rank_map(CUtensorMap* m, const uint16_t* base, int64_t rows, int r, const char* what) {
+    const int NR = rank_pad(r);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, r, rows, static_cast<uint64_t>(r) * 2, NR, 64,
+                    swizzle_for_rank(NR), what);
+}
+
+// The layout's split, lowered to the tuning cap if one is set.
+Split capped(const Split& sp, int64_t red) {
+    const int64_t cap = g_skinny_max_splits.load();
+    if (cap <= 0 || sp.splits <= cap) return sp;
+    const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
+    const int64_t steps = cdiv(KT, cap);
+    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
+}
+
+// out = bf16(scale * act[M, red] . W_r^T) as [M, r]. W_r is the rank-r
+// operand: A [r, red] read K-major, or (w_is_red_major) B [red, r] read
+// MN-major.
+qlora_status lora_down(const uint16_t* act, int64_t M, int64_t red, const uint16_t* wr, bool w_is_red_major, int r,
+                       float scale, const Split& sp_layout, float* part, int* counter, uint16_t* out, int* status,
                        cudaStream_t st) {
     const int NR = rank_pad(r);
+    const Split sp = capped(sp_layout, red);
     CUtensorMap ta, tb;
     QLORA_MAP(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, red, M, red * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "act");
-    QLORA_MAP(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, red, r, red * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "lora");
+    if (w_is_red_major) {
+        qlora_status s = make_rank_map(&tb, wr, red, r, "B");
+        if (s != QLORA_OK) return s;
+    } else {
+        QLORA_MAP(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wr, red, r, red * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+    }
     SkinnyArgs a{};
     a.NR = NR;
-    a.a_mn_major = 0;
-    a.p[0] = SkinnyProblem{M, red, sp.splits, sp.steps, part};
-    a.p[1] = a.p[0];
+    a.r = r;
+    SkinnyProblem& P = a.p[0];
+    P.rows = M;
+    P.red = red;
+    P.splits = sp.splits;
+    P.steps_per_split = sp.steps;
+    P.a_mn_major = 0;
+    P.b_mn_major = w_is_red_major ? 1 : 0;
+    P.mode = kSkinnyOutBf16;
+    P.scale = scale;
+    P.part = part;
+    P.counter = counter;
+    P.out_bf16 = out;
+    a.p[1] = P;
     a.status = status;
     a.timeout_ns = timeout_ns();
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_skinny(ta, tb, ta, tb, a, 1, st), 1, "skinny(lora down)");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_reduce_lora_down(part, sp.splits, M, NR, r, scale, out, out_t, ldt, st), 1, "reduce(lora down)");
     return QLORA_OK;
 }
 
@@ -375,6 +454,10 @@ qlora_status qlora_set_option(int option, int64_t value) {
             return QLORA_OK;
         case QLORA_OPT_STALL_PRODUCER: g_stall_producer = value ? 1 : 0; return QLORA_OK;
         case QLORA_OPT_LAUNCH_COUNT: g_launch_count = value; return QLORA_OK;
+        case QLORA_OPT_SKINNY_MAX_SPLITS:
+            if (value < 0) return QLORA_ERR_INVALID_ARG;
+            g_skinny_max_splits = value;
+            return QLORA_OK;
         default: return QLORA_ERR_INVALID_ARG;
     }
 }
@@ -386,6 +469,7 @@ int64_t qlora_get_option(int option) {
         case QLORA_OPT_WAIT_TIMEOUT_US: return g_timeout_us.load();
         case QLORA_OPT_STALL_PRODUCER: return g_stall_producer.load();
         case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
+        case QLORA_OPT_SKINNY_MAX_SPLITS: return g_skinny_max_splits.load();
         default: return -1;
     }
 }
@@ -428,7 +512,10 @@ qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, vo
     if (injected_failure()) return QLORA_ERR_CUDA;
     int sms = 0;
     if ((s = device_ready(&sms)) != QLORA_OK) return s;
-    QLORA_LAUNCH(launch_nf4_dequant(w->codes, w->qabsmax, w->s2, w->mean, w->N, w->K, W_out, tables(), sms,
+    CUtensorMap t_out;
+    QLORA_MAP(&t_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_out, kBlock, w->N * w->K / kBlock, kBlock * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B, "W_out");
+    QLORA_LAUNCH(launch_nf4_dequant(t_out, w->codes, w->qabsmax, w->s2, w->mean, w->N, w->K, tables(), sms,
                                     static_cast<cudaStream_t>(stream)),
                  1, "nf4_dequant");
     return QLORA_OK;
@@ -461,10 +548,12 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
     const float scale = alpha / static_cast<float>(r);
 
-    QLORA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st), "clear status");
+    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
-    if ((s = lora_down(X, M, K, A, r, scale, L.sT_split, partT, sT, nullptr, 0, status, st)) != QLORA_OK) return s;
+    if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
+                       status, st)) != QLORA_OK)
+        return s;
 
     const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
     if (M <= small) {
@@ -481,9 +570,14 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         ga.N = N;
         ga.K = K;
         ga.Mp = Mp;
+        ga.r = r;
         ga.splits = L.gemv.splits;
         ga.steps_per_split = L.gemv.steps;
         ga.part = reinterpret_cast<float*>(base + L.partY);
+        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
+        ga.sT = sT;
+        ga.B = B;
+        ga.Y = Y;
         ga.status = status;
         ga.timeout_ns = timeout_ns();
         if (injected_failure()) return QLORA_ERR_CUDA;
@@ -492,8 +586,6 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
         QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
         if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
-        if (injected_failure()) return QLORA_ERR_CUDA;
-        QLORA_LAUNCH(launch_gemv_reduce(ga.part, ga.splits, M, N, sT, B, r, Y, st), 1, "gemv reduce");
         return QLORA_OK;
     }
 
@@ -551,30 +643,24 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     uint8_t* base = static_cast<uint8_t*>(ws);
     int* status = reinterpret_cast<int*>(base + L.status);
     float* cT = reinterpret_cast<float*>(base + L.cT);
-    uint16_t* Bt = reinterpret_cast<uint16_t*>(base + L.Bt);
     float* partU = reinterpret_cast<float*>(base + L.partU);
     uint16_t* sU = reinterpret_cast<uint16_t*>(base + L.sU);
-    uint16_t* sUt = reinterpret_cast<uint16_t*>(base + L.sUt);
-    uint16_t* sT = reinterpret_cast<uint16_t*>(base + L.sT);
-    uint16_t* sTt = reinterpret_cast<uint16_t*>(base + L.sTt);
+    const uint16_t* sT = sT_in ? sT_in : reinterpret_cast<uint16_t*>(base + L.sT);
     float* partA = reinterpret_cast<float*>(base + L.partA);
-    float* partB = reinterpret_cast<float*>(base + L.partB);
     const float scale = alpha / static_cast<float>(r);
     const int NR = rank_pad(r);
 
-    QLORA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st), "clear status");
+    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_transpose_bf16(B, N, r, Bt, N, st), 1, "transpose B");
-    // sU = s dY B  ([M, r] and [r, M])
-    if ((s = lora_down(dY, M, N, Bt, r, scale, L.sU_split, partU, sU, sUt, L.ldt, status, st)) != QLORA_OK) return s;
-    // sT^T from the forward's sT, or sT recomputed
-    if (sT_in) {
-        if (injected_failure()) return QLORA_ERR_CUDA;
-        QLORA_LAUNCH(launch_transpose_bf16(sT_in, M, r, sTt, L.ldt, st), 1, "transpose sT");
-    } else {
-        if ((s = lora_down(X, M, K, A, r, scale, L.sT_split, partU, sT, sTt, L.ldt, status, st)) != QLORA_OK)
+    // sU = s dY B, with B [N, r] read in place (MN-major)
+    if ((s = lora_down(dY, M, N, B, true, r, scale, L.sU_split, partU, reinterpret_cast<int*>(base + L.ctrU), sU,
+                       status, st)) != QLORA_OK)
+        return s;
+    // sT from the forward, or recomputed
+    if (!sT_in) {
+        if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partU, reinterpret_cast<int*>(base + L.ctrT),
+                           reinterpret_cast<uint16_t*>(base + L.sT), status, st)) != QLORA_OK)
             return s;
     }
 
@@ -603,25 +689,34 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused dX");
     if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
 
-    // dA^T[K, NR] = X^T sU  and  dB[N, NR] = dY^T sT, split over tokens
+    // dA = sU^T X (as dA^T[K, r] = X^T sU) and dB = dY^T sT, split over tokens
     CUtensorMap ta0, tb0, ta1, tb1;
     QLORA_MAP(&ta0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
-    QLORA_MAP(&tb0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sUt, M, r, L.ldt * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "sU^T");
+    if ((s = make_rank_map(&tb0, sU, M, r, "sU")) != QLORA_OK) return s;
     QLORA_MAP(&ta1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
-    QLORA_MAP(&tb1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sTt, M, r, L.ldt * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "sT^T");
+    if ((s = make_rank_map(&tb1, sT, M, r, "sT")) != QLORA_OK) return s;
     SkinnyArgs ga{};
     ga.NR = NR;
-    ga.a_mn_major = 1;
-    ga.p[0] = SkinnyProblem{K, M, L.grad_split.splits, L.grad_split.steps, partA};
-    ga.p[1] = SkinnyProblem{N, M, L.grad_split.splits, L.grad_split.steps, partB};
+    ga.r = r;
+    const Split gsp = capped(L.grad_split, M);
+    for (int p = 0; p < 2; ++p) {
+        SkinnyProblem& P = ga.p[p];
+        P.rows = p == 0 ? K : N;
+        P.red = M;
+        P.splits = gsp.splits;
+        P.steps_per_split = gsp.steps;
+        P.a_mn_major = 1;
+        P.b_mn_major = 1;
+        P.mode = p == 0 ? kSkinnyOutF32Transposed : kSkinnyOutF32;
+        P.scale = 1.0f;
+        P.part = partA + (p == 0 ? 0 : static_cast<int64_t>(L.grad_split.splits) * K * NR);
+        P.counter = reinterpret_cast<int*>(base + (p == 0 ? L.ctrA : L.ctrB));
+        P.out_f32 = p == 0 ? dA : dB;
+    }
     ga.status = status;
     ga.timeout_ns = timeout_ns();
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_skinny(ta0, tb0, ta1, tb1, ga, 2, st), 1, "skinny(grads)");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_reduce_lora_grads(partA, L.grad_split.splits, K, partB, L.grad_split.splits, N, NR, r, dA,
-                                          dB, st),
-                 1, "reduce(grads)");
     return QLORA_OK;
 }
 

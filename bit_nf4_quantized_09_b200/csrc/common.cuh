@@ -93,7 +93,7 @@ __device__ __forceinline__ Nf4BlockLut make_block_lut(const float (&level)[16], 
 // high nibble and element 2b+1 in its low nibble) -> eight bf16 in code order,
 // as four bf16x2 words (out[i] = elements 2i, 2i+1 with 2i in the low half).
 __device__ __forceinline__ void lut_decode8(const Nf4BlockLut& t, uint32_t packed, uint32_t (&out)[4]) {
-    const uint32_t idx = packed & 0x77777777u;        // low 3 bits of every code
+    const uint32_t idx = packed & 0x77777777u;         // low 3 bits of every code
     const uint32_t top = (packed >> 3) & 0x11111111u;  // top bit of every code
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -177,6 +177,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// Shared -> global tiled bulk store (TMA), tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

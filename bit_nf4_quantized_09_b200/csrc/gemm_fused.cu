@@ -35,7 +35,7 @@ constexpr uint32_t kStageBytes = kOffC + kCBytes;  // 73 KB, a multiple of 1024
 constexpr uint32_t kBarOffset = kFusedStages * kStageBytes;
 constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;  // + barriers, + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr int kDequantThreads = 256;
+constexpr int kDequantWarps = 8;
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFusedStages; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(deq + s, kDequantThreads);
+            mbar_init(deq + s, kDequantWarps);  // one arrive per dequant warp
             mbar_init(empty + s, 1);
         }
         mbar_init(acc, 1);
@@ -197,7 +197,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int kt = 0; kt < KT; ++kt) {
             const int s = kt % kFusedStages;
             const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
-            if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
+            // every lane waits; the outcome is made warp-uniform before any branch
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(full + s, u & 1u, tmo, args.status));
+            if (!ok) break;
             uint8_t* st = smem + s * kStageBytes;
             const uint32_t codes = smem_u32(st + kOffCodes);
             const uint32_t wt = smem_u32(st + kOffW);
@@ -218,15 +220,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 dequant_block(tab, cs[a * 64 + nl], crow + (((2 * a) ^ sw) << 4), crow + (((2 * a + 1) ^ sw) << 4),
                               [&](int j) { return dst + ((static_cast<uint32_t>(j) ^ sw) << 4); });
             }
-            fence_proxy_async_smem();
-            mbar_arrive(deq + s);
+            fence_proxy_async_smem();  // this thread's tile stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(deq + s);
         }
         if (!ok) *abort_flag = 1;
 
         // ------------------------------------------------------- epilogue --
-        const bool acc_ok = mbar_wait(acc, 0, tmo, args.status);
+        const bool acc_ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, tmo, args.status));
         tc_fence_after();
-        if (acc_ok && !*abort_flag) {
+        if (__all_sync(0xFFFFFFFFu, acc_ok && !*abort_flag)) {
             const int q = warp & 3, h = warp >> 2;
             const int64_t row = m0 + h * 128 + q * 32 + lane;
             for (int c0 = 0; c0 < kFusedBN; c0 += 32) {

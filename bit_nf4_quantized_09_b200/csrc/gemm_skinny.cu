@@ -1,13 +1,19 @@
 // Rank-r ("skinny") matmuls of the LoRA path on the sm_100 tensor core.
 //
 // "waylandz ch.26" 26.2.4: y = W x + (alpha/r) B (A x). The down-projections
-// X A^T (forward) and dY B (backward) and the adapter gradients
-//   dA = s (dY B)^T X,  dB = s dY^T (X A^T)
-// ("ta-paperlens QLoRA explainer", 勾配は実際どこへ行くのか: only A and B keep
-// a gradient) all have one side of width r <= 64. Each is computed as
-// D[rows, NR] = A_op[rows, red] . B_op[NR, red]^T with NR = max(16, r) on
-// the UMMA N side, split over the reduction into fp32 partials that a second,
-// deterministic pass adds in a fixed order.
+//   sT = s X A^T (forward),  sU = s dY B (backward)
+// and the adapter gradients ("ta-paperlens QLoRA explainer",
+// 勾配は実際どこへ行くのか: only A and B keep a gradient)
+//   dA = sU^T X,  dB = dY^T sT
+// all have one side of width r <= 64. Each is D[rows, NR] = A_op[rows, red] .
+// B_op[NR, red]^T with NR = max(16, r) on the UMMA N side:
+//   A_op  K-major (X, dY read along the reduction) or MN-major (X^T, dY^T
+//         read by TMA straight out of X and dY with the 128-byte swizzle);
+//   B_op  K-major (A [r, K]) or MN-major (B [N, r], sU and sT [M, r] read in
+//         place with a 32/64/128-byte swizzle matching NR).
+// The reduction is split over CTAs; each CTA writes fp32 partials and the last
+// CTA of a row tile (atomic ticket, no waiting) adds them in split order and
+// writes the result, so outputs are deterministic.
 //   warp 0 TMA producer, warp 1 TMEM owner + UMMA issuer, warps 2-5 epilogue.
 #include <algorithm>
 
@@ -19,18 +25,35 @@ namespace qlora {
 namespace {
 
 constexpr uint32_t kABytes = 128 * 64 * 2;  // 16 KB
-constexpr uint32_t kBBytes = 64 * 64 * 2;   // up to 64 rows of 128 B
+constexpr uint32_t kBBytes = 64 * 64 * 2;   // up to 64 x 64 bf16
 constexpr uint32_t kStage = kABytes + kBBytes;
 constexpr uint32_t kBarOff = kSkinnyStages * kStage;
 constexpr uint32_t kSmem = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 64;
+
+// Shared-memory descriptor of an MN-major B tile [64 reduction rows, NR
+// columns] written by TMA with the swizzle whose span is NR * 2 bytes: rows of
+// NR*2 bytes, 8-row groups SBO = 8 * NR * 2 apart.
+__device__ __forceinline__ uint64_t mn_b_desc(uint32_t addr, int NR) {
+    const uint32_t row = static_cast<uint32_t>(NR) * 2u;
+    const uint32_t layout = NR == 16 ? 6u : (NR == 32 ? 4u : 2u);  // SW32, SW64, SW128
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;  // leading byte offset: one atom spans all NR columns
+    d |= static_cast<uint64_t>(((8u * row) >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(layout) << 61;
+    return d;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
     skinny_gemm(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
                 const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                 const SkinnyArgs args) {
     const int prob = blockIdx.z;
-    const SkinnyProblem& P = args.p[prob];
+    const SkinnyProblem P = args.p[prob];
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
     if (row0 >= P.rows || static_cast<int>(blockIdx.y) >= P.splits) return;  // whole CTA idle
     const CUtensorMap* ta = prob ? &tm_a1 : &tm_a0;
@@ -43,6 +66,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     uint64_t* acc = empty + kSkinnyStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NR = args.NR;
@@ -66,6 +90,10 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(ta);
+        tma_prefetch_desc(tb);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -86,13 +114,16 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                 const int k = (k_begin + i) * 64;
                 uint8_t* st = smem + s * kStage;
                 mbar_arrive_expect_tx(full + s, kABytes + b_bytes);
-                if (!args.a_mn_major) {
+                if (!P.a_mn_major) {
                     tma_load_2d(st, ta, full + s, k, static_cast<int>(row0));
                 } else {
                     tma_load_2d(st, ta, full + s, static_cast<int>(row0), k);
                     tma_load_2d(st + 8192, ta, full + s, static_cast<int>(row0) + 64, k);
                 }
-                tma_load_2d(st + kABytes, tb, full + s, k, 0);
+                if (!P.b_mn_major)
+                    tma_load_2d(st + kABytes, tb, full + s, k, 0);
+                else
+                    tma_load_2d(st + kABytes, tb, full + s, 0, k);
                 last_use[s] = static_cast<int>(u);
             }
             for (int s = 0; s < kSkinnyStages; ++s)
@@ -101,7 +132,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, NR, args.a_mn_major != 0, false);
+            const uint32_t idesc = idesc_bf16(128, NR, P.a_mn_major != 0, P.b_mn_major != 0);
             bool ok = true;
             for (int i = 0; i < steps; ++i) {
                 const int s = i % kSkinnyStages;
@@ -111,9 +142,10 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                 const uint32_t a = smem_u32(smem + s * kStage), b = a + kABytes;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t adesc = args.a_mn_major ? sw128_desc(a + kk * 2048, 8192, 1024)
-                                                           : sw128_desc(a + kk * 32, 16, 1024);
-                    const uint64_t bdesc = sw128_desc(b + kk * 32, 16, 1024);
+                    const uint64_t adesc = P.a_mn_major ? sw128_desc(a + kk * 2048, 8192, 1024)
+                                                        : sw128_desc(a + kk * 32, 16, 1024);
+                    const uint64_t bdesc = P.b_mn_major ? mn_b_desc(b + kk * 16 * NR * 2, NR)
+                                                        : sw128_desc(b + kk * 32, 16, 1024);
                     umma_f16(tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(empty + s);
@@ -127,26 +159,95 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         }
         __syncwarp();
     } else {
-        // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
-        const bool ok = mbar_wait(acc, 0, tmo, args.status);
+        // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1; thread = output row
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, tmo, args.status));
         tc_fence_after();
         const int q = warp & 3;
         const int64_t row = row0 + q * 32 + lane;
-        float* out = P.part + (static_cast<int64_t>(blockIdx.y) * P.rows + row) * NR;
-        for (int c0 = 0; c0 < NR; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, r);
-            tmem_ld_wait();
-            if (row < P.rows) {
-                float4* dst = reinterpret_cast<float4*>(out + c0);
-                const bool good = ok && !*abort_flag && steps > 0;
+        const bool good = ok && !*abort_flag && steps > 0;
+        float v[64];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float4 v = good ? make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                  __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                    dst[i] = v;
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            if (c0 < NR) {
+                uint32_t r[16];
+                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[c0 + i] = good ? __uint_as_float(r[i]) : 0.0f;
+            }
+        }
+        bool last = true;
+        if (P.splits > 1) {
+            if (row < P.rows) {
+                float4* dst = reinterpret_cast<float4*>(P.part + (static_cast<int64_t>(blockIdx.y) * P.rows + row) * NR);
+#pragma unroll
+                for (int c = 0; c < 64; c += 4)
+                    if (c < NR) dst[c / 4] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+            }
+            __threadfence();  // publish this split's partials before taking a ticket
+            epi_bar();
+            if (threadIdx.x == 64) {
+                const int ticket = atomicAdd(P.counter + blockIdx.x, 1);
+                *last_flag = (ticket == P.splits - 1) ? 1 : 0;
+            }
+            epi_bar();
+            last = *last_flag != 0;
+            if (last) {
+                __threadfence();  // see the other splits' partials
+                if (row < P.rows) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) v[c] = 0.0f;
+                    // splits in order; four splits' slices are loaded at once so
+                    // the loads overlap
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 16) {
+                        if (c0 < NR) {
+                            for (int s0 = 0; s0 < P.splits; s0 += 4) {
+                                float4 x[4][4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const float4* src = reinterpret_cast<const float4*>(
+                                        P.part + (static_cast<int64_t>(s0 + u) * P.rows + row) * NR + c0);
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i)
+                                        x[u][i] = (s0 + u < P.splits) ? __ldcg(src + i)
+                                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                                }
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        v[c0 + 4 * i] += x[u][i].x;
+                                        v[c0 + 4 * i + 1] += x[u][i].y;
+                                        v[c0 + 4 * i + 2] += x[u][i].z;
+                                        v[c0 + 4 * i + 3] += x[u][i].w;
+                                    }
+                                }
+                            }
+                        }
+                    }
                 }
+                if (threadIdx.x == 64) P.counter[blockIdx.x] = 0;  // ready for the next call
+            }
+        }
+        if (last && row < P.rows) {
+            const int r = args.r;
+            if (P.mode == kSkinnyOutBf16) {
+                uint16_t* o = P.out_bf16 + row * r;
+#pragma unroll
+                for (int j = 0; j < 64; j += 2)
+                    if (j < r)
+                        *reinterpret_cast<uint32_t*>(o + j) =
+                            pack_bf16x2(__fmul_rn(P.scale, v[j]), __fmul_rn(P.scale, v[j + 1]));
+            } else if (P.mode == kSkinnyOutF32Transposed) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < r) P.out_f32[static_cast<int64_t>(j) * P.rows + row] = v[j];
+            } else {
+                float4* o = reinterpret_cast<float4*>(P.out_f32 + row * r);
+#pragma unroll
+                for (int j = 0; j < 64; j += 4)
+                    if (j < r) o[j / 4] = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
     }
@@ -156,63 +257,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
-    }
-}
-
-// ------------------------------------------------------------- reductions --
-
-__global__ void reduce_lora_down_kernel(const float* __restrict__ part, int splits, int64_t M, int NR, int r,
-                                        float scale, uint16_t* __restrict__ out_rm, uint16_t* __restrict__ out_t,
-                                        int64_t ldt) {
-    const int64_t total = M * r;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t m = i / r;
-        const int j = static_cast<int>(i % r);
-        float acc = 0.0f;
-        for (int s = 0; s < splits; ++s) acc += part[(s * M + m) * NR + j];
-        const uint16_t b = static_cast<uint16_t>(pack_bf16x2(__fmul_rn(scale, acc), 0.0f) & 0xFFFFu);
-        out_rm[m * r + j] = b;
-        if (out_t) out_t[static_cast<int64_t>(j) * ldt + m] = b;
-    }
-}
-
-__global__ void reduce_lora_grads_kernel(const float* __restrict__ partA, int splitsA, int64_t K,
-                                         const float* __restrict__ partB, int splitsB, int64_t N, int NR, int r,
-                                         float* __restrict__ dA, float* __restrict__ dB) {
-    const int64_t totalA = static_cast<int64_t>(r) * K, totalB = N * r;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < totalA + totalB;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        if (i < totalA) {
-            const int j = static_cast<int>(i / K);
-            const int64_t k = i % K;
-            float acc = 0.0f;
-            for (int s = 0; s < splitsA; ++s) acc += partA[(s * K + k) * NR + j];
-            dA[i] = acc;
-        } else {
-            const int64_t t = i - totalA;
-            const int64_t n = t / r;
-            const int j = static_cast<int>(t % r);
-            float acc = 0.0f;
-            for (int s = 0; s < splitsB; ++s) acc += partB[(s * N + n) * NR + j];
-            dB[t] = acc;
-        }
-    }
-}
-
-__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int64_t rows, int64_t cols,
-                                      uint16_t* __restrict__ out, int64_t ldo) {
-    __shared__ uint16_t tile[32][33];
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int i = ty; i < 32; i += 8) {
-        const int64_t rr = r0 + i, cc = c0 + tx;
-        tile[i][tx] = (rr < rows && cc < cols) ? in[rr * cols + cc] : 0;
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int64_t cc = c0 + i, rr = r0 + tx;
-        if (cc < cols && rr < rows) out[cc * ldo + rr] = tile[tx][i];
     }
 }
 
@@ -235,30 +279,6 @@ cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CU
 
 cudaError_t skinny_init_device() {
     return cudaFuncSetAttribute(skinny_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-}
-
-cudaError_t launch_reduce_lora_down(const float* part, int splits, int64_t M, int NR, int r, float scale,
-                                    uint16_t* out_rm, uint16_t* out_t, int64_t ldt, cudaStream_t st) {
-    const int64_t total = M * r;
-    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4096));
-    reduce_lora_down_kernel<<<std::max(grid, 1), 256, 0, st>>>(part, splits, M, NR, r, scale, out_rm, out_t, ldt);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_reduce_lora_grads(const float* partA, int splitsA, int64_t K, const float* partB, int splitsB,
-                                     int64_t N, int NR, int r, float* dA, float* dB, cudaStream_t st) {
-    const int64_t total = static_cast<int64_t>(r) * K + N * r;
-    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8192));
-    reduce_lora_grads_kernel<<<std::max(grid, 1), 256, 0, st>>>(partA, splitsA, K, partB, splitsB, N, NR, r, dA,
-                                                                dB);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ldo,
-                                  cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
-    transpose_bf16_kernel<<<grid, 256, 0, st>>>(in, rows, cols, out, ldo);
-    return cudaGetLastError();
 }
 
 }  // namespace qlora

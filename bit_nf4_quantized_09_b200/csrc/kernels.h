@@ -15,8 +15,10 @@ cudaError_t launch_nf4_encode(const float* W, int64_t N, int64_t K, uint8_t* cod
 size_t dq_tree_scratch_doubles(int64_t nb);
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,
                                 float* mean, cudaStream_t st);
-cudaError_t launch_nf4_dequant(const uint8_t* codes, const uint8_t* q, const float* s2, const float* mean,
-                               int64_t N, int64_t K, uint16_t* out, const Nf4Tables& tab, int num_sms,
+// out_map: the bf16 output viewed as [N*K/64 rows, 64], box {64, 128}, SW128.
+constexpr size_t kDequantSmem = 2 * 128 * 128 + 1024;
+cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const uint8_t* q, const float* s2,
+                               const float* mean, int64_t N, int64_t K, const Nf4Tables& tab, int num_sms,
                                cudaStream_t st);
 cudaError_t launch_decode_constants_t(const uint8_t* q, const float* s2, const float* mean, int64_t N, int64_t K,
                                       int64_t ldc, float* cT, cudaStream_t st);
@@ -60,8 +62,7 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
                             const Nf4Tables& tab, cudaStream_t st);
 
 // ------------------------------------------------ small-batch dequant GEMV --
-constexpr int kGemvStages = 3;
-constexpr int kGemvThreads = 192;  // 4 dequant/epilogue warps, TMA warp, MMA warp
+constexpr int kGemvThreads = 320;  // 8 dequant warps (4 also epilogue), TMA warp, MMA warp
 constexpr int kGemvMaxM = 64;      // tokens that fit the UMMA N side of one tile
 size_t gemv_smem_bytes();
 cudaError_t gemv_init_device();
@@ -69,9 +70,14 @@ cudaError_t gemv_init_device();
 struct GemvArgs {
     int64_t M, N, K;
     int Mp;              // M rounded up to a multiple of 16
+    int r;               // LoRA rank
     int splits;          // K splits (grid.y)
     int steps_per_split;
-    float* part;         // fp32 [splits][M][N]
+    float* part;         // fp32 [splits][M][N] partials (splits > 1)
+    int* counter;        // [N/128 row tiles] tickets, zero before the launch; left zero
+    const uint16_t* sT;  // bf16 [M, r]
+    const uint16_t* B;   // bf16 [N, r]
+    uint16_t* Y;         // bf16 [M, N]
     int* status;
     uint64_t timeout_ns;
 };
@@ -80,30 +86,39 @@ struct GemvArgs {
 // cT {ldc, K/64} box {128, 1}.
 cudaError_t launch_gemv(const CUtensorMap& x, const CUtensorMap& codes, const CUtensorMap& cT, const GemvArgs& a,
                         const Nf4Tables& tab, cudaStream_t st);
-// Y[m][n] = bf16(sum_s part[s][m][n] + sum_j sT[m][j] B[n][j]).
-cudaError_t launch_gemv_reduce(const float* part, int splits, int64_t M, int64_t N, const uint16_t* sT,
-                               const uint16_t* B, int r, uint16_t* Y, cudaStream_t st);
 
 // ---------------------------------------------------------- skinny GEMMs --
-// D[rows, NR] = sum over a reduction range of A_op[rows, red] * B_op[NR, red]^T,
-// written as fp32 partials part[split][rows][NR]. Two independent problems
-// may share one launch (blockIdx.z).
+// D[rows, NR] = sum over the reduction of A_op[rows, red] * B_op[NR, red]^T,
+// split over the reduction (grid.y); the last CTA of each 128-row tile adds
+// the fp32 partials in split order and writes the output. Two independent
+// problems may share one launch (blockIdx.z).
 constexpr int kSkinnyStages = 4;
 constexpr int kSkinnyThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
 size_t skinny_smem_bytes();
 cudaError_t skinny_init_device();
 
+constexpr int kSkinnyOutBf16 = 0;           // out_bf16[row * r + j] = bf16(scale * D)
+constexpr int kSkinnyOutF32Transposed = 1;  // out_f32[j * rows + row] = D
+constexpr int kSkinnyOutF32 = 2;            // out_f32[row * r + j] = D
+
 struct SkinnyProblem {
-    int64_t rows;       // output rows (tiles of 128)
-    int64_t red;        // reduction length (steps of 64)
-    int splits;         // reduction splits (grid.y)
+    int64_t rows;        // output rows (tiles of 128)
+    int64_t red;         // reduction length (steps of 64)
+    int splits;          // reduction splits (grid.y)
     int steps_per_split;
-    float* part;        // fp32 [splits][rows][NR]
+    int a_mn_major;      // A_op rows-contiguous: two 64-wide TMA boxes per step
+    int b_mn_major;      // B_op stored [red, NR] (box {NR, 64}, swizzle = NR*2 bytes)
+    int mode;            // kSkinnyOut*
+    float scale;         // bf16 output scale
+    float* part;         // fp32 [splits][rows][NR] partials (splits > 1)
+    int* counter;        // [row tiles] tickets, zero before the launch; left zero
+    uint16_t* out_bf16;
+    float* out_f32;
 };
 
 struct SkinnyArgs {
-    int NR;             // 16, 32 or 64
-    int a_mn_major;     // A_op stored rows-contiguous (MN-major) instead of red-contiguous
+    int NR;              // 16, 32 or 64
+    int r;               // output columns
     SkinnyProblem p[2];
     int* status;
     uint64_t timeout_ns;
@@ -111,16 +126,5 @@ struct SkinnyArgs {
 
 cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                           const CUtensorMap& b1, const SkinnyArgs& args, int nproblems, cudaStream_t st);
-
-// out_rm[m][j] = bf16(scale * sum_s part[s][m][j]) for j < r (row-major [M, r]);
-// out_t[j * ldt + m] likewise transposed ([r, M], row pitch ldt) when out_t is not NULL.
-cudaError_t launch_reduce_lora_down(const float* part, int splits, int64_t M, int NR, int r, float scale,
-                                    uint16_t* out_rm, uint16_t* out_t, int64_t ldt, cudaStream_t st);
-// dA[j][k] = sum_s partA[s][k][j] (fp32 [r, K]); dB[n][j] = sum_s partB[s][n][j] (fp32 [N, r]).
-cudaError_t launch_reduce_lora_grads(const float* partA, int splitsA, int64_t K, const float* partB, int splitsB,
-                                     int64_t N, int NR, int r, float* dA, float* dB, cudaStream_t st);
-// out[j * ldo + n] = in[n][j]: bf16 [rows, cols] -> [cols, rows] with row pitch ldo >= rows.
-cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ldo,
-                                  cudaStream_t st);
 
 }  // namespace qlora

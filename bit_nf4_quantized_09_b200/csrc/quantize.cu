@@ -8,6 +8,8 @@
 // "QLoRA" glossary (ultralytics), NF4 construction and nearest-level argmin.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,7 +20,26 @@ namespace qlora {
 // consecutive weights per thread (two 16-byte loads), four packed bytes out.
 // Nearest level = number of decision thresholds strictly below v = w / c,
 // found by a 4-step binary search over the 15 thresholds in shared memory.
+//
+// v is the correctly rounded quotient, computed without a division per
+// weight by Markstein's method (P. Markstein, IBM J. Res. Dev. 34(1), 1990;
+// Muller et al., Handbook of Floating-Point Arithmetic, 2nd ed., sec. 4.9):
+// with y = RN(1/c) and q0 = RN(w*y), the remainder w - c*q0 is exact in one
+// fma and RN(q0 + (w - c*q0)*y) = RN(w/c). The theorem needs the quotient and
+// the remainder to stay in the normal range; blocks with c < 2^-96 take the
+// IEEE division instead (so no remainder of a value near a threshold can be
+// subnormal), and values far below every threshold code to the zero level
+// either way.
+// Loads of the next block run ahead of the current block's arithmetic.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t nf4_code(float q, const float* sM) {
+    int k = (q > sM[7]) ? 8 : 0;
+    k += (q > sM[k + 3]) ? 4 : 0;
+    k += (q > sM[k + 1]) ? 2 : 0;
+    k += (q > sM[k]) ? 1 : 0;
+    return static_cast<uint32_t>(k);
+}
+
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restrict__ W, int64_t nblocks,
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
                                                          Nf4Tables tab) {
@@ -26,20 +47,27 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
     if (threadIdx.x < 15) sM[threadIdx.x] = tab.thresh[threadIdx.x];
     __syncthreads();
 
-    const int sub = threadIdx.x & 7;  // position inside the block
+    const int sub = threadIdx.x & 7;               // position inside the block
     const int lane_blk = (threadIdx.x & 31) >> 3;  // which of the warp's 4 blocks
-    const int64_t warps_per_grid = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t stride = ((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) * 4;
+    int64_t bw = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * 4;
+
     // warp-uniform loop: every lane takes part in the shuffles of every pass
-    for (int64_t bw = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * 4; bw < nblocks;
-         bw += warps_per_grid * 4) {
+    float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+    if (bw + lane_blk < nblocks) {
+        x0 = __ldcs(W + (bw + lane_blk) * 16 + sub * 2);
+        x1 = __ldcs(W + (bw + lane_blk) * 16 + sub * 2 + 1);
+    }
+    for (; bw < nblocks; bw += stride) {
         const int64_t b = bw + lane_blk;
         const bool valid = b < nblocks;
-        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
-        if (valid) {
-            x0 = __ldcs(W + b * 16 + sub * 2);
-            x1 = __ldcs(W + b * 16 + sub * 2 + 1);
+        const int64_t nb = b + stride;
+        float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
+        if (nb < nblocks) {
+            n0 = __ldcs(W + nb * 16 + sub * 2);
+            n1 = __ldcs(W + nb * 16 + sub * 2 + 1);
         }
-        float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         float c = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) c = fmaxf(c, fabsf(v[i]));
@@ -47,28 +75,29 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
         c = fmaxf(c, __shfl_xor_sync(0xFFFFFFFFu, c, 2));
         c = fmaxf(c, __shfl_xor_sync(0xFFFFFFFFu, c, 4));
         uint32_t word = 0;
+        if (c == 0.0f) {
+            word = 0x77777777u;  // all-zero block: every element is the exact-zero level
+        } else if (c >= 0x1p-96f) {
+            const float y = __frcp_rn(c);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t code;
-            if (c == 0.0f) {
-                code = 7u;  // all-zero block: every element is the exact-zero level
-            } else {
-                const float q = __fdiv_rn(v[i], c);
-                int k = (q > sM[7]) ? 8 : 0;
-                k += (q > sM[k + 3]) ? 4 : 0;
-                k += (q > sM[k + 1]) ? 2 : 0;
-                k += (q > sM[k]) ? 1 : 0;
-                code = static_cast<uint32_t>(k);
+            for (int i = 0; i < 8; ++i) {
+                const float q0 = __fmul_rn(v[i], y);
+                const float rem = __fmaf_rn(-c, q0, v[i]);
+                const float q = __fmaf_rn(rem, y, q0);
+                word |= nf4_code(q, sM) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
             }
-            // element 2j -> high nibble of byte j; bytes little-endian in the word
-            const int byte = i >> 1;
-            const int shift = 8 * byte + ((i & 1) ? 0 : 4);
-            word |= code << shift;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                word |= nf4_code(__fdiv_rn(v[i], c), sM) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
         }
+        // element 2j sits in the high nibble of byte j; bytes little-endian in the word
         if (valid) {
             __stcs(codes + b * 8 + sub, word);
             if (sub == 0) absmax[b] = c;
         }
+        x0 = n0;
+        x1 = n1;
     }
 }
 
@@ -169,27 +198,80 @@ __device__ __forceinline__ float decode_constant(const uint8_t* q, const float* 
 }
 
 // ---------------------------------------------------------------------------
-// K3: standalone dequantisation to bf16, one 64-weight block per thread.
+// K3: standalone dequantisation to bf16. A CTA of 128 threads walks chunks of
+// 128 consecutive 64-weight blocks, one block per thread. The next chunk's
+// codes are loaded while the current one is decoded; the 16 KB of bf16 output
+// go to a 128-byte-swizzled shared tile (conflict-free 16-byte stores) that a
+// TMA tensor store writes to global memory as 128 rows of 128 bytes, with two
+// tiles in flight.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint4* __restrict__ codes,
-                                                           const uint8_t* __restrict__ q,
-                                                           const float* __restrict__ s2,
-                                                           const float* __restrict__ mean, int64_t nblocks,
-                                                           uint4* __restrict__ out, Nf4Tables tab) {
+constexpr int kDeqChunk = 128;
+
+__global__ void __launch_bounds__(kDeqChunk) nf4_dequant_kernel(const __grid_constant__ CUtensorMap tm_out,
+                                                                 const uint4* __restrict__ codes,
+                                                                 const uint8_t* __restrict__ q,
+                                                                 const float* __restrict__ s2,
+                                                                 const float* __restrict__ mean, int64_t nblocks,
+                                                                 Nf4Tables tab) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int t = threadIdx.x;
     const float mu = *mean;
-    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
-         b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const uint4 p0 = __ldcs(codes + 2 * b);
-        const uint4 p1 = __ldcs(codes + 2 * b + 1);
-        const Nf4BlockLut lut = make_block_lut(tab.level, decode_constant(q, s2, mu, b));
+    const int64_t nchunks = (nblocks + kDeqChunk - 1) / kDeqChunk;
+
+    // this thread's block of the first chunk: codes, 8-bit constant and group scale
+    int64_t ch = blockIdx.x;
+    uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+    uint32_t pq = 0;
+    float ps2 = 0.0f;
+    if (ch < nchunks && ch * kDeqChunk + t < nblocks) {
+        const int64_t b = ch * kDeqChunk + t;
+        p0 = __ldcs(codes + 2 * b);
+        p1 = __ldcs(codes + 2 * b + 1);
+        pq = q[b];
+        ps2 = s2[b / kGroup];
+    }
+    for (int it = 0; ch < nchunks; ch += gridDim.x, ++it) {
+        const int64_t b = ch * kDeqChunk + t;
+        const int64_t nb = b + static_cast<int64_t>(gridDim.x) * kDeqChunk;
+        // the next chunk's loads are in flight while this one is decoded
+        uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+        uint32_t nq = 0;
+        float ns2 = 0.0f;
+        if (nb < nblocks) {
+            n0 = __ldcs(codes + 2 * nb);
+            n1 = __ldcs(codes + 2 * nb + 1);
+            nq = q[nb];
+            ns2 = s2[nb / kGroup];
+        }
+        const float cprime = (b < nblocks) ? __fmaf_rn(e4m3_to_f32(pq), ps2, mu) : 0.0f;
+        const Nf4BlockLut lut = make_block_lut(tab.level, cprime);
+
+        uint8_t* tile = tiles + (it & 1) * (kDeqChunk * 128);
+        if (t == 0) bulk_wait_read<1>();  // the store issued two chunks ago has left this tile
+        __syncthreads();
+        const uint32_t row = smem_u32(tile) + t * 128;
         const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             uint32_t o[4];
             lut_decode8(lut, words[j], o);
-            __stcs(out + 8 * b + j, make_uint4(o[0], o[1], o[2], o[3]));
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((j ^ (t & 7)) << 4)), "r"(o[0]),
+                         "r"(o[1]), "r"(o[2]), "r"(o[3])
+                         : "memory");
         }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (t == 0) {
+            tma_store_2d(&tm_out, tile, 0, static_cast<int>(ch * kDeqChunk));
+            bulk_commit();
+        }
+        p0 = n0;
+        p1 = n1;
+        pq = nq;
+        ps2 = ns2;
     }
+    if (t == 0) bulk_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -283,13 +365,14 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_sc
     return cudaGetLastError();
 }
 
-cudaError_t launch_nf4_dequant(const uint8_t* codes, const uint8_t* q, const float* s2, const float* mean,
-                               int64_t N, int64_t K, uint16_t* out, const Nf4Tables& tab, int num_sms,
+cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const uint8_t* q, const float* s2,
+                               const float* mean, int64_t N, int64_t K, const Nf4Tables& tab, int num_sms,
                                cudaStream_t st) {
     const int64_t nb = N * K / kBlock;
-    const int grid = grid_for(nb, 256, num_sms * 8);
-    nf4_dequant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), q, s2, mean, nb,
-                                             reinterpret_cast<uint4*>(out), tab);
+    const int64_t nchunks = (nb + kDeqChunk - 1) / kDeqChunk;
+    const int grid = static_cast<int>(std::min<int64_t>(nchunks, static_cast<int64_t>(num_sms) * 6));
+    nf4_dequant_kernel<<<grid, kDeqChunk, kDequantSmem, st>>>(out_map, reinterpret_cast<const uint4*>(codes), q, s2,
+                                                               mean, nb, tab);
     return cudaGetLastError();
 }
 

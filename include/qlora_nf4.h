@@ -191,6 +191,9 @@ const char* qlora_last_error(void);
 #define QLORA_OPT_STALL_PRODUCER  4
 #define QLORA_OPT_LAUNCH_COUNT    5  /* read: kernels launched by this library so
                                         far in this process; set: reset to value */
+#define QLORA_OPT_SKINNY_MAX_SPLITS 6 /* tuning: cap on the reduction splits of
+                                        the rank-r matmuls (0 = no cap; a cap
+                                        only lowers them, workspaces stay valid) */
 qlora_status qlora_set_option(int option, int64_t value);
 int64_t qlora_get_option(int option);
 

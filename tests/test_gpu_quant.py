@@ -153,3 +153,30 @@ def test_e4m3_cvt_matches_oracle_sweep(q):
     want = oracle.e4m3_encode_array(x)
     bad = np.flatnonzero(got != want)
     assert bad.size == 0, (x[bad[:8]], got[bad[:8]], want[bad[:8]])
+
+
+def near_threshold_weight(nblocks=16384, seed=5):
+    """Blocks whose absmax c is random over the whole exponent range (down to
+    subnormal c) and whose other 63 values sit within +-3 ulps of c times a
+    decision threshold or a level: the places where v = w / c must be
+    rounded exactly for the nearest-level decision to be right."""
+    rng = np.random.default_rng(seed)
+    _, L = oracle.nf4_levels()
+    M = oracle.midpoints(L)
+    pts = np.concatenate([M, L]).astype(np.float32)
+    e = rng.integers(-140, 20, nblocks)
+    c = np.ldexp(1.0 + rng.random(nblocks), e).astype(np.float32)
+    W = np.empty((nblocks, 64), np.float32)
+    W[:, 0] = c * np.where(rng.random(nblocks) < 0.5, 1, -1).astype(np.float32)
+    base = (pts[rng.integers(0, pts.size, (nblocks, 63))] * c[:, None]).astype(np.float32)
+    bits = base.view(np.int32) + rng.integers(-3, 4, base.shape).astype(np.int32)
+    vals = bits.view(np.float32)
+    vals = np.where(np.isfinite(vals) & (np.abs(vals) <= c[:, None]), vals, base)
+    W[:, 1:] = vals
+    return W.reshape(256, -1)
+
+
+def test_encoder_near_thresholds_bit_exact(q):
+    W = near_threshold_weight()
+    ref = oracle.quantize_nf4(W)
+    assert_quant_equal(gpu_quant(q, W), ref)
