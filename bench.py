@@ -262,29 +262,47 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: K whole steps, events around each fused matmul too
+    # ---- eager timing (host launches every kernel): reported for reference
+    n_eager = min(args.steps, 200)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    h0 = time.perf_counter()
+    for i in range(n_eager):
+        step(i)
+    host_ms = (time.perf_counter() - h0) * 1e3 / n_eager  # host enqueue time per step
+    e1.record()
+    torch.cuda.synchronize()
+    eager_ms = e0.elapsed_time(e1) / n_eager
+
+    # ---- timed region: the K steps, every kernel of every step, replayed from
+    # one captured CUDA graph (no host launch gaps); each step records its own
+    # events around the two fused matmuls
     prof = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
             for _ in range(args.steps)]
     for pair in prof:  # torch creates events lazily: make them exist before the library records them
         for a, b in pair:
             a.record()
             b.record()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     launches0 = q.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.steps):
+            step(i, prof[i])
+    launches = q.launch_count() - launches0
+    graph.replay()  # one untimed replay of the whole graph
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
     time.sleep(0.15)
     barrier()
     torch.cuda.synchronize()
     start.record()
-    h0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i, prof[i])
-    host_ms = (time.perf_counter() - h0) * 1e3 / args.steps  # host enqueue time per step
+    graph.replay()
     stop.record()
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    launches = q.launch_count() - launches0
     ms = start.elapsed_time(stop) / args.steps
     if pg is not None:
         t = torch.tensor([ms], device=dev)
@@ -292,6 +310,7 @@ def run_ours(args, rank, world, local_rank):
         ms = float(t.item())
     fwd_ms = statistics.mean(p[0][0].elapsed_time(p[0][1]) for p in prof)
     dx_ms = statistics.mean(p[1][0].elapsed_time(p[1][1]) for p in prof)
+    del graph
 
     # ---- per-row breakdown (outside the timed region, same inputs): each row
     # is captured n times into a CUDA graph and the replay is timed, so the
@@ -358,6 +377,37 @@ def run_ours(args, rank, world, local_rank):
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
+    # ---- the other rows of the path on their own workloads (graph-timed,
+    # outside the timed region): the small-batch sweep forward and the
+    # quantiser / dequantiser on the large weights
+    sweep = {}
+    if not args.no_sweep and rank == 0:
+        pk_hbm = peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        by_shape = {}
+        for c in synth.SWEEP:
+            key = (c.N, c.K)
+            if key not in by_shape:
+                Wc = synth.weight(c).to(dev)
+                wc = q.quantize_nf4(Wc)
+                Wbc = torch.empty(c.N, c.K, dtype=torch.bfloat16, device=dev)
+                tq = timed(lambda i: q.quantize_nf4(Wc, out=wc), n=10)
+                td = timed(lambda i: q.dequantize_nf4(wc, out=Wbc), n=10)
+                qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
+                sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
+                sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}
+                del Wbc
+                by_shape[key] = (Wc, wc)
+            Wc, wc = by_shape[key]
+            Xc, Ac, Bc = synth.activations(c).to(dev), synth.lora_a(c).to(dev), synth.lora_b(c).to(dev)
+            Yc = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+            sTc = torch.empty(c.M, c.r, dtype=torch.bfloat16, device=dev)
+            wsc = torch.empty(q.workspace_bytes(q.OP_FWD, c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
+            tf = timed(lambda i: q.linear_fwd(Xc, wc, Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc))
+            gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
+            sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm}
+        by_shape.clear()
+        torch.cuda.empty_cache()
+
     flops = fwd_bwd_flops(M, N, K, r)
     value = flops * world / (ms * 1e-3) / 1e12
     pk, pk_kind = peaks()
@@ -375,6 +425,8 @@ def run_ours(args, rank, world, local_rank):
         "tokens_per_s": M * world / (ms * 1e-3),
         "dequant_gbs": deq_bytes / (rows_ms["dequantize"] * 1e-3) / 1e9,
         "rows_ms": rows_ms,
+        "timing": "timed steps replayed from one CUDA graph holding all K steps",
+        "eager_ms_per_step": eager_ms,
         "host_enqueue_ms_per_step": host_ms,
         "kernels_ms": {"fused_forward": fwd_ms, "fused_dx": dx_ms},
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -383,6 +435,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
+        "other_rows": sweep,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -402,6 +455,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the small-batch / quantiser rows")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

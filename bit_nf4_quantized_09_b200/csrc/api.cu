@@ -252,11 +252,11 @@ Split split_for(int64_t tiles, int64_t red) {
     return Split{static_cast<int>(s), static_cast<int>(steps)};
 }
 
-// K splits of the small-batch kernel: at most two waves of two CTAs per SM
+// K splits of the small-batch kernel: at most two waves of three CTAs per SM
 // (on 148 SMs), the best wave fill, and fp32 partials no larger than a
 // quarter of the packed weight.
 Split gemv_split(int64_t M, int64_t N, int64_t K) {
-    const int64_t KT = K / 64, tiles = cdiv(N, 128), slots = kTargetCtas;
+    const int64_t KT = K / 64, tiles = cdiv(N, 128), slots = 3 * 148;
     const int64_t smax = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(KT, 64), K / (32 * std::max<int64_t>(M, 1))));
     int64_t best = 1;
     double best_eff = -1.0;
@@ -583,9 +583,9 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         if (injected_failure()) return QLORA_ERR_CUDA;
         cudaEvent_t ev0, ev1;
         take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-        if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+        if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
         QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
-        if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+        if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
         return QLORA_OK;
     }
 
@@ -609,9 +609,9 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     if (injected_failure()) return QLORA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-    if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+    if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
     QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused forward");
-    if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+    if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
     return QLORA_OK;
 }
 
@@ -685,9 +685,9 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     if (injected_failure()) return QLORA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
-    if (ev0) QLORA_TRY(cudaEventRecord(ev0, st), "profile event");
+    if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
     QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused dX");
-    if (ev1) QLORA_TRY(cudaEventRecord(ev1, st), "profile event");
+    if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
 
     // dA = sU^T X (as dA^T[K, r] = X^T sU) and dB = dY^T sT, split over tokens
     CUtensorMap ta0, tb0, ta1, tb1;

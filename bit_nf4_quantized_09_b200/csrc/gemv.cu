@@ -32,7 +32,7 @@ namespace {
 constexpr uint32_t kCodeTile = 128 * 32;    // 4 KB packed
 constexpr uint32_t kCTile = 128 * 4;        // 512 B constants
 constexpr int kMaxInStages = 10;
-constexpr uint32_t kInBudget = 72 * 1024;
+constexpr uint32_t kInBudget = 40 * 1024;  // with the 32 KB ring: three CTAs per SM
 constexpr uint32_t kWTile = 128 * 64 * 2;   // 16 KB dequantised bf16
 constexpr int kWStages = 2;
 constexpr uint32_t kWOff = kInBudget;
@@ -74,7 +74,7 @@ __device__ __forceinline__ float lora_dot(const uint16_t* sT, const uint16_t* b,
     return acc;
 }
 
-__global__ void __launch_bounds__(kGemvThreads, 2)
+__global__ void __launch_bounds__(kGemvThreads, 3)
     gemv_nf4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
                     const __grid_constant__ CUtensorMap tm_c, const GemvArgs args, const Nf4Tables tab) {
     extern __shared__ uint8_t smem_raw[];

@@ -199,7 +199,9 @@ int64_t qlora_get_option(int option);
 
 /* Profiling hook: record the CUDA events ev_start / ev_stop (cudaEvent_t,
  * owned by the caller) on the launch stream immediately before and after the
- * next launch of the named kernel; the request is consumed by that launch. */
+ * next launch of the named kernel; the request is consumed by that launch.
+ * The records are external event records, so inside a captured CUDA graph
+ * they become event-record nodes that time every replay. */
 #define QLORA_KERNEL_FUSED_FWD 1   /* the dequant-fused forward matmul (the
                                       small-batch kernel when M <= 64)        */
 #define QLORA_KERNEL_FUSED_DX  2   /* the transposed-dequant dX matmul       */
