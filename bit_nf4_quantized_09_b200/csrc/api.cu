@@ -25,6 +25,7 @@ std::atomic<int64_t> g_timeout_us{1000000};
 std::atomic<int64_t> g_stall_producer{0};
 std::atomic<int64_t> g_launch_count{0};
 std::atomic<int64_t> g_skinny_max_splits{0};
+std::atomic<int64_t> g_reg_gemv_max_m{16};
 thread_local std::string g_last_error;
 
 // One-shot event requests of qlora_profile_next_launch, per kernel id.
@@ -156,7 +157,7 @@ qlora_status device_ready(int* sms_out) {
                            std::to_string(minor) + ")";
             d.status = QLORA_ERR_UNSUPPORTED_DEVICE;
         } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess ||
-                   (e = gemv_init_device()) != cudaSuccess) {
+                   (e = gemv_init_device()) != cudaSuccess || (e = gemv_mma_init_device()) != cudaSuccess) {
             d.status = cuda_fail(e, "cudaFuncSetAttribute");
         } else if (!g_encode) {
             void* fn = nullptr;
@@ -238,6 +239,7 @@ int rank_pad(int r) { return r < 16 ? 16 : r; }
 // Reduction splits of a skinny matmul: enough CTAs for two per SM of a
 // 148-SM B200 (fixed so workspace sizes do not depend on the device).
 constexpr int64_t kTargetCtas = 296;
+constexpr int kPlanSms = 148;  // the SM count the split plans are tuned for (any count runs them)
 struct Split {
     int splits;
     int steps;
@@ -285,6 +287,7 @@ struct Layout {
     size_t total = 0;
     int64_t ldc = 0;
     Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1}, gemv{1, 1};
+    GemvMmaPlan reg_gemv{1, 1, 4, 1};
 };
 
 Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
@@ -312,8 +315,14 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     if (op == QLORA_OP_FWD) {
         L.partT = take(static_cast<size_t>(L.sT_split.splits) * M * NR * 4);
         if (M <= kGemvMaxM) {
+            // either small-batch kernel may run (the choice is a runtime option)
             L.gemv = gemv_split(M, N, K);
-            L.partY = take(static_cast<size_t>(L.gemv.splits) * M * N * 4);
+            size_t part = static_cast<size_t>(L.gemv.splits) * M * N * 4;
+            if (M <= kGemvMmaMaxM) {
+                L.reg_gemv = gemv_mma_plan(M, N, K, kPlanSms);
+                part = std::max(part, static_cast<size_t>(L.reg_gemv.max_parts) * M * N * 4);
+            }
+            L.partY = take(part);
         }
     } else {
         L.sU_split = split_for(mtiles, N);
@@ -326,6 +335,16 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     }
     L.total = off;
     return L;
+}
+
+// A profiling event record; inside stream capture it becomes an external
+// event-record node, so it also times every replay of the captured graph.
+cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return e;
+    return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                                               : cudaEventRecord(ev, st);
 }
 
 qlora_status check_weight(const qlora_nf4_weight* w) {
@@ -458,6 +477,7 @@ qlora_status qlora_set_option(int option, int64_t value) {
             if (value < 0) return QLORA_ERR_INVALID_ARG;
             g_skinny_max_splits = value;
             return QLORA_OK;
+        case QLORA_OPT_REG_GEMV_MAX_M: g_reg_gemv_max_m = value; return QLORA_OK;
         default: return QLORA_ERR_INVALID_ARG;
     }
 }
@@ -470,6 +490,7 @@ int64_t qlora_get_option(int option) {
         case QLORA_OPT_STALL_PRODUCER: return g_stall_producer.load();
         case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
         case QLORA_OPT_SKINNY_MAX_SPLITS: return g_skinny_max_splits.load();
+        case QLORA_OPT_REG_GEMV_MAX_M: return g_reg_gemv_max_m.load();
         default: return -1;
     }
 }
@@ -550,12 +571,47 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
 
     QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
     if (injected_failure()) return QLORA_ERR_CUDA;
+    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
+    if (M <= small && M <= std::min<int64_t>(g_reg_gemv_max_m.load(), kGemvMmaMaxM)) {
+        // few tokens: rank-r down-projection, then the register-fed GEMV,
+        // launched as its programmatic dependent so the weight stream starts
+        // while sT is still being computed
+        if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
+                           status, st)) != QLORA_OK)
+            return s;
+        GemvMmaArgs ga{};
+        ga.X = X;
+        ga.codes = w->codes;
+        ga.qabsmax = w->qabsmax;
+        ga.s2 = w->s2;
+        ga.mean = w->mean;
+        ga.M = M;
+        ga.N = N;
+        ga.K = K;
+        ga.r = r;
+        ga.ctas = L.reg_gemv.ctas;
+        ga.units = L.reg_gemv.units;
+        ga.max_chunks = L.reg_gemv.max_chunks;
+        ga.part = reinterpret_cast<float*>(base + L.partY);
+        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
+        ga.sT = sT;
+        ga.B = B;
+        ga.Y = Y;
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        cudaEvent_t ev0, ev1;
+        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
+        // an event record between the two launches would break the
+        // programmatic edge, so a profiled call launches in plain order
+        QLORA_LAUNCH(launch_gemv_mma(ga, tables(), ev0 == nullptr, st), 1, "register gemv");
+        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
+        return QLORA_OK;
+    }
     QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
     if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
                        status, st)) != QLORA_OK)
         return s;
 
-    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
     if (M <= small) {
         // few tokens: weight-streaming swap-AB kernel, split over K
         const int Mp = static_cast<int>((M + 15) / 16 * 16);
@@ -583,9 +639,9 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         if (injected_failure()) return QLORA_ERR_CUDA;
         cudaEvent_t ev0, ev1;
         take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-        if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
+        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
         QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
-        if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
+        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
         return QLORA_OK;
     }
 
@@ -609,9 +665,9 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     if (injected_failure()) return QLORA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-    if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
+    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
     QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused forward");
-    if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
+    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
     return QLORA_OK;
 }
 
@@ -685,9 +741,9 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     if (injected_failure()) return QLORA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
-    if (ev0) QLORA_TRY(cudaEventRecordWithFlags(ev0, st, cudaEventRecordExternal), "profile event");
+    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
     QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused dX");
-    if (ev1) QLORA_TRY(cudaEventRecordWithFlags(ev1, st, cudaEventRecordExternal), "profile event");
+    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
 
     // dA = sU^T X (as dA^T[K, r] = X^T sU) and dB = dY^T sT, split over tokens
     CUtensorMap ta0, tb0, ta1, tb1;

@@ -112,6 +112,37 @@ __device__ __forceinline__ void lut_decode8(const Nf4BlockLut& t, uint32_t packe
     }
 }
 
+// prmt.b32 in its default mode: a selector nibble with bit 3 set yields the
+// sign bit of the byte it picks, replicated over the whole output byte.
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// lut_decode8 with the byte masks taken straight from the packed word: the
+// top bit of a high-nibble code is bit 7 of its byte, and that of a
+// low-nibble code is bit 7 of the same byte shifted left by 4, so one
+// sign-replicating permute yields the four 0x00/0xFF masks of a half.
+__device__ __forceinline__ void lut_decode8_sx(const Nf4BlockLut& t, uint32_t packed, uint32_t (&out)[4]) {
+    const uint32_t idx = packed & 0x77777777u;
+    const uint32_t p4 = packed << 4;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = h ? (idx >> 16) : idx;
+        // output bytes [e1, e0, e3, e2] (h = 0) or [e5, e4, e7, e6] (h = 1)
+        const uint32_t m = prmt_sx(p4, packed, h ? 0xFBEAu : 0xD9C8u);
+        const uint32_t loA = __byte_perm(t.lo[0], t.lo[1], sel);
+        const uint32_t loB = __byte_perm(t.lo[2], t.lo[3], sel);
+        const uint32_t hiA = __byte_perm(t.hi[0], t.hi[1], sel);
+        const uint32_t hiB = __byte_perm(t.hi[2], t.hi[3], sel);
+        const uint32_t lo = (loA & ~m) | (loB & m);
+        const uint32_t hi = (hiA & ~m) | (hiB & m);
+        out[2 * h + 0] = __byte_perm(lo, hi, 0x4051);
+        out[2 * h + 1] = __byte_perm(lo, hi, 0x6273);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

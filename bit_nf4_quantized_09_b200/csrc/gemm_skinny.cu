@@ -52,6 +52,9 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     skinny_gemm(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
                 const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                 const SkinnyArgs args) {
+    // a launch that depends on this one programmatically may be scheduled
+    // now; it waits for this grid's completion before reading its output
+    asm volatile("griddepcontrol.launch_dependents;");
     const int prob = blockIdx.z;
     const SkinnyProblem P = args.p[prob];
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;

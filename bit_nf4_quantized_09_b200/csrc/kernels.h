@@ -87,6 +87,41 @@ struct GemvArgs {
 cudaError_t launch_gemv(const CUtensorMap& x, const CUtensorMap& codes, const CUtensorMap& cT, const GemvArgs& a,
                         const Nf4Tables& tab, cudaStream_t st);
 
+// ------------------------------------- small-batch register-fed MMA GEMV --
+constexpr int kGemvMmaMaxM = 32;  // tokens: up to four n8 MMA tiles
+
+struct GemvMmaArgs {
+    const uint16_t* X;       // bf16 [M, K]
+    const uint8_t* codes;    // packed NF4 [N, K/2]
+    const uint8_t* qabsmax;  // E4M3 [N*K/64]
+    const float* s2;         // [groups]
+    const float* mean;       // [1]
+    int64_t M, N, K;
+    int r;                   // LoRA rank
+    int ctas;                // grid size (from the plan)
+    int64_t units;           // (N/128 row tiles) * (K/64 block columns)
+    int max_chunks;          // staged X chunks per CTA (from the plan)
+    float* part;             // fp32 [max_parts][M][N] partial sums
+    int* counter;            // [N/128 row tiles] tickets, zero before the launch; left zero
+    const uint16_t* sT;      // bf16 [M, r], read only in the epilogue
+    const uint16_t* B;       // bf16 [N, r]
+    uint16_t* Y;             // bf16 [M, N]
+};
+
+struct GemvMmaPlan {
+    int ctas;
+    int64_t units;
+    int max_chunks;
+    int max_parts;  // partial-sum slots per row tile
+};
+
+GemvMmaPlan gemv_mma_plan(int64_t M, int64_t N, int64_t K, int num_sms);
+size_t gemv_mma_smem_bytes(int64_t M, int max_chunks);
+cudaError_t gemv_mma_init_device();
+// pdl: launch as the programmatic dependent of the previous launch on the
+// stream (the kernel waits for it before reading sT).
+cudaError_t launch_gemv_mma(const GemvMmaArgs& a, const Nf4Tables& tab, bool pdl, cudaStream_t st);
+
 // ---------------------------------------------------------- skinny GEMMs --
 // D[rows, NR] = sum over the reduction of A_op[rows, red] * B_op[NR, red]^T,
 // split over the reduction (grid.y); the last CTA of each 128-row tile adds

@@ -194,6 +194,10 @@ const char* qlora_last_error(void);
 #define QLORA_OPT_SKINNY_MAX_SPLITS 6 /* tuning: cap on the reduction splits of
                                         the rank-r matmuls (0 = no cap; a cap
                                         only lowers them, workspaces stay valid) */
+#define QLORA_OPT_REG_GEMV_MAX_M  7  /* token count up to which the small-batch
+                                        forward decodes in registers and feeds
+                                        mma.sync (default 16, maximum 32; 0 =
+                                        always the tcgen05 small-batch kernel) */
 qlora_status qlora_set_option(int option, int64_t value);
 int64_t qlora_get_option(int option);
 

@@ -213,3 +213,60 @@ def test_small_batch_matches_tiled_path(q):
     e = oracle.rel_err(f64(Ys), f64(Yt))
     print(f"small-batch vs tiled: {e:.3e}")
     assert e <= 2 ** -7
+
+
+# ------------------------------ register-fed small-batch GEMV (M <= 32) ---
+
+REG = [synth.custom(N=128, K=64 * 37, M=1, r=8),       # one row tile, ten ragged K splits
+       synth.custom(N=8, K=64, M=2, r=16),             # one block, rows past N
+       synth.custom(N=136, K=320, M=7, r=32),
+       synth.custom(N=264, K=1088, M=8, r=64, outliers=True),
+       synth.custom(N=1032, K=576, M=9, r=16),
+       synth.custom(N=520, K=4160, M=16, r=8),
+       synth.custom(N=776, K=1024, M=23, r=16),
+       synth.custom(N=4096, K=1024, M=32, r=64)]
+
+
+def small_forward(q, cfg, t, reg_max):
+    w = q.quantize_nf4(t["W"].cuda())
+    old = q.get_option(q.OPT_REG_GEMV_MAX_M)
+    try:
+        q.set_option(q.OPT_REG_GEMV_MAX_M, reg_max)
+        Y, sT = q.linear_fwd(t["X"].cuda(), w, t["A"].cuda(), t["B"].cuda(), cfg.alpha)
+    finally:
+        q.set_option(q.OPT_REG_GEMV_MAX_M, old)
+    torch.cuda.synchronize()
+    return Y, sT
+
+
+@pytest.mark.parametrize("cfg", REG, ids=lambda c: c.name)
+def test_register_gemv_forward(q, cfg):
+    """Token counts across one to four n8 MMA tiles, N not a multiple of the
+    16-row warp tile, K slices that end inside a four-block step."""
+    t = inputs(cfg)
+    Y, sT = small_forward(q, cfg, t, 32)
+    What = oracle_what(t["W"])
+    Yr, T = oracle.forward(f64(t["X"]), What, f64(t["A"]), f64(t["B"]), cfg.alpha, cfg.r)
+    check("Y", f64(Y), Yr)
+    check("sT", f64(sT), (cfg.alpha / cfg.r) * T)
+
+
+def test_register_gemv_matches_tcgen05_small_path(q):
+    """The register-fed kernel against the tcgen05 small-batch kernel on the
+    same inputs; both add fp32 products of the same bf16 weights."""
+    cfg = synth.custom(N=4096, K=2048, M=16, r=16)
+    t = inputs(cfg)
+    Yr, sTr = small_forward(q, cfg, t, 32)
+    Yt, sTt = small_forward(q, cfg, t, 0)
+    assert torch.equal(sTr, sTt)
+    e = oracle.rel_err(f64(Yr), f64(Yt))
+    print(f"register vs tcgen05 small path: {e:.3e}")
+    assert e <= 2 ** -7
+
+
+def test_register_gemv_deterministic(q):
+    cfg = synth.custom(N=2048, K=4096, M=4, r=16)
+    t = inputs(cfg)
+    a, _ = small_forward(q, cfg, t, 32)
+    b, _ = small_forward(q, cfg, t, 32)
+    assert torch.equal(a, b)
