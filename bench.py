@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -383,28 +384,47 @@ def run_ours(args, rank, world, local_rank):
     sweep = {}
     if not args.no_sweep and rank == 0:
         pk_hbm = peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         by_shape = {}
         for c in synth.SWEEP:
             key = (c.N, c.K)
             if key not in by_shape:
+                # enough packed copies that the rotation over them is larger
+                # than twice the L2, so every timed call streams from HBM
                 Wc = synth.weight(c).to(dev)
-                wc = q.quantize_nf4(Wc)
+                ncopy = max(2, math.ceil(2 * l2 / (c.N * c.K * (0.5 + 1 / 64))))
+                wcs = [q.quantize_nf4(Wc) for _ in range(ncopy)]
                 Wbc = torch.empty(c.N, c.K, dtype=torch.bfloat16, device=dev)
-                tq = timed(lambda i: q.quantize_nf4(Wc, out=wc), n=10)
-                td = timed(lambda i: q.dequantize_nf4(wc, out=Wbc), n=10)
+                tq = timed(lambda i: q.quantize_nf4(Wc, out=wcs[i % ncopy]), n=10)
+                td = timed(lambda i: q.dequantize_nf4(wcs[i % ncopy], out=Wbc), n=10)
                 qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
                 sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
                 sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}
-                del Wbc
-                by_shape[key] = (Wc, wc)
-            Wc, wc = by_shape[key]
+                del Wbc, Wc
+                by_shape[key] = wcs
+            wcs = by_shape[key]
+            ncopy = len(wcs)
             Xc, Ac, Bc = synth.activations(c).to(dev), synth.lora_a(c).to(dev), synth.lora_b(c).to(dev)
             Yc = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
             sTc = torch.empty(c.M, c.r, dtype=torch.bfloat16, device=dev)
             wsc = torch.empty(q.workspace_bytes(q.OP_FWD, c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
-            tf = timed(lambda i: q.linear_fwd(Xc, wc, Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc))
+            tf = timed(lambda i: q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc))
+            # the weight-streaming kernel alone (events around it; a profiled
+            # call launches it in plain stream order)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+            for e in evs:
+                e[0].record()
+                e[1].record()
+            for i, e in enumerate(evs):
+                q.profile_next_launch(q.KERNEL_FUSED_FWD, e[0], e[1])
+                q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc)
+            torch.cuda.synchronize()
+            tk = statistics.median(e[0].elapsed_time(e[1]) for e in evs[3:])
             gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
-            sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm}
+            wb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384)
+            sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm,
+                             "weight_kernel_us": tk * 1e3, "weight_kernel_GBs": wb / tk / 1e6,
+                             "weight_kernel_frac_hbm": wb / tk / 1e6 / pk_hbm}
         by_shape.clear()
         torch.cuda.empty_cache()
 

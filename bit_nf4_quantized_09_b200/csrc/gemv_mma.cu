@@ -37,14 +37,14 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsCta = kWarps * 16;
-constexpr uint32_t kChunk = 136;  // bytes per 64 X elements in shared memory (128 + 8 pad)
+constexpr uint32_t kChunk = 144;  // bytes per 64 X elements in shared memory (128 + 16 pad)
 
-// Row pitch of the staged X slice: 136-byte chunks, the pitch congruent to
-// 32 mod 128 bytes, so the 64-bit fragment reads of one half-warp (4 token
-// rows x 4 lanes q) fall on 16 distinct bank pairs.
+// Row pitch of the staged X slice: 144-byte chunks and a pitch congruent to
+// 64 mod 128 bytes, so the 16-byte fragment reads of a quarter warp (2 token
+// rows x 4 lanes q) fall on 8 distinct groups of 4 banks.
 __host__ __device__ constexpr uint32_t x_pitch(int chunks) {
     const uint32_t raw = static_cast<uint32_t>(chunks) * kChunk;
-    return (raw + 95u) / 128u * 128u + 32u;
+    return (raw + 63u) / 128u * 128u + 64u;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -263,14 +263,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
             uint32_t oa[4], ob[4];
             lut_decode8_sx(la, wa[w], oa);
             lut_decode8_sx(lb, wb[w], ob);
+            // X fragments of MMA steps 2w and 2w + 1: 16 contiguous bytes
+            uint4 bx[MT];
+#pragma unroll
+            for (int t = 0; t < MT; ++t) bx[t] = *reinterpret_cast<const uint4*>(xstep + xtok[t] + 16 * w);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t af[4] = {oa[2 * h], ob[2 * h], oa[2 * h + 1], ob[2 * h + 1]};
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    const uint2 bx = *reinterpret_cast<const uint2*>(xstep + xtok[t] + 8 * (2 * w + h));
-                    mma_bf16(acc[t], af, bx.x, bx.y);
-                }
+                for (int t = 0; t < MT; ++t) mma_bf16(acc[t], af, h ? bx[t].z : bx[t].x, h ? bx[t].w : bx[t].y);
             }
         }
         if (gi == it0 - 1 || gi == it_all - 1) {
