@@ -212,6 +212,84 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ ours ---
 
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one
+# ncu capture of the current kernel on this workload (attn7B forward:
+# 43.35 MB read, 1.96 MB written; Y is still in L2 when the kernel ends).
+# Kernels without a capture of their current version report null.
+NCU_TRAFFIC = {"fused_forward": 45.32e6}
+
+
+def timed(fn, n=20):
+    """Mean ms per call of fn(i), i = 0..n-1, replayed from one CUDA graph."""
+    fn(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / n
+
+
+def other_rows(q, dev):
+    """The other rows of the path on their own workloads (graph-timed): the
+    quantiser and dequantiser on the large weights and the small-batch
+    forward sweep, each streaming from HBM (rotated weight copies)."""
+    sweep = {}
+    pk_hbm = peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    by_shape = {}
+    for c in synth.SWEEP:
+        key = (c.N, c.K)
+        if key not in by_shape:
+            # enough packed copies that the rotation over them is larger
+            # than twice the L2, so every timed call streams from HBM
+            Wc = synth.weight(c).to(dev)
+            ncopy = max(2, math.ceil(2 * l2 / (c.N * c.K * (0.5 + 1 / 64))))
+            wcs = [q.quantize_nf4(Wc) for _ in range(ncopy)]
+            Wbc = torch.empty(c.N, c.K, dtype=torch.bfloat16, device=dev)
+            tq = timed(lambda i: q.quantize_nf4(Wc, out=wcs[i % ncopy]), n=10)
+            td = timed(lambda i: q.dequantize_nf4(wcs[i % ncopy], out=Wbc), n=10)
+            qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
+            sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
+            sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}
+            del Wbc, Wc
+            by_shape[key] = wcs
+        wcs = by_shape[key]
+        ncopy = len(wcs)
+        Xc, Ac, Bc = synth.activations(c).to(dev), synth.lora_a(c).to(dev), synth.lora_b(c).to(dev)
+        Yc = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        sTc = torch.empty(c.M, c.r, dtype=torch.bfloat16, device=dev)
+        wsc = torch.empty(q.workspace_bytes(q.OP_FWD, c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
+        tf = timed(lambda i: q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc))
+        # the weight-streaming kernel alone (events around it; a profiled
+        # call launches it in plain stream order)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+        for e in evs:
+            e[0].record()
+            e[1].record()
+        for i, e in enumerate(evs):
+            q.profile_next_launch(q.KERNEL_FUSED_FWD, e[0], e[1])
+            q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc)
+        torch.cuda.synchronize()
+        tk = statistics.median(e[0].elapsed_time(e[1]) for e in evs[3:])
+        gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
+        wb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384)
+        sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm,
+                         "weight_kernel_us": tk * 1e3, "weight_kernel_GBs": wb / tk / 1e6,
+                         "weight_kernel_frac_hbm": wb / tk / 1e6 / pk_hbm}
+    by_shape.clear()
+    torch.cuda.empty_cache()
+    return sweep
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_nf4_quantized_09_b200 as q
 
@@ -316,23 +394,6 @@ def run_ours(args, rank, world, local_rank):
     # ---- per-row breakdown (outside the timed region, same inputs): each row
     # is captured n times into a CUDA graph and the replay is timed, so the
     # numbers are GPU time without host launch gaps
-    def timed(fn, n=20):
-        fn(0)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(n):
-                fn(i)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        del g
-        return e0.elapsed_time(e1) / n
-
     rows_ms = {
         "quantize": timed(lambda i: q.quantize_nf4(sets[i % 2]["W"], out=w, ws=ws_q)),
         "dequantize": timed(lambda i: q.dequantize_nf4(w, out=Wbf)),
@@ -381,52 +442,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- the other rows of the path on their own workloads (graph-timed,
     # outside the timed region): the small-batch sweep forward and the
     # quantiser / dequantiser on the large weights
-    sweep = {}
-    if not args.no_sweep and rank == 0:
-        pk_hbm = peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-        by_shape = {}
-        for c in synth.SWEEP:
-            key = (c.N, c.K)
-            if key not in by_shape:
-                # enough packed copies that the rotation over them is larger
-                # than twice the L2, so every timed call streams from HBM
-                Wc = synth.weight(c).to(dev)
-                ncopy = max(2, math.ceil(2 * l2 / (c.N * c.K * (0.5 + 1 / 64))))
-                wcs = [q.quantize_nf4(Wc) for _ in range(ncopy)]
-                Wbc = torch.empty(c.N, c.K, dtype=torch.bfloat16, device=dev)
-                tq = timed(lambda i: q.quantize_nf4(Wc, out=wcs[i % ncopy]), n=10)
-                td = timed(lambda i: q.dequantize_nf4(wcs[i % ncopy], out=Wbc), n=10)
-                qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
-                sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
-                sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}
-                del Wbc, Wc
-                by_shape[key] = wcs
-            wcs = by_shape[key]
-            ncopy = len(wcs)
-            Xc, Ac, Bc = synth.activations(c).to(dev), synth.lora_a(c).to(dev), synth.lora_b(c).to(dev)
-            Yc = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
-            sTc = torch.empty(c.M, c.r, dtype=torch.bfloat16, device=dev)
-            wsc = torch.empty(q.workspace_bytes(q.OP_FWD, c.M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
-            tf = timed(lambda i: q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc))
-            # the weight-streaming kernel alone (events around it; a profiled
-            # call launches it in plain stream order)
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
-            for e in evs:
-                e[0].record()
-                e[1].record()
-            for i, e in enumerate(evs):
-                q.profile_next_launch(q.KERNEL_FUSED_FWD, e[0], e[1])
-                q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc)
-            torch.cuda.synchronize()
-            tk = statistics.median(e[0].elapsed_time(e[1]) for e in evs[3:])
-            gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
-            wb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384)
-            sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm,
-                             "weight_kernel_us": tk * 1e3, "weight_kernel_GBs": wb / tk / 1e6,
-                             "weight_kernel_frac_hbm": wb / tk / 1e6 / pk_hbm}
-        by_shape.clear()
-        torch.cuda.empty_cache()
+    sweep = other_rows(q, dev) if (not args.no_sweep and rank == 0) else {}
 
     flops = fwd_bwd_flops(M, N, K, r)
     value = flops * world / (ms * 1e-3) / 1e12
@@ -450,7 +466,9 @@ def run_ours(args, rank, world, local_rank):
         "host_enqueue_ms_per_step": host_ms,
         "kernels_ms": {"fused_forward": fwd_ms, "fused_dx": dx_ms},
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": NCU_TRAFFIC.get(dom),
+                     "traffic_source": "ncu capture of one launch: dram__bytes_read.sum + dram__bytes_write.sum"
+                     if dom in NCU_TRAFFIC else None,
                      "peak_kind": f"bf16 sustained ({pk_kind})"},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -476,6 +494,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-sweep", action="store_true", help="skip the small-batch / quantiser rows")
+    ap.add_argument("--rows-only", action="store_true",
+                    help="only the small-batch / quantiser rows (one JSON line with other_rows), for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -484,6 +504,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.rows_only:
+        import bit_nf4_quantized_09_b200 as q
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"other_rows": other_rows(q, dev)}), flush=True)
     else:
         run_ours(args, rank, world, local_rank)
 
