@@ -281,7 +281,8 @@ Split gemv_split(int64_t M, int64_t N, int64_t K) {
 // call (the kernels also leave their tickets at zero).
 struct Layout {
     size_t header = 0;                                   // bytes cleared per call
-    size_t status = 0, ctrT = 0, ctrU = 0, ctrA = 0, ctrB = 0, ctrY = 0;
+    size_t status = 0, ctrT = 0, ctrU = 0, ctrA = 0, ctrB = 0, ctrY = 0, flags = 0;
+    size_t skpart = 0;                                    // fused matmul: partial tiles of stream-K contributors
     size_t cT = 0, partT = 0, sT = 0, partY = 0;          // forward
     size_t partU = 0, sU = 0, partA = 0;                  // backward (partA holds dA and dB partials)
     size_t total = 0;
@@ -302,7 +303,8 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     L.ctrA = L.ctrU + 4 * static_cast<size_t>(mtiles);
     L.ctrB = L.ctrA + 4 * static_cast<size_t>(ktiles);
     L.ctrY = L.ctrB + 4 * static_cast<size_t>(ntiles);
-    L.header = up256(L.ctrY + 4 * static_cast<size_t>(ntiles));
+    L.flags = L.ctrY + 4 * static_cast<size_t>(ntiles);
+    L.header = up256(L.flags + 4 * static_cast<size_t>(kPlanSms));
     size_t off = L.header;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -310,6 +312,10 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
         return at;
     };
     L.cT = take(static_cast<size_t>(K / kBlock) * L.ldc * 4);
+    // the fused matmul's partial tiles, one per CTA, when it splits tiles
+    L.skpart = take(static_cast<size_t>(fused_partial_ctas(M, op == QLORA_OP_FWD ? N : K, op == QLORA_OP_FWD ? K : N,
+                                                           kPlanSms)) *
+                    kFusedBM * kFusedBN * 4);
     L.sT_split = split_for(mtiles, K);
     L.sT = take(static_cast<size_t>(M) * r * 2);
     if (op == QLORA_OP_FWD) {
@@ -559,7 +565,8 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     const Layout L = layout_for(QLORA_OP_FWD, M, N, K, r);
     if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
     if (injected_failure()) return QLORA_ERR_CUDA;
-    if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* base = static_cast<uint8_t*>(ws);
@@ -658,7 +665,10 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     fa.out_cols = N;
     fa.red = K;
     fa.r = r;
+    fa.ctas = fused_ctas(M, N, K, std::min(sms, kPlanSms));
     fa.out = Y;
+    fa.part = reinterpret_cast<float*>(base + L.skpart);
+    fa.flags = reinterpret_cast<int*>(base + L.flags);
     fa.status = status;
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
@@ -688,7 +698,8 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     const Layout L = layout_for(QLORA_OP_BWD, M, N, K, r);
     if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
     if (injected_failure()) return QLORA_ERR_CUDA;
-    if ((s = device_ready(nullptr)) != QLORA_OK) return s;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (M == 0) {  // an empty batch: the adapter gradients are exactly zero
@@ -734,7 +745,10 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     fa.out_cols = K;
     fa.red = N;
     fa.r = r;
+    fa.ctas = fused_ctas(M, K, N, std::min(sms, kPlanSms));
     fa.out = dX;
+    fa.part = reinterpret_cast<float*>(base + L.skpart);
+    fa.flags = reinterpret_cast<int*>(base + L.flags);
     fa.status = status;
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = 0;

@@ -64,7 +64,65 @@ __device__ __forceinline__ void dequant_block(const Nf4Tables& tab, float cprime
     }
 }
 
-template <bool kTransW>
+// Stream-K schedule. The work is the list of (output tile, 64-deep reduction
+// step) units, tile-major; CTA c (one per SM) takes the contiguous range
+// [c W / P, (c + 1) W / P). Cut at tile boundaries, a range is a list of
+// segments. A segment that starts at step 0 makes its CTA the tile's owner:
+// it also runs the rank-r step and writes the tile. A segment that starts
+// later is a contributor: it writes its fp32 partial tile and raises a flag.
+// Contributions come first in a CTA's range and ownership last, so an owner
+// finds its partials ready, adds them in CTA order (deterministic) and
+// writes the bf16 tile.
+struct Sched {
+    int64_t W;    // tiles * KT
+    int P;        // CTAs
+    int KT;       // reduction steps per tile
+    int tiles_n;  // tiles along the output columns
+    __device__ int64_t begin(int c) const { return static_cast<int64_t>(c) * W / P; }
+    __device__ int cta_of(int64_t u) const { return static_cast<int>(((u + 1) * P - 1) / W); }
+};
+
+// Walks the segments of one CTA's range. Without splitting (kSplit false:
+// one CTA per tile) the range is exactly tile c, all of its steps.
+template <bool kSplit>
+struct SegIter {
+    const Sched& sc;
+    int64_t u, end;
+    int64_t tile;
+    int k_lo, k_hi;
+    __device__ SegIter(const Sched& s, int c)
+        : sc(s), u(kSplit ? s.begin(c) : static_cast<int64_t>(c) * s.KT),
+          end(kSplit ? s.begin(c + 1) : static_cast<int64_t>(c + 1) * s.KT), tile(0), k_lo(0), k_hi(0) {}
+    __device__ bool next() {
+        if (u >= end) return false;
+        if (!kSplit) {
+            tile = u / sc.KT;
+            k_lo = 0;
+            k_hi = sc.KT;
+            u = end;
+            return true;
+        }
+        tile = u / sc.KT;
+        k_lo = static_cast<int>(u - tile * sc.KT);
+        k_hi = static_cast<int>(min(static_cast<int64_t>(sc.KT), end - tile * sc.KT));
+        u = tile * sc.KT + k_hi;
+        return true;
+    }
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <bool kTransW, bool kSplit>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_lact,
@@ -75,24 +133,28 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     uint64_t* deq = full + kFusedStages;
     uint64_t* empty = deq + kFusedStages;
     uint64_t* acc = empty + kFusedStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
+    uint64_t* tmem_free = acc + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_free + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* parts_ok = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kFusedBM;  // first token of the tile
-    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kFusedBN;  // first output column
     const int KT = static_cast<int>((args.red + kFusedBK - 1) / kFusedBK);
+    const int tiles_n = static_cast<int>((args.out_cols + kFusedBN - 1) / kFusedBN);
+    const int tiles_m = static_cast<int>((args.M + kFusedBM - 1) / kFusedBM);
+    const Sched sc{static_cast<int64_t>(tiles_m) * tiles_n * KT, static_cast<int>(gridDim.x), KT, tiles_n};
+    const int cta = blockIdx.x;
     const bool has_lora = args.r > 0;
-    const int steps = KT + (has_lora ? 1 : 0);
     const uint64_t tmo = args.timeout_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFusedStages; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(deq + s, kDequantWarps);  // one arrive per dequant warp
+            mbar_init(deq + s, kDequantWarps);  // one arrive per dequant warp, every step
             mbar_init(empty + s, 1);
         }
         mbar_init(acc, 1);
+        mbar_init(tmem_free, kDequantWarps);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -117,17 +179,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (lane == 0) {
             int last_use[kFusedStages];
             for (int s = 0; s < kFusedStages; ++s) last_use[s] = -1;
-            if (!args.stall_producer) {
-                for (int kt = 0; kt < steps; ++kt) {
-                    const int s = kt % kFusedStages;
-                    const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
-                    if (kt >= kFusedStages && !mbar_wait(empty + s, (u - 1) & 1u, tmo, args.status)) {
+            int g = 0;    // ring position over all steps of all segments
+            int seg = -1;  // segment index
+            SegIter<kSplit> it(sc, cta);
+            while (!args.stall_producer && !*abort_flag && it.next()) {
+                ++seg;
+                const int64_t m0 = (it.tile / tiles_n) * kFusedBM, n0 = (it.tile % tiles_n) * kFusedBN;
+                const int nk = it.k_hi - it.k_lo;
+                const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+                for (int i = 0; i < steps; ++i, ++g) {
+                    const int s = g % kFusedStages;
+                    const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
+                    if (g >= kFusedStages && !mbar_wait(empty + s, (u - 1) & 1u, tmo, args.status)) {
                         *abort_flag = 1;
                         break;
                     }
                     if (*abort_flag) break;
                     uint8_t* st = smem + s * kStageBytes;
-                    if (kt < KT) {
+                    if (i < nk) {
+                        const int kt = it.k_lo + i;
                         mbar_arrive_expect_tx(full + s, kActBytes + kCodeBytes + kCBytes);
                         tma_load_2d(st, &tm_act, full + s, kt * kFusedBK, static_cast<int>(m0));
                         if (!kTransW) {
@@ -140,6 +210,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                             tma_load_2d(st + kOffC, &tm_c, full + s, kt * kFusedBK, static_cast<int>(n0 / kBlock));
                         }
                     } else {
+                        // the rank-r step lands in a weight-tile region, which the
+                        // previous segment's epilogue uses as scratch: wait for it
+                        if (seg > 0 && !mbar_wait(tmem_free, static_cast<uint32_t>(seg - 1) & 1u, tmo, args.status)) {
+                            *abort_flag = 1;
+                            break;
+                        }
                         mbar_arrive_expect_tx(full + s, kActBytes + kWBytes);
                         tma_load_2d(st, &tm_lact, full + s, 0, static_cast<int>(m0));
                         if (!kTransW) {
@@ -162,93 +238,205 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, kFusedBN, false, kTransW);
             bool ok = true;
-            for (int kt = 0; kt < steps; ++kt) {
-                const int s = kt % kFusedStages;
-                const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
-                if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
-                if (kt < KT && !mbar_wait(deq + s, u & 1u, tmo, args.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t act = smem_u32(smem + s * kStageBytes);
-                const uint32_t wt = act + kOffW;
-                const int ksub = (kt < KT) ? (kFusedBK / 16) : (args.r + 15) / 16;
-                for (int kk = 0; kk < ksub; ++kk) {
-                    const uint64_t bdesc = kTransW ? sw128_desc(wt + kk * 2048, 8192, 1024)
-                                                   : sw128_desc(wt + kk * 32, 16, 1024);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint64_t adesc = sw128_desc(act + h * 16384 + kk * 32, 16, 1024);
-                        umma_f16(tmem + h * 256, adesc, bdesc, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-                    }
+            int g = 0, seg = 0;
+            SegIter<kSplit> it(sc, cta);
+            while (ok && it.next()) {
+                // the accumulator must have been read out by the previous epilogue
+                if (seg > 0 && !mbar_wait(tmem_free, static_cast<uint32_t>(seg - 1) & 1u, tmo, args.status)) {
+                    ok = false;
+                    break;
                 }
-                umma_commit(empty + s);
+                tc_fence_after();
+                const int nk = it.k_hi - it.k_lo;
+                const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+                for (int i = 0; i < steps; ++i, ++g) {
+                    const int s = g % kFusedStages;
+                    const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
+                    if (!mbar_wait(full + s, u & 1u, tmo, args.status) || !mbar_wait(deq + s, u & 1u, tmo, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t act = smem_u32(smem + s * kStageBytes);
+                    const uint32_t wt = act + kOffW;
+                    const int ksub = (i < nk) ? (kFusedBK / 16) : (args.r + 15) / 16;
+                    for (int kk = 0; kk < ksub; ++kk) {
+                        const uint64_t bdesc = kTransW ? sw128_desc(wt + kk * 2048, 8192, 1024)
+                                                       : sw128_desc(wt + kk * 32, 16, 1024);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t adesc = sw128_desc(act + h * 16384 + kk * 32, 16, 1024);
+                            umma_f16(tmem + h * 256, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    umma_commit(empty + s);
+                }
+                umma_commit(acc);  // arrives once every UMMA of the segment has completed
+                ++seg;
             }
             if (!ok) {
                 *abort_flag = 1;
                 __threadfence_block();
+                umma_commit(acc);  // releases an epilogue waiting on this segment
             }
-            umma_commit(acc);  // arrives once every issued UMMA has completed
-            mbar_wait(acc, 0, tmo, args.status);
         }
         __syncwarp();
     } else {
-        // ----------------------------------------------------- dequantise --
+        // ---------------------------------------- dequantise, then epilogue --
         const int t = threadIdx.x;  // 0..255
+        const int q = warp & 3, h = warp >> 2;
+        const int row_l = h * 128 + q * 32 + lane;  // tile row of this thread in the epilogue
         bool ok = true;
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % kFusedStages;
-            const uint32_t u = static_cast<uint32_t>(kt / kFusedStages);
-            // every lane waits; the outcome is made warp-uniform before any branch
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(full + s, u & 1u, tmo, args.status));
-            if (!ok) break;
-            uint8_t* st = smem + s * kStageBytes;
-            const uint32_t codes = smem_u32(st + kOffCodes);
-            const uint32_t wt = smem_u32(st + kOffW);
-            const float* cs = reinterpret_cast<const float*>(st + kOffC);
-            if (!kTransW) {
-                // row t of the weight tile, k-block kt; codes rows are 32 B, 32-byte swizzled
-                const uint32_t crow = codes + t * 32;
-                const uint32_t sw = (t >> 2) & 1;
-                const uint32_t wrow = wt + t * 128;
-                dequant_block(tab, cs[t], crow + ((0 ^ sw) << 4), crow + ((1 ^ sw) << 4),
-                              [&](int j) { return wrow + ((static_cast<uint32_t>(j) ^ (t & 7)) << 4); });
-            } else {
-                // weight row nl (reduction index), k-block a of the 4 in the tile
-                const int nl = t & 63, a = t >> 6;
-                const uint32_t crow = codes + nl * 128;
-                const uint32_t sw = nl & 7;
-                const uint32_t dst = wt + a * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
-                dequant_block(tab, cs[a * 64 + nl], crow + (((2 * a) ^ sw) << 4), crow + (((2 * a + 1) ^ sw) << 4),
-                              [&](int j) { return dst + ((static_cast<uint32_t>(j) ^ sw) << 4); });
-            }
-            fence_proxy_async_smem();  // this thread's tile stores -> visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(deq + s);
-        }
-        if (!ok) *abort_flag = 1;
-
-        // ------------------------------------------------------- epilogue --
-        const bool acc_ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, tmo, args.status));
-        tc_fence_after();
-        if (__all_sync(0xFFFFFFFFu, acc_ok && !*abort_flag)) {
-            const int q = warp & 3, h = warp >> 2;
-            const int64_t row = m0 + h * 128 + q * 32 + lane;
-            for (int c0 = 0; c0 < kFusedBN; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c0, r);
-                tmem_ld_wait();
-                const int64_t col = n0 + c0;
-                if (row < args.M && col < args.out_cols) {
-                    uint32_t p[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        p[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                    uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.out_cols + col);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (col + 8 * i < args.out_cols)
-                            dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+        int g = 0, seg = 0;
+        SegIter<kSplit> it(sc, cta);
+        while (it.next()) {
+            const int64_t m0 = (it.tile / tiles_n) * kFusedBM, n0 = (it.tile % tiles_n) * kFusedBN;
+            const int nk = it.k_hi - it.k_lo;
+            const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+            for (int i = 0; ok && i < steps; ++i, ++g) {
+                const int s = g % kFusedStages;
+                const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
+                // every lane waits; the outcome is made warp-uniform before any branch
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(full + s, u & 1u, tmo, args.status));
+                if (!ok) break;
+                if (i < nk) {
+                    uint8_t* st = smem + s * kStageBytes;
+                    const uint32_t codes = smem_u32(st + kOffCodes);
+                    const uint32_t wt = smem_u32(st + kOffW);
+                    const float* cs = reinterpret_cast<const float*>(st + kOffC);
+                    if (!kTransW) {
+                        // row t of the weight tile; codes rows are 32 B, 32-byte swizzled
+                        const uint32_t crow = codes + t * 32;
+                        const uint32_t sw = (t >> 2) & 1;
+                        const uint32_t wrow = wt + t * 128;
+                        dequant_block(tab, cs[t], crow + ((0 ^ sw) << 4), crow + ((1 ^ sw) << 4),
+                                      [&](int j) { return wrow + ((static_cast<uint32_t>(j) ^ (t & 7)) << 4); });
+                    } else {
+                        // weight row nl (reduction index), k-block a of the 4 in the tile
+                        const int nl = t & 63, a = t >> 6;
+                        const uint32_t crow = codes + nl * 128;
+                        const uint32_t sw = nl & 7;
+                        const uint32_t dst = wt + a * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+                        dequant_block(tab, cs[a * 64 + nl], crow + (((2 * a) ^ sw) << 4),
+                                      crow + (((2 * a + 1) ^ sw) << 4),
+                                      [&](int j) { return dst + ((static_cast<uint32_t>(j) ^ sw) << 4); });
+                    }
+                    fence_proxy_async_smem();  // this thread's tile stores -> visible to the tensor core
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(deq + s);
             }
+            if (!ok) *abort_flag = 1;
+
+            // ------------------------------------------ segment epilogue --
+            const bool acc_ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, static_cast<uint32_t>(seg) & 1u, tmo, args.status));
+            tc_fence_after();
+            const bool good = __all_sync(0xFFFFFFFFu, acc_ok && !*abort_flag);
+            const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+            // A partial tile is private scratch laid out for the epilogue
+            // threads: float4 i of 32-column chunk c of thread t lives at
+            // ((c * 8 + i) * 256 + t), so each warp instruction moves 512
+            // contiguous bytes.
+            const int64_t tile_floats = static_cast<int64_t>(kFusedBM) * kFusedBN;
+            if (kSplit && it.k_lo > 0) {
+                // contributor: the fp32 partial tile, then the flag
+                float4* my_part = reinterpret_cast<float4*>(args.part + static_cast<int64_t>(cta) * tile_floats) + t;
+                for (int c = 0; c < kFusedBN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(trow + 32 * c, r);
+                    tmem_ld_wait();
+                    if (good) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            my_part[(c * 8 + i) * 256] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                                     __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tmem_free);
+                __threadfence();
+                epi_bar();
+                if (t == 0 && good) st_release(args.flags + cta, 1);
+            } else {
+                // owner: wait for the contributors of the tile's later steps
+                const int first = cta + 1;
+                const int last = (kSplit && it.k_hi < KT) ? sc.cta_of(it.tile * KT + KT - 1) : cta;
+                if (first <= last) {  // only a split tile waits and fences
+                if (t == 0) {
+                    int okp = good ? 1 : 0;
+                    const uint64_t t0 = global_timer_ns();
+                    for (int cc = first; cc <= last && okp; ++cc) {
+                        while (ld_acquire(args.flags + cc) == 0) {
+                            if (global_timer_ns() - t0 > tmo) {
+                                atomicOr(args.status, kStatusTimeout);
+                                okp = 0;
+                                break;
+                            }
+                        }
+                    }
+                    *parts_ok = okp;
+                }
+                epi_bar();
+                __threadfence();
+                }
+                const bool write = good && (first > last || *parts_ok);
+                const int64_t row = m0 + row_l;
+                // 2 KB scratch of this warp in stage 0's weight region, idle now
+                const uint32_t scratch = smem_u32(smem + kOffW) + warp * 2048;
+                for (int c = 0; c < kFusedBN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(trow + 32 * c, r);
+                    tmem_ld_wait();
+                    if (write && row < args.M) {
+                        float v[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                        for (int cc = first; cc <= last; ++cc) {
+                            const float4* src =
+                                reinterpret_cast<const float4*>(args.part + static_cast<int64_t>(cc) * tile_floats) + t;
+                            float4 pv[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) pv[i] = __ldcg(src + (c * 8 + i) * 256);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                v[4 * i] += pv[i].x;
+                                v[4 * i + 1] += pv[i].y;
+                                v[4 * i + 2] += pv[i].z;
+                                v[4 * i + 3] += pv[i].w;
+                            }
+                        }
+                        // this row's 32 columns as bf16 into the warp's scratch:
+                        // 64-byte rows, 16-byte pieces XOR-swizzled by the row
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t w4[4] = {pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                                    pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                                    pack_bf16x2(v[8 * j + 6], v[8 * j + 7])};
+                            sts128(scratch + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), w4);
+                        }
+                    }
+                    __syncwarp();
+                    if (write) {
+                        // whole 64-byte row segments: 8 rows of the warp per store
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = 8 * i + (lane >> 2), pc = lane & 3;
+                            const int64_t orow = m0 + row_l - lane + rr;
+                            const int64_t ocol = n0 + 32 * c + 8 * pc;
+                            const uint4 d = lds128(scratch + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4));
+                            if (orow < args.M && ocol < args.out_cols)
+                                *reinterpret_cast<uint4*>(args.out + orow * args.out_cols + ocol) = d;
+                        }
+                    }
+                    __syncwarp();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tmem_free);
+            }
+            ++seg;
+            if (!ok) break;
         }
     }
 
@@ -264,9 +452,11 @@ template <bool kTransW>
 cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                          const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
                          cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>((a.out_cols + kFusedBN - 1) / kFusedBN),
-              static_cast<unsigned>((a.M + kFusedBM - 1) / kFusedBM));
-    fused_nf4_gemm<kTransW><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
+    const dim3 grid(static_cast<unsigned>(a.ctas));
+    if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, a.out_cols))
+        fused_nf4_gemm<kTransW, false><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
+    else
+        fused_nf4_gemm<kTransW, true><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
     return cudaGetLastError();
 }
 
@@ -275,10 +465,15 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
 size_t fused_smem_bytes() { return kSmemBytes; }
 
 cudaError_t fused_init_device() {
-    cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(fused_nf4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(fused_nf4_gemm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kSmemBytes))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fused_nf4_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kSmemBytes))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fused_nf4_gemm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kSmemBytes))) != cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(fused_nf4_gemm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kSmemBytes));
 }
 

@@ -40,11 +40,32 @@ struct FusedArgs {
     int64_t out_cols;   // N (forward) or K (dX)
     int64_t red;        // reduction length: K (forward) or N (dX)
     int r;              // LoRA rank (extra reduction columns of the last step)
+    int ctas;           // CTAs (ranges of (tile, step) units): fused_ctas()
     uint16_t* out;      // bf16 [M, out_cols]
+    float* part;        // fp32 [fused_partial_ctas()][256][256] partial tiles of contributing CTAs
+    int* flags;         // [fused_partial_ctas()] partial-ready flags, zero before the launch
     int* status;        // device status word
     uint64_t timeout_ns;
     int stall_producer; // test hook: load nothing
 };
+
+// CTAs of a fused launch. With at least as many output tiles as SMs
+// (max_ctas), one CTA per tile: no tile is split. With fewer, one CTA per SM
+// (at most one per reduction step) and the tiles' steps dealt out in equal
+// ranges, so every SM works; split tiles then go through fp32 partials.
+inline int64_t fused_tiles(int64_t M, int64_t out_cols) {
+    return ((M + kFusedBM - 1) / kFusedBM) * ((out_cols + kFusedBN - 1) / kFusedBN);
+}
+inline int fused_ctas(int64_t M, int64_t out_cols, int64_t red, int max_ctas) {
+    const int64_t tiles = fused_tiles(M, out_cols);
+    if (tiles >= max_ctas) return static_cast<int>(tiles);
+    const int64_t units = tiles * ((red + kFusedBK - 1) / kFusedBK);
+    return static_cast<int>(units < max_ctas ? units : max_ctas);
+}
+// CTAs that may write a partial tile (0 when no tile is split).
+inline int fused_partial_ctas(int64_t M, int64_t out_cols, int64_t red, int max_ctas) {
+    return fused_tiles(M, out_cols) >= max_ctas ? 0 : fused_ctas(M, out_cols, red, max_ctas);
+}
 
 // Forward: out = A_op . deq(W)^T + lora_a . lora_b^T, A_op = X [M, K].
 // Maps: act {K, M} box {64, 256} SW128; codes {K/2, N} box {32, 256} SW32;

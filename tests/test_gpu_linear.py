@@ -270,3 +270,31 @@ def test_register_gemv_deterministic(q):
     a, _ = small_forward(q, cfg, t, 32)
     b, _ = small_forward(q, cfg, t, 32)
     assert torch.equal(a, b)
+
+
+# ---------------------- fused matmuls with split tiles (stream-K ranges) ---
+
+SPLIT = [synth.custom(N=1024, K=2048, M=256, r=16),         # forward: 4 tiles x 32 steps on 128 CTAs
+         synth.custom(N=2048, K=1024, M=512, r=8),          # forward: 16 tiles x 16 steps on 148 CTAs
+         synth.custom(N=4096, K=1024, M=300, r=32),         # dX: 8 tiles of the M x K output, 64 steps each
+         synth.custom(N=264, K=2560, M=520, r=64),          # ragged: 3 x 10 tiles, 5 steps (dX) / 40 (forward)
+         synth.custom(N=256 * 149, K=128, M=256, r=16)]     # 149 tiles: one CTA per tile
+
+
+@pytest.mark.parametrize("cfg", SPLIT, ids=lambda c: c.name)
+def test_fused_split_tiles(q, cfg):
+    """Fewer output tiles than SMs: the CTAs take equal ranges of (tile,
+    step) units, so a tile is split between contributors, which write fp32
+    partials, and its owner, which adds them in CTA order. Every output of
+    the forward and of dX against the fp64 oracle."""
+    g, errs = full_compare(q, cfg)
+    print({k: f"{v:.2e}" for k, v in errs.items()})
+
+
+def test_fused_split_tiles_deterministic(q):
+    cfg = SPLIT[1]
+    t = inputs(cfg)
+    a = gpu_run(q, cfg, t)
+    b = gpu_run(q, cfg, t)
+    for k in ("Y", "dX", "dA", "dB"):
+        assert torch.equal(a[k], b[k]), k
