@@ -19,7 +19,7 @@ using namespace qlora;
 namespace {
 
 // ------------------------------------------------------------ options ----
-std::atomic<int64_t> g_small_m_max{kGemvMaxM};
+std::atomic<int64_t> g_small_m_max{16};
 std::atomic<int64_t> g_fail_launches{0};
 std::atomic<int64_t> g_timeout_us{1000000};
 std::atomic<int64_t> g_stall_producer{0};

@@ -341,11 +341,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             if (kSplit && it.k_lo > 0) {
                 // contributor: the fp32 partial tile, then the flag
                 float4* my_part = reinterpret_cast<float4*>(args.part + static_cast<int64_t>(cta) * tile_floats) + t;
+                const bool live = m0 + row_l < args.M;  // rows past M are never read back
                 for (int c = 0; c < kFusedBN / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32(trow + 32 * c, r);
                     tmem_ld_wait();
-                    if (good) {
+                    if (good && live) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             my_part[(c * 8 + i) * 256] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),

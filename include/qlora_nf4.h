@@ -174,9 +174,11 @@ const char* qlora_status_string(qlora_status s);
 const char* qlora_last_error(void);
 
 /* Test and tuning hooks (not needed for normal use).
- *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses the
- *                           small-batch dequant-GEMV kernel (default and
- *                           maximum 64; 0 forces the tiled GEMM for every M)
+ *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses a
+ *                           small-batch weight-streaming kernel (default 16,
+ *                           maximum 64; 0 forces the tiled GEMM for every M);
+ *                           above it the tiled GEMM, which splits its tiles
+ *                           over K when they are fewer than the SMs
  *   QLORA_OPT_FAIL_LAUNCHES the next `value` kernel launches report
  *                           QLORA_ERR_CUDA without launching (host-side fault
  *                           injection; nothing reaches the GPU)

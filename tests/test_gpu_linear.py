@@ -196,15 +196,17 @@ def test_small_batch_ragged(q, cfg):
 
 
 def test_small_batch_matches_tiled_path(q):
-    """The same forward through the small-batch kernel and through the tiled
-    256 x 256 kernel (forced by QLORA_OPT_SMALL_M_MAX = 0)."""
+    """The same forward through the tcgen05 small-batch kernel (forced by
+    QLORA_OPT_SMALL_M_MAX = 64) and through the tiled 256 x 256 kernel
+    (forced by 0; 16 tiles, so it splits them over K)."""
     cfg = synth.custom(N=4096, K=2048, M=48, r=16)
     t = inputs(cfg)
     w = q.quantize_nf4(t["W"].cuda())
     args = (t["X"].cuda(), w, t["A"].cuda(), t["B"].cuda(), cfg.alpha)
-    Ys, _ = q.linear_fwd(*args)
     old = q.get_option(q.OPT_SMALL_M_MAX)
     try:
+        q.set_option(q.OPT_SMALL_M_MAX, 64)
+        Ys, _ = q.linear_fwd(*args)
         q.set_option(q.OPT_SMALL_M_MAX, 0)
         Yt, _ = q.linear_fwd(*args)
     finally:
@@ -228,13 +230,17 @@ REG = [synth.custom(N=128, K=64 * 37, M=1, r=8),       # one row tile, ten ragge
 
 
 def small_forward(q, cfg, t, reg_max):
+    """Forward through the small-batch kernels: the register-fed one up to
+    reg_max tokens, the tcgen05 one above."""
     w = q.quantize_nf4(t["W"].cuda())
-    old = q.get_option(q.OPT_REG_GEMV_MAX_M)
+    old = q.get_option(q.OPT_REG_GEMV_MAX_M), q.get_option(q.OPT_SMALL_M_MAX)
     try:
         q.set_option(q.OPT_REG_GEMV_MAX_M, reg_max)
+        q.set_option(q.OPT_SMALL_M_MAX, 64)
         Y, sT = q.linear_fwd(t["X"].cuda(), w, t["A"].cuda(), t["B"].cuda(), cfg.alpha)
     finally:
-        q.set_option(q.OPT_REG_GEMV_MAX_M, old)
+        q.set_option(q.OPT_REG_GEMV_MAX_M, old[0])
+        q.set_option(q.OPT_SMALL_M_MAX, old[1])
     torch.cuda.synchronize()
     return Y, sT
 
