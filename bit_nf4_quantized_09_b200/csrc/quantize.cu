@@ -18,8 +18,15 @@ namespace qlora {
 // ---------------------------------------------------------------------------
 // K1: absmax + encode + pack. Eight threads per 64-weight block, eight
 // consecutive weights per thread (two 16-byte loads), four packed bytes out.
-// Nearest level = number of decision thresholds strictly below v = w / c,
-// found by a 4-step binary search over the 15 thresholds in shared memory.
+// The code of v = w / c is the number of decision thresholds strictly below
+// v. It is read from a table over a uniform grid of 129 cells of width 1/64
+// on [-1, 1]: cell j = RN(64 v + 64) covers [(j - 64.5)/64, (j - 63.5)/64],
+// holds the number of thresholds below the cell and the one threshold inside
+// it, if any (neighbouring thresholds are more than 1/64 apart), so the code
+// is base_j + [v > t_j]. RN(64 v + 64) is the low bits of one fma with
+// 1.5 * 2^23 + 64; at a cell edge either cell gives the same code. The table
+// is replicated 16 times so that a half warp reads it without bank
+// conflicts.
 //
 // v is the correctly rounded quotient, computed without a division per
 // weight by Markstein's method (P. Markstein, IBM J. Res. Dev. 34(1), 1990;
@@ -32,20 +39,33 @@ namespace qlora {
 // either way.
 // Loads of the next block run ahead of the current block's arithmetic.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t nf4_code(float q, const float* sM) {
-    int k = (q > sM[7]) ? 8 : 0;
-    k += (q > sM[k + 3]) ? 4 : 0;
-    k += (q > sM[k + 1]) ? 2 : 0;
-    k += (q > sM[k]) ? 1 : 0;
-    return static_cast<uint32_t>(k);
+constexpr int kCells = 129;
+constexpr int kCellCopies = 16;
+
+__device__ __forceinline__ uint32_t nf4_code(float q, const float2* sLut, int copy) {
+    const int j = __float_as_int(__fmaf_rn(q, 64.0f, 12582976.0f)) - 0x4B400000;  // RN(64 q + 64), 0..128
+    const float2 e = sLut[j * kCellCopies + copy];  // {threshold in the cell (2 if none), thresholds below}
+    return static_cast<uint32_t>(__float_as_int(e.y)) + (q > e.x ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restrict__ W, int64_t nblocks,
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
                                                          Nf4Tables tab) {
-    __shared__ float sM[16];
-    if (threadIdx.x < 15) sM[threadIdx.x] = tab.thresh[threadIdx.x];
+    __shared__ float2 sLut[kCells * kCellCopies];
+    for (int i = threadIdx.x; i < kCells * kCellCopies; i += blockDim.x) {
+        const int j = i / kCellCopies;
+        const float lo = (static_cast<float>(j) - 64.5f) * 0.015625f, hi = lo + 0.015625f;  // exact
+        int below = 0;
+        float inside = 2.0f;
+#pragma unroll
+        for (int k = 0; k < 15; ++k) {
+            below += tab.thresh[k] < lo ? 1 : 0;
+            if (tab.thresh[k] >= lo && tab.thresh[k] < hi) inside = tab.thresh[k];
+        }
+        sLut[i] = make_float2(inside, __int_as_float(below));
+    }
     __syncthreads();
+    const int copy = threadIdx.x & (kCellCopies - 1);
 
     const int sub = threadIdx.x & 7;               // position inside the block
     const int lane_blk = (threadIdx.x & 31) >> 3;  // which of the warp's 4 blocks
@@ -84,12 +104,12 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
                 const float q0 = __fmul_rn(v[i], y);
                 const float rem = __fmaf_rn(-c, q0, v[i]);
                 const float q = __fmaf_rn(rem, y, q0);
-                word |= nf4_code(q, sM) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+                word |= nf4_code(q, sLut, copy) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
             }
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                word |= nf4_code(__fdiv_rn(v[i], c), sM) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+                word |= nf4_code(__fdiv_rn(v[i], c), sLut, copy) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
         }
         // element 2j sits in the high nibble of byte j; bytes little-endian in the word
         if (valid) {
