@@ -786,7 +786,10 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     ga.status = status;
     ga.timeout_ns = timeout_ns();
     if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_skinny(ta0, tb0, ta1, tb1, ga, 2, st), 1, "skinny(grads)");
+    // dA and dB need only sU and sT: launched as dX's programmatic
+    // dependent they start once every dX tile has started, on the SMs dX's
+    // last wave leaves idle (a profiled call keeps plain stream order)
+    QLORA_LAUNCH(launch_skinny(ta0, tb0, ta1, tb1, ga, 2, st, ev1 == nullptr), 1, "skinny(grads)");
     return QLORA_OK;
 }
 

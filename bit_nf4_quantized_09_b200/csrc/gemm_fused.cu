@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_lact,
                    const __grid_constant__ CUtensorMap tm_lw, const FusedArgs args, const Nf4Tables tab) {
+    // a launch that depends on this one programmatically (the adapter
+    // gradients beside dX) is admitted once every tile of this launch has
+    // started, i.e. onto the SMs its last wave leaves idle
+    asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
@@ -453,12 +457,24 @@ template <bool kTransW>
 cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                          const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
                          cudaStream_t st) {
-    const dim3 grid(static_cast<unsigned>(a.ctas));
+    // the highest scheduling priority: work overlapping this launch only
+    // takes SMs its tiles leave idle
+    int least = 0, greatest = 0;
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.ctas));
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributePriority;
+    attr[0].val.priority = greatest;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, a.out_cols))
-        fused_nf4_gemm<kTransW, false><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
-    else
-        fused_nf4_gemm<kTransW, true><<<grid, kFusedThreads, kSmemBytes, st>>>(act, codes, cT, lact, lw, a, tab);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, false>, act, codes, cT, lact, lw, a, tab);
+    return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, true>, act, codes, cT, lact, lw, a, tab);
 }
 
 }  // namespace

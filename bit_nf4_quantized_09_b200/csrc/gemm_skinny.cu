@@ -261,6 +261,10 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // launched as a programmatic dependent (beside a fused matmul), this
+    // grid completes only after its primary, so later work on the stream
+    // still sees the primary's results; otherwise a no-op
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
@@ -268,16 +272,25 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 size_t skinny_smem_bytes() { return kSmem; }
 
 cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
-                          const SkinnyArgs& args, int nproblems, cudaStream_t st) {
+                          const SkinnyArgs& args, int nproblems, cudaStream_t st, bool pdl) {
     int64_t max_tiles = 0;
     int max_splits = 0;
     for (int p = 0; p < nproblems; ++p) {
         max_tiles = std::max<int64_t>(max_tiles, (args.p[p].rows + 127) / 128);
         max_splits = std::max(max_splits, args.p[p].splits);
     }
-    dim3 grid(static_cast<unsigned>(max_tiles), static_cast<unsigned>(max_splits), static_cast<unsigned>(nproblems));
-    skinny_gemm<<<grid, kSkinnyThreads, kSmem, st>>>(a0, b0, a1, b1, args);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(max_tiles), static_cast<unsigned>(max_splits),
+                       static_cast<unsigned>(nproblems));
+    cfg.blockDim = dim3(kSkinnyThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, skinny_gemm, a0, b0, a1, b1, args);
 }
 
 cudaError_t skinny_init_device() {

@@ -180,7 +180,10 @@ struct SkinnyArgs {
     uint64_t timeout_ns;
 };
 
+// pdl: launch as the programmatic dependent of the previous launch on st (it
+// may start once every CTA of that launch has started; it completes after it).
 cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
-                          const CUtensorMap& b1, const SkinnyArgs& args, int nproblems, cudaStream_t st);
+                          const CUtensorMap& b1, const SkinnyArgs& args, int nproblems, cudaStream_t st,
+                          bool pdl = false);
 
 }  // namespace qlora

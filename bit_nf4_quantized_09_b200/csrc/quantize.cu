@@ -52,8 +52,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
                                                          Nf4Tables tab) {
     __shared__ float2 sLut[kCells * kCellCopies];
-    for (int i = threadIdx.x; i < kCells * kCellCopies; i += blockDim.x) {
-        const int j = i / kCellCopies;
+    for (int j = threadIdx.x; j < kCells; j += blockDim.x) {
         const float lo = (static_cast<float>(j) - 64.5f) * 0.015625f, hi = lo + 0.015625f;  // exact
         int below = 0;
         float inside = 2.0f;
@@ -62,7 +61,9 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
             below += tab.thresh[k] < lo ? 1 : 0;
             if (tab.thresh[k] >= lo && tab.thresh[k] < hi) inside = tab.thresh[k];
         }
-        sLut[i] = make_float2(inside, __int_as_float(below));
+        const float2 e = make_float2(inside, __int_as_float(below));
+#pragma unroll
+        for (int c = 0; c < kCellCopies; ++c) sLut[j * kCellCopies + c] = e;
     }
     __syncthreads();
     const int copy = threadIdx.x & (kCellCopies - 1);
