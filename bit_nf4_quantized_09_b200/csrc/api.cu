@@ -676,7 +676,10 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused forward");
+    // programmatic dependent of the sT launch: the main loop overlaps it
+    // (a profiled call keeps plain stream order)
+    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
+                 "fused forward");
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
     return QLORA_OK;
 }
@@ -756,7 +759,9 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), st), 1, "fused dX");
+    // plain stream order after the rank-r launches: the adapter gradients,
+    // dX's programmatic dependent, read sU and sT from their first step
+    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
 
     // dA = sU^T X (as dA^T[K, r] = X^T sU) and dB = dY^T sT, split over tokens

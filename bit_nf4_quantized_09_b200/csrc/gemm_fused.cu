@@ -214,6 +214,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                             tma_load_2d(st + kOffC, &tm_c, full + s, kt * kFusedBK, static_cast<int>(n0 / kBlock));
                         }
                     } else {
+                        // the rank-r input (sT or sU) comes from the preceding
+                        // launch, of which this one may be a programmatic dependent
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
                         // the rank-r step lands in a weight-tile region, which the
                         // previous segment's epilogue uses as scratch: wait for it
                         if (seg > 0 && !mbar_wait(tmem_free, static_cast<uint32_t>(seg - 1) & 1u, tmo, args.status)) {
@@ -456,7 +459,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 template <bool kTransW>
 cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                          const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
-                         cudaStream_t st) {
+                         bool pdl, cudaStream_t st) {
     // the highest scheduling priority: work overlapping this launch only
     // takes SMs its tiles leave idle
     int least = 0, greatest = 0;
@@ -467,11 +470,13 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
     cfg.blockDim = dim3(kFusedThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributePriority;
     attr[0].val.priority = greatest;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, a.out_cols))
         return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, false>, act, codes, cT, lact, lw, a, tab);
     return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, true>, act, codes, cT, lact, lw, a, tab);
@@ -496,14 +501,14 @@ cudaError_t fused_init_device() {
 
 cudaError_t launch_fused_fwd(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                              const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
-                             const Nf4Tables& tab, cudaStream_t st) {
-    return launch_fused<false>(act, codes, cT, lora_act, lora_w, a, tab, st);
+                             const Nf4Tables& tab, bool pdl, cudaStream_t st) {
+    return launch_fused<false>(act, codes, cT, lora_act, lora_w, a, tab, pdl, st);
 }
 
 cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
-                            const Nf4Tables& tab, cudaStream_t st) {
-    return launch_fused<true>(act, codes, cT, lora_act, lora_w, a, tab, st);
+                            const Nf4Tables& tab, bool pdl, cudaStream_t st) {
+    return launch_fused<true>(act, codes, cT, lora_act, lora_w, a, tab, pdl, st);
 }
 
 }  // namespace qlora

@@ -71,16 +71,18 @@ inline int fused_partial_ctas(int64_t M, int64_t out_cols, int64_t red, int max_
 // Maps: act {K, M} box {64, 256} SW128; codes {K/2, N} box {32, 256} SW32;
 // cT {ldc, K/64} box {256, 1}; lora_act = sT {r, M} box {64, 256} SW128;
 // lora_w = B {r, N} box {64, 256} SW128.
+// pdl: launch as the programmatic dependent of the previous launch on st (the
+// rank-r input, its output, is waited for only before the rank-r step).
 cudaError_t launch_fused_fwd(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                              const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
-                             const Nf4Tables& tab, cudaStream_t st);
+                             const Nf4Tables& tab, bool pdl, cudaStream_t st);
 // dX: out = dY . deq(W) + sU . A.
 // Maps: act = dY {N, M} box {64, 256} SW128; codes {K/2, N} box {128, 64} SW128;
 // cT {ldc, K/64} box {64, 4}; lora_act = sU {r, M} box {64, 256} SW128;
 // lora_w = A {K, r} box {64, 64} SW128 (four boxes per step).
 cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
-                            const Nf4Tables& tab, cudaStream_t st);
+                            const Nf4Tables& tab, bool pdl, cudaStream_t st);
 
 // ------------------------------------------------ small-batch dequant GEMV --
 constexpr int kGemvThreads = 320;  // 8 dequant warps (4 also epilogue), TMA warp, MMA warp
