@@ -257,6 +257,15 @@ def other_rows(q, dev):
             Wbc = torch.empty(c.N, c.K, dtype=torch.bfloat16, device=dev)
             tq = timed(lambda i: q.quantize_nf4(Wc, out=wcs[i % ncopy]), n=10)
             td = timed(lambda i: q.dequantize_nf4(wcs[i % ncopy], out=Wbc), n=10)
+            # the same weight stored in bf16 (a scratch packed copy: the rotated
+            # copies keep the fp32 weight's codes for the sweep below)
+            Wc16 = Wc.to(torch.bfloat16)
+            scratch = q.NF4Weight.empty(c.N, c.K, dev)
+            tq16 = timed(lambda i: q.quantize_nf4(Wc16, out=scratch), n=10)
+            q16b = c.N * c.K * (2 + 0.5 + 1 / 64)
+            sweep[f"quantize_bf16_{c.N}x{c.K}"] = {"us": tq16 * 1e3, "GBs": q16b / tq16 / 1e6,
+                                                   "frac_hbm": q16b / tq16 / 1e6 / pk_hbm}
+            del Wc16, scratch
             qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
             sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
             sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}

@@ -51,6 +51,7 @@ _SIGNATURES = {
     "qlora_workspace_bytes": (_sz, [_int, _i64, _i64, _i64, _int]),
     "qlora_quantize_nf4": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_quantize_nf4_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "qlora_quantize_nf4_bf16": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_dequantize_nf4": (_int, [_wp, _vp, _vp]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -186,16 +187,18 @@ def _ws(nbytes: int, device, ws: torch.Tensor | None = None) -> torch.Tensor:
 
 
 def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, ws: torch.Tensor | None = None) -> NF4Weight:
-    """NF4 + double quantisation of an fp32 [N, K] CUDA tensor."""
-    assert W.dtype == torch.float32 and W.is_cuda and W.dim() == 2
+    """NF4 + double quantisation of an fp32 or bf16 [N, K] CUDA tensor (a bf16
+    weight gives the bits of its fp32 upcast)."""
+    assert W.dtype in (torch.float32, torch.bfloat16) and W.is_cuda and W.dim() == 2
     N, K = W.shape
     w = out if out is not None else NF4Weight.empty(N, K, W.device)
     nbytes = workspace_bytes(OP_QUANTIZE, 0, N, K, 0)
     if nbytes == 0:
         raise QLoraError(-2, "qlora_quantize_nf4", f"shape {tuple(W.shape)}")
     ws = _ws(nbytes, W.device, ws)
-    _check(lib().qlora_quantize_nf4(_ptr(W), N, K, _ptr(w.codes), _ptr(w.qabsmax), _ptr(w.s2), _ptr(w.mean),
-                                    _ptr(ws), ws.numel(), _stream(W.device)), "qlora_quantize_nf4")
+    entry = "qlora_quantize_nf4_bf16" if W.dtype == torch.bfloat16 else "qlora_quantize_nf4"
+    _check(getattr(lib(), entry)(_ptr(W), N, K, _ptr(w.codes), _ptr(w.qabsmax), _ptr(w.s2), _ptr(w.mean),
+                                 _ptr(ws), ws.numel(), _stream(W.device)), entry)
     return w
 
 

@@ -509,8 +509,24 @@ qlora_status qlora_nf4_tables(float* levels_host, float* thresholds_host) {
     return QLORA_OK;
 }
 
+namespace {
+qlora_status quantize_any(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
+                          float* mean, void* ws, size_t ws_bytes, void* stream);
+}  // namespace
+
 qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
                                 float* mean, void* ws, size_t ws_bytes, void* stream) {
+    return quantize_any(W, false, N, K, codes, qabsmax, s2, mean, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_quantize_nf4_bf16(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax,
+                                     float* s2, float* mean, void* ws, size_t ws_bytes, void* stream) {
+    return quantize_any(W, true, N, K, codes, qabsmax, s2, mean, ws, ws_bytes, stream);
+}
+
+namespace {
+qlora_status quantize_any(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
+                          float* mean, void* ws, size_t ws_bytes, void* stream) {
     if (!W || !codes || !qabsmax || !s2 || !mean || !ws) return QLORA_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0 || K % kBlock != 0) return QLORA_ERR_BAD_SHAPE;
     if (!aligned16(W) || !aligned16(codes) || !aligned16(qabsmax) || !aligned16(s2) || !aligned16(ws) ||
@@ -525,11 +541,12 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K, uint8_t* c
     const int64_t nb = N * K / kBlock;
     float* absmax = static_cast<float*>(ws);
     double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + up256(static_cast<size_t>(nb) * 4));
-    QLORA_LAUNCH(launch_nf4_encode(W, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
+    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
     return QLORA_OK;
 }
+}  // namespace
 
 qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
     if (!W_out) return QLORA_ERR_INVALID_ARG;
@@ -891,7 +908,7 @@ extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, in
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* absmax = static_cast<float*>(scratch);
     double* tree = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocAbsmaxBytes);
-    QLORA_LAUNCH(launch_nf4_encode(W, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
+    QLORA_LAUNCH(launch_nf4_encode(W, false, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
     if (injected_failure()) return QLORA_ERR_CUDA;
     QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
     return QLORA_OK;

@@ -10,7 +10,8 @@
 namespace qlora {
 
 // ----------------------------------------------------------- quantisation --
-cudaError_t launch_nf4_encode(const float* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+// W: fp32 [N, K], or bf16 [N, K] when bf16 is true.
+cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
                               const Nf4Tables& tab, int num_sms, cudaStream_t st);
 size_t dq_tree_scratch_doubles(int64_t nb);
 cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,

@@ -48,7 +48,47 @@ __device__ __forceinline__ uint32_t nf4_code(float q, const float2* sLut, int co
     return static_cast<uint32_t>(__float_as_int(e.y)) + (q > e.x ? 1u : 0u);
 }
 
-__global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restrict__ W, int64_t nblocks,
+// One thread's eight consecutive weights of a block, as loaded: two float4
+// of fp32 input, or one uint4 of bf16 input (every bf16 value is an fp32
+// value, so a bf16 weight codes exactly as its fp32 upcast).
+template <bool kBf16>
+struct Raw8 {
+    float4 a, b;
+};
+template <>
+struct Raw8<true> {
+    uint4 a;
+};
+
+template <bool kBf16>
+__device__ __forceinline__ Raw8<kBf16> load8(const void* W, int64_t blk, int sub) {
+    Raw8<kBf16> r;
+    if constexpr (kBf16) {
+        r.a = __ldcs(reinterpret_cast<const uint4*>(W) + blk * 8 + sub);
+    } else {
+        r.a = __ldcs(reinterpret_cast<const float4*>(W) + blk * 16 + sub * 2);
+        r.b = __ldcs(reinterpret_cast<const float4*>(W) + blk * 16 + sub * 2 + 1);
+    }
+    return r;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float (&v)[8]) {
+    if constexpr (kBf16) {
+        const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);  // element 2i in the low half
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        v[0] = r.a.x, v[1] = r.a.y, v[2] = r.a.z, v[3] = r.a.w;
+        v[4] = r.b.x, v[5] = r.b.y, v[6] = r.b.z, v[7] = r.b.w;
+    }
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) nf4_encode_kernel(const void* __restrict__ W, int64_t nblocks,
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
                                                          Nf4Tables tab) {
     __shared__ float2 sLut[kCells * kCellCopies];
@@ -74,21 +114,16 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
     int64_t bw = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * 4;
 
     // warp-uniform loop: every lane takes part in the shuffles of every pass
-    float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
-    if (bw + lane_blk < nblocks) {
-        x0 = __ldcs(W + (bw + lane_blk) * 16 + sub * 2);
-        x1 = __ldcs(W + (bw + lane_blk) * 16 + sub * 2 + 1);
-    }
+    Raw8<kBf16> x{};
+    if (bw + lane_blk < nblocks) x = load8<kBf16>(W, bw + lane_blk, sub);
     for (; bw < nblocks; bw += stride) {
         const int64_t b = bw + lane_blk;
         const bool valid = b < nblocks;
         const int64_t nb = b + stride;
-        float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
-        if (nb < nblocks) {
-            n0 = __ldcs(W + nb * 16 + sub * 2);
-            n1 = __ldcs(W + nb * 16 + sub * 2 + 1);
-        }
-        const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        Raw8<kBf16> nx{};
+        if (nb < nblocks) nx = load8<kBf16>(W, nb, sub);
+        float v[8];
+        unpack8<kBf16>(x, v);
         float c = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) c = fmaxf(c, fabsf(v[i]));
@@ -117,8 +152,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const float4* __restric
             __stcs(codes + b * 8 + sub, word);
             if (sub == 0) absmax[b] = c;
         }
-        x0 = n0;
-        x1 = n1;
+        x = nx;
     }
 }
 
@@ -337,12 +371,14 @@ static int grid_for(int64_t work_items, int threads, int max_ctas) {
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-cudaError_t launch_nf4_encode(const float* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
                               const Nf4Tables& tab, int num_sms, cudaStream_t st) {
     const int64_t nb = N * K / kBlock;
     const int grid = grid_for(nb * 8, 256, num_sms * 8);
-    nf4_encode_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(W), nb,
-                                            reinterpret_cast<uint32_t*>(codes), absmax, tab);
+    if (bf16)
+        nf4_encode_kernel<true><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab);
+    else
+        nf4_encode_kernel<false><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab);
     return cudaGetLastError();
 }
 

@@ -103,6 +103,17 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t N, int64_t K,
                                 uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
                                 void* ws, size_t ws_bytes, void* stream);
 
+/* qlora_quantize_nf4 for a weight stored in bf16 (bf16 [N, K], device): the
+ * ordinary 16-bit form of pretrained weights [explainer, opening: a 65B
+ * model is 130 GB of BF16 weights], and the form a 16-bit merge of the
+ * adapters produces before it is quantised again [explainer 落とし穴].
+ * Every bf16 value is exactly an fp32 value, so the result is bit for bit
+ * that of qlora_quantize_nf4 on the fp32 upcast of W; the encoder reads half
+ * the bytes. Arguments, workspace and errors as for qlora_quantize_nf4. */
+qlora_status qlora_quantize_nf4_bf16(const uint16_t* W, int64_t N, int64_t K,
+                                     uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
+                                     void* ws, size_t ws_bytes, void* stream);
+
 /* The same quantisation as qlora_quantize_nf4, for callers that cannot
  * allocate device memory at the point of the call: inference-runtime plugin
  * interfaces that hand over only input and output buffers and no workspace,

@@ -180,3 +180,32 @@ def test_encoder_near_thresholds_bit_exact(q):
     W = near_threshold_weight()
     ref = oracle.quantize_nf4(W)
     assert_quant_equal(gpu_quant(q, W), ref)
+
+
+# ------------------------------------------------------ bf16-input quantiser
+
+@pytest.mark.parametrize("shape", [(8, 64), (264, 320), (1000, 512), (4096, 4096)])
+def test_bf16_input_quantize_bit_exact(q, shape):
+    """A bf16 weight quantises to the oracle's result on its exact fp32
+    upcast, and to the fp32 entry point's result on that upcast."""
+    rng = np.random.default_rng(shape[0] + 3 * shape[1])
+    Wb = torch.from_numpy((rng.standard_normal(shape) * 0.03).astype(np.float32)).to(torch.bfloat16)
+    up = Wb.float().numpy()
+    ref = oracle.quantize_nf4(up)
+    got = q.quantize_nf4(Wb.cuda())
+    torch.cuda.synchronize()
+    assert_quant_equal(got, ref)
+    via_fp32 = gpu_quant(q, up)
+    for a, b in ((got.codes, via_fp32.codes), (got.qabsmax, via_fp32.qabsmax), (got.s2, via_fp32.s2),
+                 (got.mean, via_fp32.mean)):
+        assert torch.equal(a, b)
+
+
+def test_bf16_input_adversarial_blocks(q):
+    """The adversarial blocks (zeros, subnormals, outliers, values at the
+    thresholds) rounded to bf16: still the oracle's bits on the upcast."""
+    Wb = torch.from_numpy(adversarial_weight()).to(torch.bfloat16)
+    ref = oracle.quantize_nf4(Wb.float().numpy())
+    got = q.quantize_nf4(Wb.cuda())
+    torch.cuda.synchronize()
+    assert_quant_equal(got, ref)
