@@ -1,6 +1,11 @@
-// Small-batch forward (a few tokens): the weight-streaming, memory-bound
-// regime. "ta-paperlens QLoRA explainer", 落とし穴: 4-bit weights pay off in
-// small-batch, token-at-a-time generation because far fewer bytes are read.
+// Small-batch forward (a few tokens) on the tcgen05 tensor core: the
+// weight-streaming, memory-bound regime. "ta-paperlens QLoRA explainer",
+// 落とし穴: 4-bit weights pay off in small-batch, token-at-a-time generation
+// because far fewer bytes are read. The default routing sends up to 16 tokens
+// to the register-fed kernel (gemv_mma.cu) and more to the tiled GEMM (split
+// over K when its tiles are fewer than the SMs), which measured faster; this
+// kernel serves up to 64 tokens when QLORA_OPT_SMALL_M_MAX and
+// QLORA_OPT_REG_GEMV_MAX_M select it.
 //
 // Swap-AB on the tensor core: D[128 weight rows, Mp tokens] accumulates
 // deq(W)[rows, k] . X[tokens, k]^T, so the dequantised weight tile fills the

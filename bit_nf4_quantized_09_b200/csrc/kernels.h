@@ -87,7 +87,7 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
 
 // ------------------------------------------------ small-batch dequant GEMV --
 constexpr int kGemvThreads = 320;  // 8 dequant warps (4 also epilogue), TMA warp, MMA warp
-constexpr int kGemvMaxM = 64;      // tokens that fit the UMMA N side of one tile
+constexpr int kGemvMaxM = 64;      // tokens that fit the UMMA N side of one tile (largest small-batch M)
 size_t gemv_smem_bytes();
 cudaError_t gemv_init_device();
 

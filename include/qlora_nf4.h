@@ -217,10 +217,13 @@ int64_t qlora_get_option(int option);
 /* Profiling hook: record the CUDA events ev_start / ev_stop (cudaEvent_t,
  * owned by the caller) on the launch stream immediately before and after the
  * next launch of the named kernel; the request is consumed by that launch.
- * The records are external event records, so inside a captured CUDA graph
- * they become event-record nodes that time every replay. */
-#define QLORA_KERNEL_FUSED_FWD 1   /* the dequant-fused forward matmul (the
-                                      small-batch kernel when M <= 64)        */
+ * Inside stream capture the records are external event records, so the
+ * captured graph times every replay. A profiled call launches that kernel in
+ * plain stream order (an event between two launches breaks a programmatic
+ * dependent launch), so it may run a little slower than an unprofiled one. */
+#define QLORA_KERNEL_FUSED_FWD 1   /* the forward's weight kernel: the
+                                      dequant-fused matmul, or the small-batch
+                                      kernel when M <= QLORA_OPT_SMALL_M_MAX  */
 #define QLORA_KERNEL_FUSED_DX  2   /* the transposed-dequant dX matmul       */
 qlora_status qlora_profile_next_launch(int kernel, void* ev_start, void* ev_stop);
 
