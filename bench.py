@@ -183,6 +183,24 @@ class OracleSample:
                           f"rows of W (C oracle), {el:.1f} s on {self.threads} host threads"}
 
 
+# ---------------------------------------------------------------- ranks ----
+
+def max_over_ranks(x: float, pg, dev) -> float:
+    """The largest of every rank's x (a time): the job takes as long as its
+    slowest replica. pg is torch.distributed (any backend) or None."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job rate: every replica does the same step (weak scaling), so
+    the job does world steps' work per (max over ranks) step time."""
+    return flops_per_step_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ reference ----
 
 def run_reference(args, rank, world):
@@ -391,11 +409,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = start.elapsed_time(stop) / args.steps
-    if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(stop) / args.steps, pg, dev)
     fwd_ms = statistics.mean(p[0][0].elapsed_time(p[0][1]) for p in prof)
     dx_ms = statistics.mean(p[1][0].elapsed_time(p[1][1]) for p in prof)
     del graph
@@ -442,11 +456,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if pg is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
 
     # ---- the other rows of the path on their own workloads (graph-timed,
     # outside the timed region): the small-batch sweep forward and the
@@ -454,7 +464,7 @@ def run_ours(args, rank, world, local_rank):
     sweep = other_rows(q, dev) if (not args.no_sweep and rank == 0) else {}
 
     flops = fwd_bwd_flops(M, N, K, r)
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = job_tflops(flops, world, ms)
     pk, pk_kind = peaks()
     # dominant kernel: the fused matmul with the larger time per step
     kern = {"fused_forward": (fwd_ms, 2 * M * N * (K + r)), "fused_dx": (dx_ms, 2 * M * K * (N + r))}
@@ -479,7 +489,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic_source": "ncu capture of one launch: dram__bytes_read.sum + dram__bytes_write.sum"
                      if dom in NCU_TRAFFIC else None,
                      "peak_kind": f"bf16 sustained ({pk_kind})"},
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "other_rows": sweep,
