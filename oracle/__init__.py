@@ -62,6 +62,13 @@ def lib():
         L.oracle_storage_bytes.restype = ctypes.c_int64
         L.oracle_storage_bytes.argtypes = [_i64, _i64, ctypes.c_int]
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_quantize_nf4_nodq.restype = ctypes.c_int
+        L.oracle_quantize_nf4_nodq.argtypes = [_f32p, _i64, _i64, _u8p, _f32p]
+        L.oracle_dequant_f32_nodq.argtypes = [_u8p, _f32p, _i64, _i64, _f32p]
+        L.oracle_dequant_bf16_nodq.argtypes = [_u8p, _f32p, _i64, _i64, _u16p]
+        L.oracle_f64_to_bf16.restype = ctypes.c_uint16
+        L.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_f64_to_bf16_array.argtypes = [_f64p, _i64, _u16p]
         _lib = L
     return _lib
 
@@ -215,6 +222,50 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+# ------------------------------------- storage without double quantisation --
+
+def quantize_nf4_nodq(W):
+    """fp32 W [N, K] -> dict(codes packed uint8[N*K/2], absmax fp32[nb]): the
+    blockwise quantiser with each block's fp32 absmax kept as its constant
+    ([p1] 二重量子化, 4 + 32/64 = 4.5 bits per weight)."""
+    W = _f32(W)
+    N, K = W.shape
+    codes = np.zeros(N * K // 2, np.uint8)
+    absmax = np.zeros(N * K // 64, np.float32)
+    rc = lib().oracle_quantize_nf4_nodq(_p(W, _f32p), N, K, _p(codes, _u8p), _p(absmax, _f32p))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_nf4_nodq: bad shape {W.shape}")
+    return dict(codes=codes, absmax=absmax, N=N, K=K)
+
+
+def dequant_f32_nodq(codes, absmax, N: int, K: int) -> np.ndarray:
+    """fp32 [N, K] restore level[code] * absmax of a weight without double
+    quantisation."""
+    codes = np.ascontiguousarray(np.asarray(codes, np.uint8))
+    absmax = _f32(absmax)
+    out = np.zeros((N, K), np.float32)
+    lib().oracle_dequant_f32_nodq(_p(codes, _u8p), _p(absmax, _f32p), N, K, _p(out, _f32p))
+    return out
+
+
+def dequant_bf16_bits_nodq(codes, absmax, N: int, K: int) -> np.ndarray:
+    """bf16 bit patterns (uint16 [N, K]) of dequant_f32_nodq's values."""
+    codes = np.ascontiguousarray(np.asarray(codes, np.uint8))
+    absmax = _f32(absmax)
+    out = np.zeros((N, K), np.uint16)
+    lib().oracle_dequant_bf16_nodq(_p(codes, _u8p), _p(absmax, _f32p), N, K, _p(out, _u16p))
+    return out
+
+
+def f64_to_bf16_bits(x) -> np.ndarray:
+    """bf16 bit patterns of fp64 values, each rounded once (nearest, ties to
+    even; overflow to infinity)."""
+    x = np.ascontiguousarray(np.asarray(x, np.float64))
+    out = np.zeros(x.shape, np.uint16)
+    lib().oracle_f64_to_bf16_array(_p(x, _f64p), x.size, _p(out, _u16p))
+    return out
+
+
 def storage_bytes(N: int, K: int, double_quant: bool = True) -> int:
     return int(lib().oracle_storage_bytes(N, K, 1 if double_quant else 0))
 
@@ -254,6 +305,24 @@ def backward(dY, X, What, A, B, alpha: float, r: int):
     dA = s * (U.T @ X)
     dB = s * (dY.T @ (X @ A.T))
     return dX, dA, dB
+
+
+# ------------------------------------------------------------ adapter merge --
+
+def merge_lora(What, A, B, alpha: float, r: int) -> np.ndarray:
+    """W_merged = What + (alpha/r) B A in fp64: the adapter folded into the
+    weight once, for inference ([p2] 26.2.2, LoRAの学習設定, inference: merge
+    once, then use W_merged like the original weight). B is [N, r], A is
+    [r, K], What the dequantised [N, K] weight. Merging into the 16-bit weight
+    rather than the 4-bit one is [p1] 落とし穴 (an update added to the NF4
+    weight and re-quantised is mostly lost)."""
+    s = alpha / r
+    return What + s * (B @ A)
+
+
+def merge_lora_bf16_bits(What, A, B, alpha: float, r: int) -> np.ndarray:
+    """merge_lora rounded once to bf16 (uint16 bit patterns)."""
+    return f64_to_bf16_bits(merge_lora(What, A, B, alpha, r))
 
 
 def rel_err(got, ref) -> float:

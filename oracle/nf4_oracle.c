@@ -347,6 +347,89 @@ int oracle_quantize_nf4(const float* W, int64_t N, int64_t K, uint8_t* packed,
     return 0;
 }
 
+/* ------------------------------------------------------------------------- */
+/* Storage without double quantisation                                       */
+/* ------------------------------------------------------------------------- */
+
+/* [p1] 二重量子化, first paragraph: before the constants are themselves
+ * quantised, each block of 64 keeps its absmax c as one fp32 (4 + 32/64 = 4.5
+ * bits per weight). The codes are those of the whole quantiser above; the
+ * constants are the block absmax values, unchanged. */
+int oracle_quantize_nf4_nodq(const float* W, int64_t N, int64_t K, uint8_t* packed, float* absmax)
+{
+    if (N <= 0 || K <= 0 || K % ORACLE_BLOCK != 0) return -1;
+    int64_t n = N * K, nb = n / ORACLE_BLOCK;
+    float L[16];
+    oracle_nf4_levels(NULL, L);
+    uint8_t* codes = (uint8_t*)malloc((size_t)n);
+    oracle_encode_blocks(W, nb, ORACLE_BLOCK, L, 16, 7, absmax, codes);
+    oracle_pack_nibbles(codes, n, packed);
+    free(codes);
+    return 0;
+}
+
+/* [p1] 量子化を1段落で: x_hat = c * level[code] with c the block's own fp32
+ * absmax, one fp32 rounding (the restore of the glossary's snippet). */
+void oracle_dequant_f32_nodq(const uint8_t* packed, const float* absmax, int64_t N, int64_t K, float* out)
+{
+    float L[16];
+    oracle_nf4_levels(NULL, L);
+    int64_t nb = N * K / ORACLE_BLOCK;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int i = 0; i < ORACLE_BLOCK; ++i) {
+            int64_t e = b * ORACLE_BLOCK + i;
+            uint8_t byte = packed[e / 2];
+            uint8_t code = (e % 2 == 0) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
+            out[e] = L[code] * absmax[b];
+        }
+    }
+}
+
+/* The same restore, then one bf16 rounding (computed in BF16, [p1]
+ * 勾配は実際どこへ行くのか). */
+void oracle_dequant_bf16_nodq(const uint8_t* packed, const float* absmax, int64_t N, int64_t K, uint16_t* out)
+{
+    int64_t n = N * K;
+    float* f = (float*)malloc((size_t)n * sizeof(float));
+    oracle_dequant_f32_nodq(packed, absmax, N, K, f);
+    for (int64_t e = 0; e < n; ++e) out[e] = oracle_f32_to_bf16(f[e]);
+    free(f);
+}
+
+/* ------------------------------------------------------------------------- */
+/* fp64 -> bf16, one rounding (for the adapter merge)                        */
+/* ------------------------------------------------------------------------- */
+
+/* Round x to the nearest bf16 value, ties to the even significand, in one
+ * step from the fp64 value. bf16 keeps 8 significant bits; for |x| in
+ * [2^(e-1), 2^e) neighbouring values are 2^(e-8) apart, and below the
+ * smallest normal 2^-126 they are 2^-133 apart (subnormals). A result of
+ * 2^128 or more overflows to infinity. nearbyint rounds to nearest even in the
+ * default rounding mode; dividing by a power of two is exact. */
+uint16_t oracle_f64_to_bf16(double x)
+{
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double a = fabs(x);
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e);
+    int qe = e - 8 < -133 ? -133 : e - 8;
+    double r = ldexp(nearbyint(ldexp(a, -qe)), qe);
+    if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+    float f = (float)r;  /* exact: r is a bf16 value */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+void oracle_f64_to_bf16_array(const double* x, int64_t n, uint16_t* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f64_to_bf16(x[i]);
+}
+
 /* Storage of one quantised N x K weight, in bytes: packed codes (4 bits per
  * weight), one 8-bit constant per block of 64, one fp32 per group of 256
  * blocks, one fp32 mean ([p1] 二重量子化). Without double quantisation the
