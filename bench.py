@@ -287,6 +287,27 @@ def other_rows(q, dev):
             qb, db = c.N * c.K * (4 + 0.5 + 1 / 64), c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2)
             sweep[f"quantize_{c.N}x{c.K}"] = {"us": tq * 1e3, "GBs": qb / tq / 1e6, "frac_hbm": qb / tq / 1e6 / pk_hbm}
             sweep[f"dequantize_{c.N}x{c.K}"] = {"us": td * 1e3, "GBs": db / td / 1e6, "frac_hbm": db / td / 1e6 / pk_hbm}
+            # the same weight stored without double quantisation (the rotated
+            # copies' codes, rewritten with identical values, and fp32 constants)
+            nodq = [q.NF4Weight(wcs[i].codes, None, None, None, c.N, c.K,
+                                absmax=torch.empty(c.N * c.K // 64, dtype=torch.float32, device=dev))
+                    for i in range(ncopy)]
+            tqn = timed(lambda i: q.quantize_nf4_nodq(Wc, out=nodq[i % ncopy]), n=10)
+            tdn = timed(lambda i: q.dequantize_nf4(nodq[i % ncopy], out=Wbc), n=10)
+            qnb, dnb = c.N * c.K * (4 + 0.5 + 4 / 64), c.N * c.K * (0.5 + 4 / 64 + 2)
+            sweep[f"quantize_nodq_{c.N}x{c.K}"] = {"us": tqn * 1e3, "GBs": qnb / tqn / 1e6,
+                                                   "frac_hbm": qnb / tqn / 1e6 / pk_hbm}
+            sweep[f"dequantize_nodq_{c.N}x{c.K}"] = {"us": tdn * 1e3, "GBs": dnb / tdn / 1e6,
+                                                     "frac_hbm": dnb / tdn / 1e6 / pk_hbm}
+            del nodq
+            # adapter merge into the bf16 weight
+            for rm in (16, 64):
+                cm = synth.custom(N=c.N, K=c.K, M=1, r=rm)
+                Am, Bm = synth.lora_a(cm).to(dev), synth.lora_b(cm).to(dev)
+                tm = timed(lambda i: q.merge_lora(wcs[i % ncopy], Am, Bm, cm.alpha, out=Wbc), n=10)
+                mb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384 + 2) + 2 * rm * (c.N + c.K)
+                sweep[f"merge_r{rm}_{c.N}x{c.K}"] = {"us": tm * 1e3, "GBs": mb / tm / 1e6,
+                                                     "frac_hbm": mb / tm / 1e6 / pk_hbm}
             del Wbc, Wc
             by_shape[key] = wcs
         wcs = by_shape[key]

@@ -37,7 +37,8 @@ class QLoraError(RuntimeError):
 
 class Nf4WeightC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("qabsmax", ctypes.c_void_p), ("s2", ctypes.c_void_p),
-                ("mean", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+                ("mean", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("absmax", ctypes.c_void_p)]
 
 
 _lib = None
@@ -52,7 +53,10 @@ _SIGNATURES = {
     "qlora_quantize_nf4": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_quantize_nf4_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "qlora_quantize_nf4_bf16": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_quantize_nf4_nodq": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "qlora_quantize_nf4_bf16_nodq": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "qlora_dequantize_nf4": (_int, [_wp, _vp, _vp]),
+    "qlora_merge_lora": (_int, [_wp, _vp, _vp, _int, _f32, _vp, _vp]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_nf4_tables": (_int, [ctypes.POINTER(_f32), ctypes.POINTER(_f32)]),
@@ -151,21 +155,28 @@ def get_option(option: int) -> int:
 
 @dataclasses.dataclass
 class NF4Weight:
-    """A quantised N x K weight: four device tensors owned by torch."""
-    codes: torch.Tensor     # uint8 [N*K/2]
-    qabsmax: torch.Tensor   # uint8 [N*K/64]
-    s2: torch.Tensor        # float32 [ceil(N*K/64/256)]
-    mean: torch.Tensor      # float32 [1]
+    """A quantised N x K weight: device tensors owned by torch. With double
+    quantisation codes, qabsmax, s2 and mean are set and absmax is None;
+    without it codes and absmax are set and the other three are None."""
+    codes: torch.Tensor             # uint8 [N*K/2]
+    qabsmax: torch.Tensor | None    # uint8 [N*K/64]
+    s2: torch.Tensor | None         # float32 [ceil(N*K/64/256)]
+    mean: torch.Tensor | None       # float32 [1]
     N: int
     K: int
+    absmax: torch.Tensor | None = None  # float32 [N*K/64], storage without double quantisation
+
+    @property
+    def double_quant(self) -> bool:
+        return self.absmax is None
 
     def c_view(self) -> Nf4WeightC:
-        key = (self.codes.data_ptr(), self.qabsmax.data_ptr(), self.s2.data_ptr(), self.mean.data_ptr(),
-               self.N, self.K)
+        key = tuple(t.data_ptr() if t is not None else 0
+                    for t in (self.codes, self.qabsmax, self.s2, self.mean, self.absmax)) + (self.N, self.K)
         cached = self.__dict__.get("_c_view")
         if cached is None or cached[0] != key:
             cached = (key, Nf4WeightC(_ptr(self.codes), _ptr(self.qabsmax), _ptr(self.s2), _ptr(self.mean),
-                                      self.N, self.K))
+                                      self.N, self.K, _ptr(self.absmax)))
             self.__dict__["_c_view"] = cached
         return cached[1]
 
@@ -200,6 +211,34 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, ws: torch.Tensor
     _check(getattr(lib(), entry)(_ptr(W), N, K, _ptr(w.codes), _ptr(w.qabsmax), _ptr(w.s2), _ptr(w.mean),
                                  _ptr(ws), ws.numel(), _stream(W.device)), entry)
     return w
+
+
+def quantize_nf4_nodq(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
+    """NF4 without double quantisation (one fp32 absmax per block of 64) of
+    an fp32 or bf16 [N, K] CUDA tensor."""
+    assert W.dtype in (torch.float32, torch.bfloat16) and W.is_cuda and W.dim() == 2
+    N, K = W.shape
+    if K <= 0 or K % 64 != 0 or N <= 0:
+        raise QLoraError(-2, "qlora_quantize_nf4_nodq", f"shape {tuple(W.shape)}")
+    if out is None:
+        out = NF4Weight(torch.empty(N * K // 2, dtype=torch.uint8, device=W.device), None, None, None, N, K,
+                        absmax=torch.empty(N * K // 64, dtype=torch.float32, device=W.device))
+    assert out.absmax is not None and (out.N, out.K) == (N, K)
+    entry = "qlora_quantize_nf4_bf16_nodq" if W.dtype == torch.bfloat16 else "qlora_quantize_nf4_nodq"
+    _check(getattr(lib(), entry)(_ptr(W), N, K, _ptr(out.codes), _ptr(out.absmax), _stream(W.device)), entry)
+    return out
+
+
+def merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [N, K] = deq(W) + (alpha/r) B A: the adapter folded into a 16-bit
+    copy of the weight."""
+    r = A.shape[0]
+    out = out if out is not None else torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
+    v = w.c_view()
+    _check(lib().qlora_merge_lora(ctypes.byref(v), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                                  _stream(out.device)), "qlora_merge_lora")
+    return out
 
 
 def quantize_nf4_noalloc(W: torch.Tensor, out: NF4Weight) -> NF4Weight:

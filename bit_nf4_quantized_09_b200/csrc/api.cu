@@ -353,12 +353,22 @@ cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
                                                : cudaEventRecord(ev, st);
 }
 
+// A weight stored with double quantisation needs qabsmax, s2 and mean; one
+// stored without it (absmax set) needs only its fp32 constants.
 qlora_status check_weight(const qlora_nf4_weight* w) {
-    if (!w || !w->codes || !w->qabsmax || !w->s2 || !w->mean) return QLORA_ERR_INVALID_ARG;
+    if (!w || !w->codes) return QLORA_ERR_INVALID_ARG;
+    if (!w->absmax && (!w->qabsmax || !w->s2 || !w->mean)) return QLORA_ERR_INVALID_ARG;
     if (w->N <= 0 || w->K <= 0 || w->K % kBlock != 0 || w->N % 8 != 0) return QLORA_ERR_BAD_SHAPE;
-    if (!aligned16(w->codes) || !aligned16(w->qabsmax) || !aligned16(w->s2) || (reinterpret_cast<uintptr_t>(w->mean) & 3u))
+    if (!aligned16(w->codes)) return QLORA_ERR_MISALIGNED;
+    if (w->absmax) return aligned16(w->absmax) ? QLORA_OK : QLORA_ERR_MISALIGNED;
+    if (!aligned16(w->qabsmax) || !aligned16(w->s2) || (reinterpret_cast<uintptr_t>(w->mean) & 3u))
         return QLORA_ERR_MISALIGNED;
     return QLORA_OK;
+}
+
+BlockConstants constants_of(const qlora_nf4_weight* w) {
+    if (w->absmax) return BlockConstants{nullptr, nullptr, nullptr, w->absmax};
+    return BlockConstants{w->qabsmax, w->s2, w->mean, nullptr};
 }
 
 uint64_t timeout_ns() { return static_cast<uint64_t>(std::max<int64_t>(1, g_timeout_us.load())) * 1000ull; }
@@ -548,6 +558,55 @@ qlora_status quantize_any(const void* W, bool bf16, int64_t N, int64_t K, uint8_
 }
 }  // namespace
 
+namespace {
+qlora_status quantize_nodq(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+                           void* stream) {
+    if (!W || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return QLORA_ERR_BAD_SHAPE;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax)) return QLORA_ERR_MISALIGNED;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    qlora_status s = device_ready(&sms);
+    if (s != QLORA_OK) return s;
+    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, tables(), sms, static_cast<cudaStream_t>(stream)), 1,
+                 "nf4_encode");
+    return QLORA_OK;
+}
+}  // namespace
+
+qlora_status qlora_quantize_nf4_nodq(const float* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+                                     void* stream) {
+    return quantize_nodq(W, false, N, K, codes, absmax, stream);
+}
+
+qlora_status qlora_quantize_nf4_bf16_nodq(const uint16_t* W, int64_t N, int64_t K, uint8_t* codes, float* absmax,
+                                          void* stream) {
+    return quantize_nodq(W, true, N, K, codes, absmax, stream);
+}
+
+qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                              uint16_t* W_out, void* stream) {
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    if (!rank_ok(r)) return QLORA_ERR_UNSUPPORTED_RANK;
+    if (!A || !B || !W_out || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
+    MergeArgs a{};
+    a.codes = w->codes;
+    a.c = constants_of(w);
+    a.A = A;
+    a.B = B;
+    a.scale = alpha / static_cast<float>(r);
+    a.N = w->N;
+    a.K = w->K;
+    a.W_out = W_out;
+    QLORA_LAUNCH(launch_merge_lora(a, r, tables(), sms, static_cast<cudaStream_t>(stream)), 1, "merge_lora");
+    return QLORA_OK;
+}
+
 qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
     if (!W_out) return QLORA_ERR_INVALID_ARG;
     qlora_status s = check_weight(w);
@@ -559,7 +618,7 @@ qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, vo
     CUtensorMap t_out;
     QLORA_MAP(&t_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_out, kBlock, w->N * w->K / kBlock, kBlock * 2, 64, 128,
               CU_TENSOR_MAP_SWIZZLE_128B, "W_out");
-    QLORA_LAUNCH(launch_nf4_dequant(t_out, w->codes, w->qabsmax, w->s2, w->mean, w->N, w->K, tables(), sms,
+    QLORA_LAUNCH(launch_nf4_dequant(t_out, w->codes, constants_of(w), w->N, w->K, tables(), sms,
                                     static_cast<cudaStream_t>(stream)),
                  1, "nf4_dequant");
     return QLORA_OK;
@@ -609,6 +668,7 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         ga.qabsmax = w->qabsmax;
         ga.s2 = w->s2;
         ga.mean = w->mean;
+        ga.absmax = w->absmax;
         ga.M = M;
         ga.N = N;
         ga.K = K;
@@ -631,7 +691,7 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
         if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
         return QLORA_OK;
     }
-    QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
+    QLORA_LAUNCH(launch_decode_constants_t(constants_of(w), N, K, L.ldc, cT, st), 1, "decode constants");
     if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
                        status, st)) != QLORA_OK)
         return s;
@@ -739,7 +799,7 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
 
     QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
     if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_decode_constants_t(w->qabsmax, w->s2, w->mean, N, K, L.ldc, cT, st), 1, "decode constants");
+    QLORA_LAUNCH(launch_decode_constants_t(constants_of(w), N, K, L.ldc, cT, st), 1, "decode constants");
     // sU = s dY B, with B [N, r] read in place (MN-major)
     if ((s = lora_down(dY, M, N, B, true, r, scale, L.sU_split, partU, reinterpret_cast<int*>(base + L.ctrU), sU,
                        status, st)) != QLORA_OK)

@@ -112,6 +112,19 @@ __device__ __forceinline__ void lut_decode8(const Nf4BlockLut& t, uint32_t packe
     }
 }
 
+// D += A . B on the legacy tensor path, mma.m16n8k16 with bf16 operands and
+// fp32 accumulation. Lane (g, q) = (lane / 4, lane % 4) holds
+//   a[0] = A(g, 2q..2q+1), a[1] = A(g+8, 2q..2q+1), a[2] = A(g, 2q+8..2q+9),
+//   a[3] = A(g+8, 2q+8..2q+9); b0 = B(2q..2q+1, g), b1 = B(2q+8..2q+9, g);
+//   d[0..1] = D(g, 2q..2q+1), d[2..3] = D(g+8, 2q..2q+1)
+// (the lower index in the low half of each 32-bit register).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // prmt.b32 in its default mode: a selector nibble with bit 3 set yields the
 // sign bit of the byte it picks, replicated over the whole output byte.
 __device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {

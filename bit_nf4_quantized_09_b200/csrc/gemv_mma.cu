@@ -69,13 +69,6 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // sum_{j < R} sT[j] * B[j] over bf16 operands, fp32 products and sums in
@@ -145,7 +138,7 @@ struct Sched {
     __device__ int parts(int tile) const { return cta_of(min((tile + 1) * KB, U) - 1) - cta_of(tile * KB) + 1; }
 };
 
-template <int MT>
+template <int MT, bool kNoDq>
 __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
     gemv_mma_kernel(const GemvMmaArgs a, const Nf4Tables tab) {
     constexpr int kStages = Cfg<MT>::kStages;
@@ -206,10 +199,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
             cp_async16(d + 16, a.codes + ia * 32 + 16);
             cp_async16(d + 32, a.codes + ib * 32);
             cp_async16(d + 48, a.codes + ib * 32 + 16);
-            cp_async4(d + 64, a.qabsmax + (ia & ~int64_t(3)));
-            cp_async4(d + 68, a.qabsmax + (ib & ~int64_t(3)));
-            cp_async4(d + 72, a.s2 + (ia >> 8));
-            cp_async4(d + 76, a.s2 + (ib >> 8));
+            if (kNoDq) {  // the two fp32 constants
+                cp_async4(d + 64, a.absmax + ia);
+                cp_async4(d + 68, a.absmax + ib);
+            } else {
+                cp_async4(d + 64, a.qabsmax + (ia & ~int64_t(3)));
+                cp_async4(d + 68, a.qabsmax + (ib & ~int64_t(3)));
+                cp_async4(d + 72, a.s2 + (ia >> 8));
+                cp_async4(d + 76, a.s2 + (ib >> 8));
+            }
         }
         cp_async_commit();  // possibly empty: keeps one group per step
     };
@@ -232,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
 #pragma unroll
     for (int i = 0; i < kStages - 1; ++i) issue(i);
 
-    const float mean = __ldg(a.mean);
+    const float mean = kNoDq ? 0.0f : __ldg(a.mean);
     float acc[MT][4];
 #pragma unroll
     for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
@@ -249,10 +247,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
         cp_async_wait<kStages - 1>();  // this lane's copies of step gi have landed
         const uint32_t d = ring + (gi % kStages) * (kSlot * kThreads);
         const uint4 a0 = lds128(d), a1 = lds128(d + 16), b0 = lds128(d + 32), b1 = lds128(d + 48);
-        const uint4 cq = lds128(d + 64);  // q words A, B; s2 A, B
+        const uint4 cq = lds128(d + 64);  // q words A, B; s2 A, B (kNoDq: constants A, B)
         const uint32_t sh = gi >= it0 ? seg1.sh : seg0.sh;
-        const float cpa = __fmaf_rn(e4m3_to_f32(cq.x >> (sh & 31u)), __uint_as_float(cq.z), mean);
-        const float cpb = __fmaf_rn(e4m3_to_f32(cq.y >> (sh >> 8)), __uint_as_float(cq.w), mean);
+        const float cpa = kNoDq ? __uint_as_float(cq.x)
+                                : __fmaf_rn(e4m3_to_f32(cq.x >> (sh & 31u)), __uint_as_float(cq.z), mean);
+        const float cpb = kNoDq ? __uint_as_float(cq.y)
+                                : __fmaf_rn(e4m3_to_f32(cq.y >> (sh >> 8)), __uint_as_float(cq.w), mean);
         const Nf4BlockLut la = make_block_lut(tab.level, cpa);
         const Nf4BlockLut lb = make_block_lut(tab.level, cpb);
         const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
     }
 }
 
-template <int MT>
+template <int MT, bool kNoDq>
 cudaError_t launch_mt(const GemvMmaArgs& a, const Nf4Tables& tab, size_t smem, bool pdl, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(a.ctas));
@@ -349,7 +349,7 @@ cudaError_t launch_mt(const GemvMmaArgs& a, const Nf4Tables& tab, size_t smem, b
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_mma_kernel<MT>, a, tab);
+    return cudaLaunchKernelEx(&cfg, gemv_mma_kernel<MT, kNoDq>, a, tab);
 }
 
 constexpr int kMaxMt = 4;
@@ -385,24 +385,39 @@ GemvMmaPlan gemv_mma_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
     return plan;
 }
 
-cudaError_t gemv_mma_init_device() {
+namespace {
+template <bool kNoDq>
+cudaError_t gemv_mma_opt_in(int smax) {
     cudaError_t e;
+    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<1, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<2, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) !=
+        cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(gemv_mma_kernel<4, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
+}
+}  // namespace
+
+cudaError_t gemv_mma_init_device() {
     const int smax = 220 * 1024;  // above any plan (the plan keeps two or three CTAs per SM)
-    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) != cudaSuccess)
-        return e;
-    return cudaFuncSetAttribute(gemv_mma_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
+    const cudaError_t e = gemv_mma_opt_in<false>(smax);
+    return e != cudaSuccess ? e : gemv_mma_opt_in<true>(smax);
 }
 
 cudaError_t launch_gemv_mma(const GemvMmaArgs& a, const Nf4Tables& tab, bool pdl, cudaStream_t st) {
     if (a.M < 1 || a.M > kGemvMmaMaxM || a.ctas < 1) return cudaErrorInvalidValue;
     const size_t smem = gemv_mma_smem_bytes(a.M, a.max_chunks);
     const int mt = token_tiles(a.M);
-    if (mt == 1) return launch_mt<1>(a, tab, smem, pdl, st);
-    if (mt == 2) return launch_mt<2>(a, tab, smem, pdl, st);
     static_assert(kMaxMt * 8 == kGemvMmaMaxM, "token tiles");
-    return launch_mt<4>(a, tab, smem, pdl, st);
+    if (a.absmax) {
+        if (mt == 1) return launch_mt<1, true>(a, tab, smem, pdl, st);
+        if (mt == 2) return launch_mt<2, true>(a, tab, smem, pdl, st);
+        return launch_mt<4, true>(a, tab, smem, pdl, st);
+    }
+    if (mt == 1) return launch_mt<1, false>(a, tab, smem, pdl, st);
+    if (mt == 2) return launch_mt<2, false>(a, tab, smem, pdl, st);
+    return launch_mt<4, false>(a, tab, smem, pdl, st);
 }
 
 }  // namespace qlora

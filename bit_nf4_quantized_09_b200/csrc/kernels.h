@@ -9,6 +9,16 @@
 
 namespace qlora {
 
+// The first-level block constants of a quantised weight: with double
+// quantisation c'_b = fmaf(E4M3(qabsmax[b]), s2[b / 256], *mean); without
+// (absmax != nullptr) c_b = absmax[b] and the other three are not read.
+struct BlockConstants {
+    const uint8_t* qabsmax;
+    const float* s2;
+    const float* mean;
+    const float* absmax;
+};
+
 // ----------------------------------------------------------- quantisation --
 // W: fp32 [N, K], or bf16 [N, K] when bf16 is true.
 cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
@@ -18,11 +28,10 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_sc
                                 float* mean, cudaStream_t st);
 // out_map: the bf16 output viewed as [N*K/64 rows, 64], box {64, 128}, SW128.
 constexpr size_t kDequantSmem = 2 * 128 * 128 + 1024;
-cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const uint8_t* q, const float* s2,
-                               const float* mean, int64_t N, int64_t K, const Nf4Tables& tab, int num_sms,
-                               cudaStream_t st);
-cudaError_t launch_decode_constants_t(const uint8_t* q, const float* s2, const float* mean, int64_t N, int64_t K,
-                                      int64_t ldc, float* cT, cudaStream_t st);
+cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const BlockConstants& c, int64_t N,
+                               int64_t K, const Nf4Tables& tab, int num_sms, cudaStream_t st);
+cudaError_t launch_decode_constants_t(const BlockConstants& c, int64_t N, int64_t K, int64_t ldc, float* cT,
+                                      cudaStream_t st);
 cudaError_t launch_e4m3_encode(const float* x, uint8_t* q, int64_t n, cudaStream_t st);
 
 // ------------------------------------------------------ fused NF4 GEMMs --
@@ -120,6 +129,7 @@ struct GemvMmaArgs {
     const uint8_t* qabsmax;  // E4M3 [N*K/64]
     const float* s2;         // [groups]
     const float* mean;       // [1]
+    const float* absmax;     // fp32 [N*K/64] when stored without double quantisation (then the three above are unused)
     int64_t M, N, K;
     int r;                   // LoRA rank
     int ctas;                // grid size (from the plan)
@@ -188,5 +198,19 @@ struct SkinnyArgs {
 cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                           const CUtensorMap& b1, const SkinnyArgs& args, int nproblems, cudaStream_t st,
                           bool pdl = false);
+
+// ---------------------------------------------------------- adapter merge --
+struct MergeArgs {
+    const uint8_t* codes;  // packed NF4 [N, K/2]
+    BlockConstants c;
+    const uint16_t* A;     // bf16 [r, K]
+    const uint16_t* B;     // bf16 [N, r]
+    float scale;           // alpha / r
+    int64_t N, K;
+    uint16_t* W_out;       // bf16 [N, K]
+};
+
+// W_out = bf16(deq(W) + scale . B . A); r in {8, 16, 32, 64}.
+cudaError_t launch_merge_lora(const MergeArgs& a, int r, const Nf4Tables& tab, int num_sms, cudaStream_t st);
 
 }  // namespace qlora

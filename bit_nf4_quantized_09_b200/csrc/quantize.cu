@@ -254,7 +254,9 @@ __device__ __forceinline__ float decode_constant(const uint8_t* q, const float* 
 
 // ---------------------------------------------------------------------------
 // K3: standalone dequantisation to bf16. A CTA of 128 threads walks chunks of
-// 128 consecutive 64-weight blocks, one block per thread. The next chunk's
+// 128 consecutive 64-weight blocks, one block per thread. kNoDq: the weight
+// keeps one fp32 absmax per block (no double quantisation) and q, s2, mean
+// are not read. The next chunk's
 // codes are loaded while the current one is decoded; the 16 KB of bf16 output
 // go to a 128-byte-swizzled shared tile (conflict-free 16-byte stores) that a
 // TMA tensor store writes to global memory as 128 rows of 128 bytes, with two
@@ -262,19 +264,22 @@ __device__ __forceinline__ float decode_constant(const uint8_t* q, const float* 
 // ---------------------------------------------------------------------------
 constexpr int kDeqChunk = 128;
 
+template <bool kNoDq>
 __global__ void __launch_bounds__(kDeqChunk) nf4_dequant_kernel(const __grid_constant__ CUtensorMap tm_out,
                                                                  const uint4* __restrict__ codes,
                                                                  const uint8_t* __restrict__ q,
                                                                  const float* __restrict__ s2,
-                                                                 const float* __restrict__ mean, int64_t nblocks,
+                                                                 const float* __restrict__ mean,
+                                                                 const float* __restrict__ absmax, int64_t nblocks,
                                                                  Nf4Tables tab) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int t = threadIdx.x;
-    const float mu = *mean;
+    const float mu = kNoDq ? 0.0f : *mean;
     const int64_t nchunks = (nblocks + kDeqChunk - 1) / kDeqChunk;
 
-    // this thread's block of the first chunk: codes, 8-bit constant and group scale
+    // this thread's block of the first chunk: codes, then the 8-bit constant
+    // and group scale (or, kNoDq, the fp32 constant in ps2)
     int64_t ch = blockIdx.x;
     uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
     uint32_t pq = 0;
@@ -283,8 +288,12 @@ __global__ void __launch_bounds__(kDeqChunk) nf4_dequant_kernel(const __grid_con
         const int64_t b = ch * kDeqChunk + t;
         p0 = __ldcs(codes + 2 * b);
         p1 = __ldcs(codes + 2 * b + 1);
-        pq = q[b];
-        ps2 = s2[b / kGroup];
+        if (kNoDq) {
+            ps2 = absmax[b];
+        } else {
+            pq = q[b];
+            ps2 = s2[b / kGroup];
+        }
     }
     for (int it = 0; ch < nchunks; ch += gridDim.x, ++it) {
         const int64_t b = ch * kDeqChunk + t;
@@ -296,10 +305,14 @@ __global__ void __launch_bounds__(kDeqChunk) nf4_dequant_kernel(const __grid_con
         if (nb < nblocks) {
             n0 = __ldcs(codes + 2 * nb);
             n1 = __ldcs(codes + 2 * nb + 1);
-            nq = q[nb];
-            ns2 = s2[nb / kGroup];
+            if (kNoDq) {
+                ns2 = absmax[nb];
+            } else {
+                nq = q[nb];
+                ns2 = s2[nb / kGroup];
+            }
         }
-        const float cprime = (b < nblocks) ? __fmaf_rn(e4m3_to_f32(pq), ps2, mu) : 0.0f;
+        const float cprime = (b < nblocks) ? (kNoDq ? ps2 : __fmaf_rn(e4m3_to_f32(pq), ps2, mu)) : 0.0f;
         const Nf4BlockLut lut = make_block_lut(tab.level, cprime);
 
         uint8_t* tile = tiles + (it & 1) * (kDeqChunk * 128);
@@ -332,20 +345,25 @@ __global__ void __launch_bounds__(kDeqChunk) nf4_dequant_kernel(const __grid_con
 // ---------------------------------------------------------------------------
 // Decoded constants transposed for the matmul kernels: cT[kb * ldc + n] =
 // c' of block (n, kb), so a run of consecutive output rows n for one k-block
-// is contiguous (one TMA box). 32 x 32 tiles through shared memory.
+// is contiguous (one TMA box). 32 x 32 tiles through shared memory. kNoDq:
+// the constants are the weight's fp32 absmax values, transposed unchanged.
 // ---------------------------------------------------------------------------
+template <bool kNoDq>
 __global__ void __launch_bounds__(256) decode_constants_t_kernel(const uint8_t* __restrict__ q,
                                                                   const float* __restrict__ s2,
-                                                                  const float* __restrict__ mean, int64_t N,
+                                                                  const float* __restrict__ mean,
+                                                                  const float* __restrict__ absmax, int64_t N,
                                                                   int64_t KB, int64_t ldc,
                                                                   float* __restrict__ cT) {
     __shared__ float tile[32][33];
-    const float mu = *mean;
+    const float mu = kNoDq ? 0.0f : *mean;
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 32, kb0 = static_cast<int64_t>(blockIdx.x) * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
     for (int i = ty; i < 32; i += 8) {
         const int64_t n = n0 + i, kb = kb0 + tx;
-        tile[i][tx] = (n < N && kb < KB) ? decode_constant(q, s2, mu, n * KB + kb) : 0.0f;
+        float c = 0.0f;
+        if (n < N && kb < KB) c = kNoDq ? absmax[n * KB + kb] : decode_constant(q, s2, mu, n * KB + kb);
+        tile[i][tx] = c;
     }
     __syncthreads();
     for (int i = ty; i < 32; i += 8) {
@@ -422,22 +440,29 @@ cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_sc
     return cudaGetLastError();
 }
 
-cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const uint8_t* q, const float* s2,
-                               const float* mean, int64_t N, int64_t K, const Nf4Tables& tab, int num_sms,
-                               cudaStream_t st) {
+cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const BlockConstants& c, int64_t N,
+                               int64_t K, const Nf4Tables& tab, int num_sms, cudaStream_t st) {
     const int64_t nb = N * K / kBlock;
     const int64_t nchunks = (nb + kDeqChunk - 1) / kDeqChunk;
     const int grid = static_cast<int>(std::min<int64_t>(nchunks, static_cast<int64_t>(num_sms) * 6));
-    nf4_dequant_kernel<<<grid, kDeqChunk, kDequantSmem, st>>>(out_map, reinterpret_cast<const uint4*>(codes), q, s2,
-                                                               mean, nb, tab);
+    const uint4* cw = reinterpret_cast<const uint4*>(codes);
+    if (c.absmax)
+        nf4_dequant_kernel<true><<<grid, kDeqChunk, kDequantSmem, st>>>(out_map, cw, nullptr, nullptr, nullptr,
+                                                                         c.absmax, nb, tab);
+    else
+        nf4_dequant_kernel<false><<<grid, kDeqChunk, kDequantSmem, st>>>(out_map, cw, c.qabsmax, c.s2, c.mean,
+                                                                          nullptr, nb, tab);
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_constants_t(const uint8_t* q, const float* s2, const float* mean, int64_t N, int64_t K,
-                                      int64_t ldc, float* cT, cudaStream_t st) {
+cudaError_t launch_decode_constants_t(const BlockConstants& c, int64_t N, int64_t K, int64_t ldc, float* cT,
+                                      cudaStream_t st) {
     const int64_t KB = K / kBlock;
     dim3 grid(static_cast<unsigned>((KB + 31) / 32), static_cast<unsigned>((ldc + 31) / 32));
-    decode_constants_t_kernel<<<grid, 256, 0, st>>>(q, s2, mean, N, KB, ldc, cT);
+    if (c.absmax)
+        decode_constants_t_kernel<true><<<grid, 256, 0, st>>>(nullptr, nullptr, nullptr, c.absmax, N, KB, ldc, cT);
+    else
+        decode_constants_t_kernel<false><<<grid, 256, 0, st>>>(c.qabsmax, c.s2, c.mean, nullptr, N, KB, ldc, cT);
     return cudaGetLastError();
 }
 

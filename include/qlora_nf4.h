@@ -38,6 +38,12 @@
  *   mean    float[1]      mean of all first-level absmax constants
  *   Dequantised weight: c'_b = fmaf(E4M3(qabsmax_b), s2_g, mean) (one fp32
  *   rounding), w_hat = bf16_rn(fp32_rn(level[code] * c'_b)).
+ *
+ * Storage without double quantisation (absmax set in qlora_nf4_weight): the
+ * same codes, and one fp32 constant per block, absmax float[nb] = the block's
+ * max|w| itself, 4 + 32/64 = 4.5 bits per weight [explainer 二重量子化, the
+ * count before the constants are quantised]. w_hat = bf16_rn(fp32_rn(
+ * level[code] * absmax_b)).
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -63,8 +69,11 @@ typedef int qlora_status;
 #define QLORA_ERR_UNSUPPORTED_DEVICE   -8  /* current device is not sm_100             */
 #define QLORA_ERR_EXCEEDS_STATIC_SCRATCH -9 /* N*K above the no-allocation limit        */
 
-/* Read-only view of a quantised weight. All five pointers are device
- * pointers owned by the caller; the library never writes through them. */
+/* Read-only view of a quantised weight. All pointers are device pointers
+ * owned by the caller; the library never writes through them. With absmax
+ * NULL (zero-initialised) the weight uses double quantisation and qabsmax,
+ * s2 and mean are required; with absmax set it is stored without, and
+ * qabsmax, s2 and mean are ignored (they may be NULL). */
 typedef struct {
     const uint8_t* codes;
     const uint8_t* qabsmax;
@@ -72,6 +81,7 @@ typedef struct {
     const float*   mean;
     int64_t        N;
     int64_t        K;
+    const float*   absmax;
 } qlora_nf4_weight;
 
 /* Sizes in bytes of the four buffers of an N x K quantised weight. Host only;
@@ -140,9 +150,36 @@ qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, int64_t K,
                                         uint8_t* codes, uint8_t* qabsmax, float* s2, float* mean,
                                         void* stream);
 
+/* Quantise without double quantisation [explainer 二重量子化, first
+ * paragraph: one fp32 constant per block of 64, 4.5 bits per weight].
+ * Codes exactly as qlora_quantize_nf4 (same rule, same bits); absmax
+ * (float[N*K/64], device) receives each block's max|w|. W is fp32 [N, K]
+ * (qlora_quantize_nf4_nodq) or bf16 [N, K] (qlora_quantize_nf4_bf16_nodq,
+ * the bits of its fp32 upcast). No workspace; one kernel launch. Use the
+ * result through a qlora_nf4_weight with absmax set. */
+qlora_status qlora_quantize_nf4_nodq(const float* W, int64_t N, int64_t K,
+                                     uint8_t* codes, float* absmax, void* stream);
+qlora_status qlora_quantize_nf4_bf16_nodq(const uint16_t* W, int64_t N, int64_t K,
+                                          uint8_t* codes, float* absmax, void* stream);
+
 /* Dequantise to bf16 [N, K] (device W_out), bit-exact with the format's
- * definition above. [explainer 量子化を1段落で: x_hat = c * level[code]] */
+ * definition above, for either storage. [explainer 量子化を1段落で:
+ * x_hat = c * level[code]] */
 qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream);
+
+/* Fold an adapter into a 16-bit copy of the weight for inference [waylandz
+ * 26.2.2, inference: merge once, W_merged = W + (alpha/r) B A; explainer
+ * 落とし穴: the merge goes to the 16-bit weight, not to the 4-bit one]:
+ *   W_out = bf16_rn( fmaf(s, sum_j B[n, j] A[j, k], w_hat[n, k]) ),  s = alpha/r,
+ * w_hat the dequantised weight above (either storage), the rank-r sum of
+ * exact bf16 products accumulated in fp32 (order unspecified): an entry is
+ * off the exact merge by at most one bf16 step plus that fp32 error.
+ * A: bf16 [r, K]; B: bf16 [N, r]; W_out: bf16 [N, K] (device, caller-owned);
+ * r in {8, 16, 32, 64}. No workspace. Errors as for qlora_linear_fwd. To
+ * store the merged weight in 4 bits again, quantise W_out with
+ * qlora_quantize_nf4_bf16 (the update may be lost, as the explainer warns). */
+qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
+                              int r, float alpha, uint16_t* W_out, void* stream);
 
 /* Forward of the QLoRA linear layer [waylandz 26.2.4; explainer 勾配は...]:
  *   sT = bf16( s * X A^T )                    (M x r, written to sT_save if not NULL)

@@ -110,6 +110,36 @@ def test_host_validation_without_gpu(q):
     assert bwd(wsb=bws - 256) == -5
 
 
+def test_host_validation_storage_without_dq_and_merge(q):
+    L = q.lib()
+    P = 0x7000000
+    # a weight without double quantisation needs only codes and absmax
+    nodq = q.Nf4WeightC(P, None, None, None, 512, 512, P + 0x100000)
+    bad = q.Nf4WeightC(P, None, None, None, 512, 512, None)   # neither storage complete
+    mis = q.Nf4WeightC(P, None, None, None, 512, 512, P + 4)
+    assert L.qlora_dequantize_nf4(ctypes.byref(bad), P, None) == -1
+    assert L.qlora_dequantize_nf4(ctypes.byref(mis), P, None) == -3
+    assert L.qlora_dequantize_nf4(ctypes.byref(nodq), None, None) == -1
+    # quantise without double quantisation
+    for entry in (L.qlora_quantize_nf4_nodq, L.qlora_quantize_nf4_bf16_nodq):
+        assert entry(P, 512, 500, P, P, None) == -2
+        assert entry(P, 0, 512, P, P, None) == -2
+        assert entry(None, 512, 512, P, P, None) == -1
+        assert entry(P, 512, 512, P, None, None) == -1
+        assert entry(P, 512, 512, P, P + 4, None) == -3
+    # merge
+    w = _weight(q)
+    merge = lambda **kw: L.qlora_merge_lora(ctypes.byref(kw.get("w", w)), kw.get("A", P), kw.get("B", P),
+                                            kw.get("r", 8), kw.get("alpha", 16.0), kw.get("out", P), None)
+    assert merge(r=12) == -4
+    assert merge(A=None) == -1
+    assert merge(out=None) == -1
+    assert merge(alpha=float("inf")) == -1
+    assert merge(B=P + 2) == -3
+    assert merge(w=bad) == -1
+    assert merge(w=_weight(q, N=12)) == -2
+
+
 def test_host_fault_injection(q):
     """An injected launch failure is reported as QLORA_ERR_CUDA with its text,
     and nothing reaches a GPU (none is needed for this test)."""
