@@ -13,18 +13,24 @@
 //
 // The rank-r product is a dense contraction, so it runs on mma.m16n8k16: a
 // warp unit is 16 weight rows (MMA rows) by one 64-column NF4 block column
-// (eight n8 MMA tiles, tile t covering columns 8t .. 8t + 7), r/16 MMA steps
-// over the rank (r = 8 pads the upper half of its one step with zeros). The
-// A operand is B's rows (row-major, rank pairs contiguous); the B operand is
-// columns of A, gathered with 16-bit loads once per block column and kept in
-// registers while the warp walks down the rows (units are ordered block
-// column first, row group second, and each warp takes one contiguous range).
-// Lane (g, q) holds the sums of rows g and g + 8 at columns 8t + 2q, 8t + 2q
-// + 1, whose codes are byte q of each 32-bit word of the block's 32 packed
-// bytes: two byte permutes per pair of words gather them, and the per-block
-// lookup table turns them into the bf16 pairs of w_hat. The bf16 results go
-// straight to global memory, 4 bytes per lane and tile; a warp's stores
-// cover 128 contiguous bytes of each of its 16 rows.
+// (eight n8 MMA tiles), r/16 MMA steps over the rank (r = 8 pads the upper
+// half of its one step with zeros). The A operand is B's rows (row-major,
+// rank pairs contiguous); the B operand is columns of A, gathered with 16-bit
+// loads once per block column and kept in registers while the warp walks
+// down the rows (units are ordered block column first, row group second, and
+// each warp takes one contiguous range).
+//
+// The columns of the eight tiles are permuted so that lane (g, q), which
+// holds the sums of rows g and g + 8 at MMA columns 2q and 2q + 1 of every
+// tile, owns block columns 8q .. 8q + 7 (tiles 0-3) and 32 + 8q .. 39 + 8q
+// (tiles 4-7): MMA column c of tile t is block column
+//   8 (c / 2) + 32 (t / 4) + 2 (t % 4) + c % 2.
+// So the lane's codes are two whole 32-bit words of the block's 32 packed
+// bytes (words q and 4 + q), decoded by the per-block lookup table into the
+// bf16 pairs of w_hat in tile order, and its results leave as two 16-byte
+// stores per row: one warp store covers 64 contiguous bytes of each of 8
+// rows (whole 32-byte sectors). The next unit's codes, constants and rank
+// rows are loaded while the current one is computed.
 //
 // The kernel is bound by HBM: 0.5 B of codes, 1/64 B of constants and 2 B of
 // output per weight; A and B are read from L2.
@@ -39,39 +45,81 @@ namespace {
 
 constexpr int kMergeWarps = 8;
 constexpr int kMergeThreads = kMergeWarps * 32;
+// CTAs per SM the register budget is set for (the B-operand cache grows
+// with r: 64 registers at r = 64)
+template <int R>
+constexpr int kMergeMinBlocks = R >= 64 ? 1 : 2;
 
 // A[j, kk] | A[j + 1, kk] << 16: a bf16 pair of consecutive rank rows
 __device__ __forceinline__ uint32_t rank_pair(const uint16_t* A, int j, int64_t kk, int64_t K) {
     return static_cast<uint32_t>(__ldg(A + j * K + kk)) | (static_cast<uint32_t>(__ldg(A + (j + 1) * K + kk)) << 16);
 }
 
-template <bool kNoDq>
-__device__ __forceinline__ float block_constant(const BlockConstants& c, int64_t b, float mu) {
-    if (kNoDq) return __ldg(c.absmax + b);
-    return __fmaf_rn(e4m3_to_f32(__ldg(c.qabsmax + b)), __ldg(c.s2 + (b >> 8)), mu);
+// Loads of one unit that do not depend on the block column's A fragments.
+template <int S, bool kNoDq>
+struct UnitLoads {
+    uint32_t codes[2][2];  // rows g, g + 8: words q and 4 + q of the block
+    uint32_t qa[2];        // E4M3 constants (or, kNoDq, fp32 constants as bits)
+    float s2[2];
+    uint32_t af[S][4];     // A operand: rows g, g + 8 of B, rank pairs 2q (+8)
+};
+
+template <int R, bool kNoDq>
+__device__ __forceinline__ void load_unit(const MergeArgs& a, int64_t kb, int64_t rg, int g, int q,
+                                          UnitLoads<(R >= 16 ? R / 16 : 1), kNoDq>& L) {
+    constexpr int S = R >= 16 ? R / 16 : 1;
+    const int64_t N = a.N, K = a.K, KB = K / kBlock;
+    // rows past N read row N - 1; their results are not stored
+    const int64_t rows[2] = {min(rg * 16 + g, N - 1), min(rg * 16 + g + 8, N - 1)};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(a.codes + rows[h] * (K / 2) + kb * 32);
+        L.codes[h][0] = __ldg(cw + q);
+        L.codes[h][1] = __ldg(cw + 4 + q);
+        const int64_t b = rows[h] * KB + kb;
+        if (kNoDq) {
+            L.qa[h] = __float_as_uint(__ldg(a.c.absmax + b));
+            L.s2[h] = 0.0f;
+        } else {
+            L.qa[h] = __ldg(a.c.qabsmax + b);
+            L.s2[h] = __ldg(a.c.s2 + (b >> 8));
+        }
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const uint16_t* p = a.B + rows[h] * R + 16 * s + 2 * q;
+            L.af[s][h] = __ldg(reinterpret_cast<const uint32_t*>(p));
+            L.af[s][2 + h] = R >= 16 ? __ldg(reinterpret_cast<const uint32_t*>(p + 8)) : 0u;
+        }
+    }
 }
 
 template <int R, bool kNoDq>
-__global__ void __launch_bounds__(kMergeThreads) merge_lora_kernel(const MergeArgs a, const Nf4Tables tab) {
+__global__ void __launch_bounds__(kMergeThreads, kMergeMinBlocks<R>) merge_lora_kernel(const MergeArgs a, const Nf4Tables tab) {
     constexpr int S = R >= 16 ? R / 16 : 1;  // k16 MMA steps over the rank
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int64_t N = a.N, K = a.K, KB = K / kBlock, RG = (N + 15) / 16, U = RG * KB;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * kMergeWarps;
     const int64_t w = static_cast<int64_t>(blockIdx.x) * kMergeWarps + (threadIdx.x >> 5);
-    const int64_t u_end = U * (w + 1) / warps;
+    const int64_t u_begin = U * w / warps, u_end = U * (w + 1) / warps;
+    if (u_begin >= u_end) return;
     const float mu = kNoDq ? 0.0f : __ldg(a.c.mean);
-    const uint32_t sel = static_cast<uint32_t>(q) | (static_cast<uint32_t>(q + 4) << 4);  // byte q of two words
 
     uint32_t bf[8][S][2];  // B operand of tile t, step s (columns of A)
     int64_t kb_loaded = -1;
+    UnitLoads<S, kNoDq> cur;
+    load_unit<R, kNoDq>(a, u_begin / RG, u_begin % RG, g, q, cur);
 #pragma unroll 1
-    for (int64_t u = U * w / warps; u < u_end; ++u) {
+    for (int64_t u = u_begin; u < u_end; ++u) {
         const int64_t kb = u / RG, rg = u - kb * RG, k0 = kb * kBlock;
+        // the next unit's loads (the last unit reloads itself)
+        const int64_t un = u + 1 < u_end ? u + 1 : u;
+        UnitLoads<S, kNoDq> nxt;
+        load_unit<R, kNoDq>(a, un / RG, un % RG, g, q, nxt);
         if (kb != kb_loaded) {
             kb_loaded = kb;
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-                const int64_t kk = k0 + 8 * t + g;
+                const int64_t kk = k0 + 8 * (g >> 1) + 32 * (t >> 2) + 2 * (t & 3) + (g & 1);
 #pragma unroll
                 for (int s = 0; s < S; ++s) {
                     bf[t][s][0] = rank_pair(a.A, 16 * s + 2 * q, kk, K);
@@ -79,69 +127,36 @@ __global__ void __launch_bounds__(kMergeThreads) merge_lora_kernel(const MergeAr
                 }
             }
         }
-        // rows g and g + 8 of the group; loads of rows past N read row N - 1
-        // and their results are not stored
-        const int64_t nA = rg * 16 + g, nB = nA + 8;
-        const int64_t rA = nA < N ? nA : N - 1, rB = nB < N ? nB : N - 1;
-        uint32_t af[S][4];
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            const uint16_t* pa = a.B + rA * R + 16 * s + 2 * q;
-            const uint16_t* pb = a.B + rB * R + 16 * s + 2 * q;
-            af[s][0] = __ldg(reinterpret_cast<const uint32_t*>(pa));
-            af[s][1] = __ldg(reinterpret_cast<const uint32_t*>(pb));
-            af[s][2] = R >= 16 ? __ldg(reinterpret_cast<const uint32_t*>(pa + 8)) : 0u;
-            af[s][3] = R >= 16 ? __ldg(reinterpret_cast<const uint32_t*>(pb + 8)) : 0u;
-        }
-        const uint4* pcA = reinterpret_cast<const uint4*>(a.codes + rA * (K / 2) + kb * 32);
-        const uint4* pcB = reinterpret_cast<const uint4*>(a.codes + rB * (K / 2) + kb * 32);
-        const uint4 cA0 = __ldg(pcA), cA1 = __ldg(pcA + 1), cB0 = __ldg(pcB), cB1 = __ldg(pcB + 1);
-        const float cvA = block_constant<kNoDq>(a.c, rA * KB + kb, mu);
-        const float cvB = block_constant<kNoDq>(a.c, rB * KB + kb, mu);
 
         float acc[8][4];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
 #pragma unroll
-            for (int s = 0; s < S; ++s) mma_bf16(acc[t], af[s], bf[t][s][0], bf[t][s][1]);
-        }
-
-        // byte q of words 0..3 and 4..7: the codes of columns 8t + 2q (high
-        // nibble) and 8t + 2q + 1 (low nibble) for t = 0..3 and 4..7
-        auto gather = [sel](uint32_t x, uint32_t y, uint32_t z, uint32_t v) {
-            return __byte_perm(__byte_perm(x, y, sel), __byte_perm(z, v, sel), 0x5410);
-        };
-        uint32_t hA[8], hB[8];  // w_hat pairs of tile t (column 8t + 2q in the low half)
-        {
-            const Nf4BlockLut lA = make_block_lut(tab.level, cvA);
-            uint32_t o0[4], o1[4];
-            lut_decode8(lA, gather(cA0.x, cA0.y, cA0.z, cA0.w), o0);
-            lut_decode8(lA, gather(cA1.x, cA1.y, cA1.z, cA1.w), o1);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) hA[i] = o0[i], hA[i + 4] = o1[i];
-        }
-        {
-            const Nf4BlockLut lB = make_block_lut(tab.level, cvB);
-            uint32_t o0[4], o1[4];
-            lut_decode8(lB, gather(cB0.x, cB0.y, cB0.z, cB0.w), o0);
-            lut_decode8(lB, gather(cB1.x, cB1.y, cB1.z, cB1.w), o1);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) hB[i] = o0[i], hB[i + 4] = o1[i];
+            for (int s = 0; s < S; ++s) mma_bf16(acc[t], cur.af[s], bf[t][s][0], bf[t][s][1]);
         }
 
         const float sc = a.scale;
-        uint16_t* outA = a.W_out + nA * K + k0 + 2 * q;
-        uint16_t* outB = a.W_out + nB * K + k0 + 2 * q;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const uint32_t vA = pack_bf16x2(__fmaf_rn(sc, acc[t][0], __uint_as_float(hA[t] << 16)),
-                                            __fmaf_rn(sc, acc[t][1], __uint_as_float(hA[t] & 0xFFFF0000u)));
-            const uint32_t vB = pack_bf16x2(__fmaf_rn(sc, acc[t][2], __uint_as_float(hB[t] << 16)),
-                                            __fmaf_rn(sc, acc[t][3], __uint_as_float(hB[t] & 0xFFFF0000u)));
-            if (nA < N) *reinterpret_cast<uint32_t*>(outA + 8 * t) = vA;
-            if (nB < N) *reinterpret_cast<uint32_t*>(outB + 8 * t) = vB;
+        for (int h = 0; h < 2; ++h) {
+            const int64_t n = rg * 16 + g + 8 * h;
+            const float c = kNoDq ? __uint_as_float(cur.qa[h]) : __fmaf_rn(e4m3_to_f32(cur.qa[h]), cur.s2[h], mu);
+            const Nf4BlockLut lut = make_block_lut(tab.level, c);
+            uint32_t wh[8];  // w_hat pairs of tile t: columns of MMA columns 2q, 2q + 1
+            lut_decode8(lut, cur.codes[h][0], *reinterpret_cast<uint32_t(*)[4]>(wh));
+            lut_decode8(lut, cur.codes[h][1], *reinterpret_cast<uint32_t(*)[4]>(wh + 4));
+            uint32_t v[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                v[t] = pack_bf16x2(__fmaf_rn(sc, acc[t][2 * h], __uint_as_float(wh[t] << 16)),
+                                   __fmaf_rn(sc, acc[t][2 * h + 1], __uint_as_float(wh[t] & 0xFFFF0000u)));
+            if (n < N) {
+                uint4* o = reinterpret_cast<uint4*>(a.W_out + n * K + k0 + 8 * q);
+                o[0] = make_uint4(v[0], v[1], v[2], v[3]);  // columns 8q .. 8q + 7
+                o[4] = make_uint4(v[4], v[5], v[6], v[7]);  // columns 32 + 8q .. 39 + 8q
+            }
         }
+        cur = nxt;
     }
 }
 
