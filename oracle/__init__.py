@@ -11,6 +11,9 @@ Two halves:
   * forward and backward of the layer in fp64 with numpy matmuls as the only
     library step ([p2] "26.2.4 スケーリング係数アルファ": y = W x + (alpha/r) B (A x);
     gradients by the chain rule, none for the frozen W, [p1] "勾配は実際どこへ行くのか").
+Beside them: storage without double quantisation, the adapter merge with its
+one-step fp64 -> bf16 rounding, a batch whose rows use different adapters over
+one base, and projections that share their input.
 """
 from __future__ import annotations
 
@@ -323,6 +326,50 @@ def merge_lora(What, A, B, alpha: float, r: int) -> np.ndarray:
 def merge_lora_bf16_bits(What, A, B, alpha: float, r: int) -> np.ndarray:
     """merge_lora rounded once to bf16 (uint16 bit patterns)."""
     return f64_to_bf16_bits(merge_lora(What, A, B, alpha, r))
+
+
+# ------------------------------------------------- several adapters, one base --
+
+def forward_multi(X, What, As, Bs, ids, alpha: float, r: int):
+    """Y for a batch whose token rows use different adapters over one frozen
+    base: row m uses adapter ids[m], Y_m = X_m What^T + (alpha/r) (X_m A_k^T)
+    B_k^T with k = ids[m]. [p2] 26.7.3: one base model hosts many adapters and
+    switches between them at run time; [p3] 利用ケース: one 4-bit base serves
+    several adapters. As: [P, r, K]; Bs: [P, N, r]; ids: int [M] in [0, P).
+    Written as the single-adapter forward applied to each adapter's rows."""
+    ids = np.asarray(ids)
+    if ids.size and (ids.min() < 0 or ids.max() >= len(As)):
+        raise ValueError("adapter id out of range")
+    Y = np.zeros((X.shape[0], What.shape[0]))
+    for k in range(len(As)):
+        rows = np.flatnonzero(ids == k)
+        if rows.size:
+            Y[rows], _ = forward(X[rows], What, As[k], Bs[k], alpha, r)
+    return Y
+
+
+def backward_multi(dY, X, What, As, Bs, ids, alpha: float, r: int):
+    """Gradients of <dY, forward_multi>: dX row by row with the row's adapter;
+    dA_k and dB_k from the rows that use adapter k only (zero for an adapter no
+    row uses)."""
+    ids = np.asarray(ids)
+    dX = np.zeros_like(X, dtype=np.float64)
+    dAs = np.zeros((len(As),) + As[0].shape)
+    dBs = np.zeros((len(Bs),) + Bs[0].shape)
+    for k in range(len(As)):
+        rows = np.flatnonzero(ids == k)
+        if rows.size:
+            dX[rows], dAs[k], dBs[k] = backward(dY[rows], X[rows], What, As[k], Bs[k], alpha, r)
+    return dX, dAs, dBs
+
+
+# ------------------------------------------ projections that share the input --
+
+def forward_group(X, Whats, As, Bs, alpha: float, r: int):
+    """Projections of one input with their own frozen weights and adapters
+    (q, k, v of attention, or gate and up of the MLP), outputs side by side:
+    [Y_1 | Y_2 | ...], Y_i the layer's forward with (What_i, A_i, B_i)."""
+    return np.concatenate([forward(X, Wi, Ai, Bi, alpha, r)[0] for Wi, Ai, Bi in zip(Whats, As, Bs)], axis=1)
 
 
 def rel_err(got, ref) -> float:
