@@ -12,10 +12,12 @@
  *     none; only A and B are trained);
  *   - "QLoRA" glossary (ultralytics), the NF4 level construction and the
  *     nearest-level argmin;
- *   - "waylandz LLM book ch.26", 26.2.4: y = W x + (alpha/r) B (A x).
+ *   - "waylandz LLM book ch.26", 26.2.4: y = W x + (alpha/r) B (A x); 26.2.2:
+ *     the adapter merged once for inference, W + (alpha/r) B A.
  *
  * Conventions
- *   W is N x K row-major fp32 (N = out features, K = in features), K % 64 == 0.
+ *   W is N x K row-major fp32 (bf16 for the *_bf16 quantisers; N = out
+ *   features, K = in features), K % 64 == 0.
  *   X is M x K, Y is M x N, A is r x K, B is N x r, dY is M x N, all row-major.
  *   bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
  *   s = alpha / r.
