@@ -178,3 +178,27 @@ def test_merge_rounding_brute_force(seed):
         for k in range(K):
             exact = Fraction(What[n, k]) + s * sum(Fraction(B[n, j]) * Fraction(A[j, k]) for j in range(r))
             assert got[n, k] == _brute_bf16(exact), (n, k)
+
+
+def test_requantised_merge_loses_the_update():
+    """The explainer's 落とし穴: an adapter update added to the 4-bit weight and
+    quantised again is mostly lost, so the merge goes to 16 bits. With an
+    update of 5 % of the weights' rms, the bf16 merge keeps it to within 10 %,
+    while quantising the merged weight to NF4 again leaves an error as large as
+    the update itself."""
+    rng = np.random.default_rng(30)
+    N, K, r = 256, 512, 16
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    z = oracle.quantize_nf4(W)
+    What = oracle.bf16_bits_to_f64(oracle.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], N, K))
+    A = rng.standard_normal((r, K)) * np.sqrt(2 / r)
+    B = rng.standard_normal((N, r))
+    B *= 0.05 * 0.02 / np.sqrt(np.mean((B @ A) ** 2))  # alpha = r: s = 1
+    update = oracle.merge_lora(What, A, B, float(r), r) - What
+    Wm = oracle.bf16_bits_to_f64(oracle.merge_lora_bf16_bits(What, A, B, float(r), r))
+    z2 = oracle.quantize_nf4(Wm.astype(np.float32))
+    Wrq = oracle.bf16_bits_to_f64(oracle.dequant_bf16_bits(z2["codes"], z2["qabsmax"], z2["s2"], z2["mean"], N, K))
+    err16 = np.linalg.norm(Wm - What - update) / np.linalg.norm(update)
+    err4 = np.linalg.norm(Wrq - What - update) / np.linalg.norm(update)
+    assert err16 < 0.1
+    assert err4 > 0.9
