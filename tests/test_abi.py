@@ -38,6 +38,21 @@ def test_every_declared_symbol_is_exported(q):
     assert set(names) == set(q._SIGNATURES)
 
 
+def test_binding_arity_matches_header(q):
+    """Every binding signature has as many arguments as the header's
+    prototype, and the weight struct as many fields as qlora_nf4_weight."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = re.findall(r"\b(qlora_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert len(protos) == len(q._SIGNATURES)
+    for name, params in protos:
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        assert len(q._SIGNATURES[name][1]) == n, name
+    struct = re.search(r"typedef struct \{(.*?)\} qlora_nf4_weight;", text, flags=re.S).group(1)
+    fields = [f for f in struct.split(";") if f.strip()]
+    assert [f[0] for f in q.Nf4WeightC._fields_] == [f.split()[-1] for f in fields]
+
+
 def test_nf4_bytes_match_oracle_storage(q):
     for N, K in [(512, 512), (4096, 4096), (11008, 4096), (8192, 22016), (8, 64)]:
         sz = q.nf4_bytes(N, K)
