@@ -185,3 +185,19 @@ def test_status_strings_and_options(q):
         q.set_option(q.OPT_WAIT_TIMEOUT_US, 0)
     with pytest.raises(q.QLoraError):
         q.set_option(99, 1)
+
+
+def test_missing_library_fails_loudly():
+    """Without the built library every call raises: there is no CPU path.
+    Run in a fresh interpreter with the library path pointed elsewhere."""
+    import subprocess
+    import sys
+    code = ("import bit_nf4_quantized_09_b200 as q\n"
+            "q.LIB_PATH = '/nonexistent/libqlora_nf4.so'\n"
+            "q._lib = None\n"
+            "try:\n"
+            "    q.nf4_tables()\n"
+            "except ImportError as e:\n"
+            "    print('raised', 'no CPU fallback' in str(e))\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.stdout.strip() == "raised True", out.stdout + out.stderr
