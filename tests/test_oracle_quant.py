@@ -343,3 +343,18 @@ def test_dequant_round_trip_and_zero_sign():
     cp = np.repeat(cprime.astype(np.float64).reshape(64, 4), 64, axis=1)
     err = np.abs(What - W)
     assert np.all(err <= blk * gap + np.abs(cp - blk) + np.abs(W) * 2 ** -8 + 1e-12)
+
+
+def test_no_negative_decoded_constant_on_the_workloads():
+    """Reading: a decoded constant c' = E4M3(q) s2 + mean is not clamped, so
+    a tiny block next to a large mean could get c' < 0. Count it over every
+    block of every workload weight: none. The sign is taken from the exact
+    sum (E4M3 times s2 is exact in fp64, and adding the fp32 mean cannot flip
+    the sign of a nonzero value), which is the sign of the fp32 fma."""
+    import synth
+    e4 = np.array([oracle.e4m3_decode(v) for v in range(256)])
+    for cfg in (synth.TINY, synth.ATTN7B, *synth.MLP7B, *synth.L65B):
+        z = oracle.quantize_nf4(synth.weight(cfg).numpy())
+        nb = z["qabsmax"].size
+        cp = e4[z["qabsmax"]] * z["s2"].astype(np.float64)[np.arange(nb) // 256] + np.float64(z["mean"])
+        assert np.count_nonzero(cp <= 0) == 0, cfg.name
