@@ -97,3 +97,24 @@ def test_rel_err_metric():
     assert oracle.rel_err([1.0, 2.0], [1.0, 2.0]) == 0.0
     assert oracle.rel_err([1.0, 2.5], [1.0, 2.0]) == 0.25
     assert oracle.rel_err([0.0], [0.0]) == 0.0
+
+
+def test_alpha_scaling_is_linear_and_b_zero_is_the_base_layer():
+    """Y(alpha) - Y(0) grows linearly with alpha ([p2] 26.2.4: the update is
+    scaled by alpha/r), and B = 0 leaves the base layer X W^T with dA = 0 and
+    dB = s dY^T (X A^T)."""
+    rng = np.random.default_rng(40)
+    M, N, K, r = 6, 10, 12, 4
+    X, W, A, B, dY = (rng.standard_normal(s) for s in ((M, K), (N, K), (r, K), (N, r), (M, N)))
+    Y0, _ = oracle.forward(X, W, A, B, 0.0, r)
+    Y1, _ = oracle.forward(X, W, A, B, 8.0, r)
+    Y3, _ = oracle.forward(X, W, A, B, 24.0, r)
+    assert np.allclose(Y3 - Y0, 3.0 * (Y1 - Y0), rtol=1e-12, atol=1e-12)
+    assert np.allclose(Y0, X @ W.T, rtol=1e-13, atol=1e-13)
+    Zb = np.zeros_like(B)
+    Yb, _ = oracle.forward(X, W, A, Zb, 8.0, r)
+    assert np.array_equal(Yb, X @ W.T + 0.0)
+    dX, dA, dB = oracle.backward(dY, X, W, A, Zb, 8.0, r)
+    assert not dA.any()
+    assert np.allclose(dB, (8.0 / r) * dY.T @ (X @ A.T), rtol=1e-13, atol=1e-13)
+    assert np.allclose(dX, dY @ W, rtol=1e-13, atol=1e-13)
