@@ -1,20 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the frozen-NF4 QLoRA linear layer on B200.
 
-One step = one pass of the whole hot path over one batch, on inputs already
-resident in HBM:
-    quantize W (fp32 -> NF4 + double quant) -> dequantize to bf16
-    -> forward (Y, sT) -> backward (dX, dA, dB)
-Workload: the LLaMA-7B attention projection, W 4096 x 4096 (0.1% outliers),
-M = 4096 tokens (8 x 512), r = 16, alpha = 32, synthetic seeded inputs.
-Two input sets alternate between steps; one step touches ~0.26 GB, more than
-the 126 MB L2.
+Headline workload: the 65B-scale MLP pair, the up projection W 22016 x 8192
+and the down projection W 8192 x 22016, each ~N(0, 0.015), M = 2048 tokens
+(4 x 512), LoRA r = 64, alpha = 16, synthetic seeded inputs. One step is one
+pass of the whole hot path over one batch, on inputs already resident in HBM,
+for each of the two linears:
+    quantize W (fp32 -> NF4 + double quant)
+    -> forward (Y, sT; the weight dequantised inside the matmul)
+    -> backward (dX through deq(W), dA, dB)
+No bf16 copy of either weight is written (weight bytes 4-bit only); the
+standalone dequantiser is timed as its own row. Two input sets alternate
+between steps (about 3.4 GB, far more than the 126 MB L2).
 
-Metric value: fwd+bwd algorithmic TFLOP/s = (4MNK + 6Mr(N+K)) / step time,
-whole job (all ranks). Under torchrun every rank runs an independent replica
-(weak scaling, no collective on the data path); timing is the max over ranks.
+Metric value: fwd+bwd algorithmic TFLOP/s = sum over the two linears of
+(4MNK + 6Mr(N+K)) / step time, whole job (all ranks). Under torchrun every
+rank runs an independent replica (weak scaling, no collective on the data
+path); timing is the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --case step|fwd:<workload>|bwd:<workload>|quantize:<workload>|
+                           dequantize:<workload>|merge:<workload> [--reps R]
+        (one call repeated, for profiler captures; prints nothing else)
 """
 from __future__ import annotations
 
@@ -40,9 +47,11 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and tokens/s; NF4 dequant GB/s (% of roofline)"
-CFG = synth.ATTN7B
+HEADLINE = synth.L65B[1:]  # MLP up 22016 x 8192, down 8192 x 22016; M 2048, r 64
+WORKLOAD = "65b_mlp_up22016x8192_down8192x22016_m2048_r64"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0  # dense bf16, spec sheet (context only)
 
 
 def peaks():
@@ -58,13 +67,18 @@ def fwd_bwd_flops(M, N, K, r):
     return 4 * M * N * K + 6 * M * r * (N + K)
 
 
-def workload_config(cfg, extra=None):
-    c = {"workload": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "r": cfg.r, "alpha": cfg.alpha,
-         "step": "quantize(W fp32) + dequantize(bf16) + forward + backward",
-         "l2": "inputs larger than L2: two alternating input sets, ~0.26 GB touched per step"}
-    if extra:
-        c.update(extra)
-    return c
+def step_flops(cfgs):
+    return sum(fwd_bwd_flops(c.M, c.N, c.K, c.r) for c in cfgs)
+
+
+def workload_config():
+    """The workload named identically by both arms."""
+    return {"workload": WORKLOAD,
+            "linears": [{"name": c.name, "N": c.N, "K": c.K} for c in HEADLINE],
+            "M": HEADLINE[0].M, "r": HEADLINE[0].r, "alpha": HEADLINE[0].alpha, "w_std": HEADLINE[0].w_std,
+            "step": "per linear: quantize(W fp32 -> NF4 + double quant) + forward + backward "
+                    "(no bf16 weight written)",
+            "l2": "inputs larger than L2: two alternating input sets, ~3.4 GB"}
 
 
 # ------------------------------------------------------------- clocks ------
@@ -100,7 +114,7 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
+        sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
@@ -109,6 +123,7 @@ class ClockSampler:
             try:
                 sm.append(float(parts[1]))
                 smax.append(float(parts[2]))
+                power.append(float(parts[3]))
             except ValueError:
                 continue
             for n, v in zip(names, parts[5:9]):
@@ -117,45 +132,45 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w_max": max(power) if power else None, "samples": len(sm)}
 
 
 # ------------------------------------------------------- CPU oracle leg ----
 
 class OracleSample:
-    """The CPU oracle on a proportional slice of the workload: m_s tokens
-    forward+backward in fp64 against the oracle's dequantised W, plus the
-    quantisation and dequantisation of m_s rows of W (the share of the
-    one-per-step weight work that m_s of the M tokens carry)."""
+    """The CPU oracle on a proportional slice of the workload: for each
+    linear, m_s tokens forward+backward in fp64 against the oracle's
+    dequantised W, plus the quantisation of m_s rows of W (the share of the
+    once-per-step weight work that m_s of the M tokens carry)."""
 
-    def __init__(self, cfg):
+    def __init__(self, cfgs):
         import oracle
         self.o = oracle
-        self.cfg = cfg
-        W = synth.weight(cfg).numpy()
-        z = oracle.quantize_nf4(W)
-        self.W = W
-        self.What = oracle.bf16_bits_to_f64(
-            oracle.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], cfg.N, cfg.K))
-        self.X = synth.activations(cfg).float().numpy().astype(np.float64)
-        self.dY = synth.grad_output(cfg).float().numpy().astype(np.float64)
-        self.A = synth.lora_a(cfg).float().numpy().astype(np.float64)
-        self.B = synth.lora_b(cfg).float().numpy().astype(np.float64)
+        self.cfgs = cfgs
+        self.layers = []
+        for cfg in cfgs:
+            W = synth.weight(cfg).numpy()
+            z = oracle.quantize_nf4(W)
+            What = oracle.bf16_bits_to_f64(
+                oracle.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], cfg.N, cfg.K))
+            f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+            self.layers.append(dict(cfg=cfg, W=W, What=What, X=f64(synth.activations(cfg)),
+                                    dY=f64(synth.grad_output(cfg)), A=f64(synth.lora_a(cfg)), B=f64(synth.lora_b(cfg))))
         self.threads = oracle.num_threads()
 
     def step(self, m_s: int, offset: int = 0):
-        c = self.cfg
-        lo = offset % (c.M - m_s + 1)
-        rows = slice(lo, lo + m_s)
-        wrows = slice(lo % (c.N - m_s + 1), lo % (c.N - m_s + 1) + m_s) if m_s <= c.N else slice(0, c.N)
-        z = self.o.quantize_nf4(self.W[wrows])
-        self.o.dequant_bf16_bits(z["codes"], z["qabsmax"], z["s2"], z["mean"], z["N"], z["K"])
-        X, dY = self.X[rows], self.dY[rows]
-        self.o.forward(X, self.What, self.A, self.B, c.alpha, c.r)
-        self.o.backward(dY, X, self.What, self.A, self.B, c.alpha, c.r)
+        for L in self.layers:
+            c = L["cfg"]
+            lo = offset % (c.M - m_s + 1)
+            rows = slice(lo, lo + m_s)
+            w0 = lo % (c.N - m_s + 1) if m_s <= c.N else 0
+            self.o.quantize_nf4(L["W"][w0:w0 + min(m_s, c.N)])
+            X, dY = L["X"][rows], L["dY"][rows]
+            self.o.forward(X, L["What"], L["A"], L["B"], c.alpha, c.r)
+            self.o.backward(dY, X, L["What"], L["A"], L["B"], c.alpha, c.r)
 
     def flops(self, m_s):
-        return fwd_bwd_flops(m_s, self.cfg.N, self.cfg.K, self.cfg.r)
+        return sum(fwd_bwd_flops(m_s, c.N, c.K, c.r) for c in self.cfgs)
 
     def calibrate(self, target_s: float) -> int:
         t0 = time.perf_counter()
@@ -163,9 +178,13 @@ class OracleSample:
         dt = max(time.perf_counter() - t0, 1e-4)
         m = int(16 * target_s / dt)
         m_s = 1
-        while m_s * 2 <= max(m, 1) and m_s * 2 <= self.cfg.M:
+        while m_s * 2 <= max(m, 1) and m_s * 2 <= min(c.M for c in self.cfgs):
             m_s *= 2
         return m_s
+
+    def describe(self, m_s):
+        return (f"{m_s} tokens of fwd+bwd per linear (fp64 numpy) + quantisation of {m_s} rows of each W "
+                f"(C oracle), on {self.threads} host threads")
 
     def sample_line(self, seconds: float = 10.0):
         m_s = self.calibrate(1.0)
@@ -179,8 +198,7 @@ class OracleSample:
                 break
         value = self.flops(m_s) * n / el / 1e12
         return {"value": value, "unit": "TFLOP/s", "cores": self.threads, "kind": "oracle",
-                "sample": f"{n} slices of {m_s} tokens fwd+bwd (fp64 numpy) + quantize/dequantize of {m_s} "
-                          f"rows of W (C oracle), {el:.1f} s on {self.threads} host threads"}
+                "sample": f"{n} slices of {self.describe(m_s)}, {el:.1f} s"}
 
 
 # ---------------------------------------------------------------- ranks ----
@@ -206,7 +224,7 @@ def job_tflops(flops_per_step_per_rank: float, world: int, ms_per_step: float) -
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    s = OracleSample(CFG)
+    s = OracleSample(HEADLINE)
     budget = 150.0 / max(args.steps + args.warmup, 1)  # whole run within ~2.5 minutes
     m_s = s.calibrate(budget)
     for i in range(args.warmup):
@@ -219,22 +237,19 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": workload_config(CFG, {"sample_tokens_per_step": m_s,
-                                            "reference": "CPU oracle (C + numpy fp64), no GPU"}),
+            "data": "synthetic", "config": workload_config(),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle",
-                             "sample": f"per step: {m_s} tokens fwd+bwd + quantize/dequantize of {m_s} rows of W"},
+                             "sample": "per step: " + s.describe(m_s)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ ours ---
 
-# DRAM bytes (read + write) of one launch of the dominant kernel, from one
-# ncu capture of the current kernel on this workload (attn7B forward:
-# 43.35 MB read, 3.06 MB written; most of Y is still in L2 when the kernel
-# ends). Kernels without a capture of their current version report null.
-NCU_TRAFFIC = {"fused_forward": 46.41e6}
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu
+# capture of its current build on this workload (per kernel key). A kernel
+# without a capture of its current version reports null.
+NCU_TRAFFIC: dict = {}
 
 
 def timed(fn, n=20):
@@ -256,10 +271,100 @@ def timed(fn, n=20):
     return e0.elapsed_time(e1) / n
 
 
+def assert_device_ok(q, workspaces, where):
+    """Every bounded wait of the pipelined kernels ended in time: a wait that
+    ran out leaves its tile unwritten and sets the workspace status word."""
+    for ws in workspaces:
+        st = q.device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"{where}: device status {q.STATUS.get(st, st)}")
+
+
+class Linear:
+    """Device buffers of one linear of the workload: two input sets (W fp32,
+    X, A, B, dY), the packed weight, outputs and workspaces."""
+
+    def __init__(self, q, cfg, dev, sets=2, w_fp32=True):
+        self.q, self.cfg = q, cfg
+        c = cfg
+        host = []
+        for s in range(sets):
+            cs = c if s == 0 else synth.custom(N=c.N, K=c.K, M=c.M, r=c.r, alpha=c.alpha,
+                                               seed_base=77 + 10 * c.layer_id + s, w_std=c.w_std,
+                                               outliers=c.outliers)
+            h = dict(X=synth.activations(cs), A=synth.lora_a(cs), B=synth.lora_b(cs), dY=synth.grad_output(cs))
+            if w_fp32:
+                h["W"] = synth.weight(cs)
+            host.append(h)
+        self.host = host
+        self.sets = [{k: v.to(dev) for k, v in h.items()} for h in host]
+        M, N, K, r = c.M, c.N, c.K, c.r
+        self.w = q.NF4Weight.empty(N, K, dev)
+        if not w_fp32:
+            q.quantize_nf4(synth.weight(c).to(dev), out=self.w)
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+        self.dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+        self.ws_q = torch.empty(q.workspace_bytes(q.OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
+        # zeroed, so the status word reads clean before the first call too
+        self.ws_f = torch.zeros(q.workspace_bytes(q.OP_FWD, M, N, K, r), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.zeros(q.workspace_bytes(q.OP_BWD, M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def quantize(self, i):
+        self.q.quantize_nf4(self.sets[i % len(self.sets)]["W"], out=self.w, ws=self.ws_q)
+
+    def fwd(self, i, prof=None):
+        s = self.sets[i % len(self.sets)]
+        if prof is not None:
+            self.q.profile_next_launch(self.q.KERNEL_FUSED_FWD, *prof)
+        self.q.linear_fwd(s["X"], self.w, s["A"], s["B"], self.cfg.alpha, Y=self.Y, sT=self.sT, ws=self.ws_f)
+
+    def bwd(self, i, prof=None):
+        s = self.sets[i % len(self.sets)]
+        if prof is not None:
+            self.q.profile_next_launch(self.q.KERNEL_FUSED_DX, *prof)
+        self.q.linear_bwd(s["dY"], s["X"], self.w, s["A"], s["B"], self.cfg.alpha, sT=self.sT, dX=self.dX,
+                          dA=self.dA, dB=self.dB, ws=self.ws_b)
+
+    def step(self, i, prof=None):
+        self.quantize(i)
+        self.fwd(i, None if prof is None else prof[0])
+        self.bwd(i, None if prof is None else prof[1])
+
+    def workspaces(self):
+        return [self.ws_f, self.ws_b]
+
+    def fused_flops(self):
+        c = self.cfg
+        return {"fwd": 2 * c.M * c.N * (c.K + c.r), "dx": 2 * c.M * c.K * (c.N + c.r)}
+
+
+def fwd_bwd_rows(q, dev):
+    """fwd+bwd of every other configuration's linears (weights quantised
+    once, graph-timed): TFLOP/s and tokens/s per linear."""
+    pk = peaks()[0]
+    out = {}
+    for cfg in [synth.TINY, synth.ATTN7B, *synth.MLP7B, synth.L65B[0]]:
+        L = Linear(q, cfg, dev, sets=2, w_fp32=False)
+        t = timed(lambda i: (L.fwd(i), L.bwd(i)), n=20)
+        tf = timed(lambda i: L.fwd(i), n=20)
+        assert_device_ok(q, L.workspaces(), cfg.name)
+        fl = fwd_bwd_flops(cfg.M, cfg.N, cfg.K, cfg.r)
+        out[cfg.name] = {"fwd_bwd_us": t * 1e3, "fwd_us": tf * 1e3, "TFLOPs": fl / (t * 1e-3) / 1e12,
+                         "tokens_per_s": cfg.M / (t * 1e-3),
+                         "frac_bf16_burst": fl / (t * 1e-3) / 1e12 / pk.get("bf16_tflops", 1590.0)}
+        del L
+        torch.cuda.empty_cache()
+    return out
+
+
 def other_rows(q, dev):
     """The other rows of the path on their own workloads (graph-timed): the
-    quantiser and dequantiser on the large weights and the small-batch
-    forward sweep, each streaming from HBM (rotated weight copies)."""
+    quantiser and dequantiser on the large weights, the adapter merge and
+    the small-batch forward sweep, each streaming from HBM (rotated weight
+    copies)."""
     sweep = {}
     pk_hbm = peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -327,6 +432,7 @@ def other_rows(q, dev):
             q.profile_next_launch(q.KERNEL_FUSED_FWD, e[0], e[1])
             q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc)
         torch.cuda.synchronize()
+        assert_device_ok(q, [wsc], c.name)
         tk = statistics.median(e[0].elapsed_time(e[1]) for e in evs[3:])
         gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
         wb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384)
@@ -354,43 +460,18 @@ def run_ours(args, rank, world, local_rank):
         if pg is not None:
             pg.barrier()
 
-    cfg = CFG
-    M, N, K, r, alpha = cfg.M, cfg.N, cfg.K, cfg.r, cfg.alpha
-    host = [dict(W=synth.weight(cfg), X=synth.activations(cfg), A=synth.lora_a(cfg), B=synth.lora_b(cfg),
-                 dY=synth.grad_output(cfg))]
-    # second input set: the same distributions, other seeds
-    cfg2 = synth.custom(N=N, K=K, M=M, r=r, alpha=alpha, seed_base=77, outliers=True)
-    host.append(dict(W=synth.weight(cfg2), X=synth.activations(cfg2), A=synth.lora_a(cfg2),
-                     B=synth.lora_b(cfg2), dY=synth.grad_output(cfg2)))
-    sets = [{k: v.to(dev) for k, v in h.items()} for h in host]
-
-    w = q.NF4Weight.empty(N, K, dev)
-    Wbf = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    sT = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
-    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
-    ws_q = torch.empty(q.workspace_bytes(q.OP_QUANTIZE, 0, N, K, 0), dtype=torch.uint8, device=dev)
-    ws_f = torch.empty(q.workspace_bytes(q.OP_FWD, M, N, K, r), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(q.workspace_bytes(q.OP_BWD, M, N, K, r), dtype=torch.uint8, device=dev)
+    layers = [Linear(q, c, dev) for c in HEADLINE]
 
     def step(i, prof=None):
-        s = sets[i % 2]
-        q.quantize_nf4(s["W"], out=w, ws=ws_q)
-        q.dequantize_nf4(w, out=Wbf)
-        if prof is not None:
-            q.profile_next_launch(q.KERNEL_FUSED_FWD, *prof[0])
-            q.profile_next_launch(q.KERNEL_FUSED_DX, *prof[1])
-        q.linear_fwd(s["X"], w, s["A"], s["B"], alpha, Y=Y, sT=sT, ws=ws_f)
-        q.linear_bwd(s["dY"], s["X"], w, s["A"], s["B"], alpha, sT=sT, dX=dX, dA=dA, dB=dB, ws=ws_b)
+        for j, L in enumerate(layers):
+            L.step(i, None if prof is None else prof[j])
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
 
     # ---- eager timing (host launches every kernel): reported for reference
-    n_eager = min(args.steps, 200)
+    n_eager = min(args.steps, 50)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     h0 = time.perf_counter()
@@ -403,13 +484,15 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- timed region: the K steps, every kernel of every step, replayed from
     # one captured CUDA graph (no host launch gaps); each step records its own
-    # events around the two fused matmuls
-    prof = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
-            for _ in range(args.steps)]
-    for pair in prof:  # torch creates events lazily: make them exist before the library records them
-        for a, b in pair:
-            a.record()
-            b.record()
+    # events around the four fused matmuls (forward and dX of each linear)
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+    prof = [[[(ev(), ev()) for _ in range(2)] for _ in layers] for _ in range(args.steps)]
+    for per_step in prof:  # torch creates events lazily: make them exist before the library records them
+        for per_layer in per_step:
+            for a, b in per_layer:
+                a.record()
+                b.record()
     torch.cuda.synchronize()
     launches0 = q.launch_count()
     graph = torch.cuda.CUDAGraph()
@@ -431,93 +514,155 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop()
     ms = max_over_ranks(start.elapsed_time(stop) / args.steps, pg, dev)
-    fwd_ms = statistics.mean(p[0][0].elapsed_time(p[0][1]) for p in prof)
-    dx_ms = statistics.mean(p[1][0].elapsed_time(p[1][1]) for p in prof)
+    for L in layers:
+        assert_device_ok(q, L.workspaces(), "timed step")
+    # per launch: (name, ms, flops) of the four fused matmuls of every step
+    fused = []
+    for per_step in prof:
+        for j, L in enumerate(layers):
+            fl = L.fused_flops()
+            fused.append((f"fwd_{L.cfg.name}", per_step[j][0][0].elapsed_time(per_step[j][0][1]), fl["fwd"]))
+            fused.append((f"dx_{L.cfg.name}", per_step[j][1][0].elapsed_time(per_step[j][1][1]), fl["dx"]))
     del graph
 
-    # ---- per-row breakdown (outside the timed region, same inputs): each row
-    # is captured n times into a CUDA graph and the replay is timed, so the
-    # numbers are GPU time without host launch gaps
-    rows_ms = {
-        "quantize": timed(lambda i: q.quantize_nf4(sets[i % 2]["W"], out=w, ws=ws_q)),
-        "dequantize": timed(lambda i: q.dequantize_nf4(w, out=Wbf)),
-        "forward": timed(lambda i: q.linear_fwd(sets[i % 2]["X"], w, sets[i % 2]["A"], sets[i % 2]["B"], alpha,
-                                                Y=Y, sT=sT, ws=ws_f)),
-        "backward": timed(lambda i: q.linear_bwd(sets[i % 2]["dY"], sets[i % 2]["X"], w, sets[i % 2]["A"],
-                                                 sets[i % 2]["B"], alpha, sT=sT, dX=dX, dA=dA, dB=dB, ws=ws_b)),
-    }
+    # ---- per-row breakdown (outside the timed region, same inputs), each
+    # graph-timed
+    rows_ms = {}
+    for L in layers:
+        n = L.cfg.name
+        rows_ms[f"quantize_{n}"] = timed(L.quantize)
+        rows_ms[f"forward_{n}"] = timed(L.fwd)
+        rows_ms[f"backward_{n}"] = timed(L.bwd)
+    for L in layers:
+        assert_device_ok(q, L.workspaces(), "rows")
 
-    # ---- end to end through the public API with host buffers
-    pin = [{k: v.pin_memory() for k, v in h.items()} for h in host]
-    out_host = dict(Y=torch.empty_like(Y, device="cpu").pin_memory(), dX=torch.empty_like(dX, device="cpu").pin_memory(),
-                    dA=torch.empty_like(dA, device="cpu").pin_memory(), dB=torch.empty_like(dB, device="cpu").pin_memory(),
-                    Wbf=torch.empty_like(Wbf, device="cpu").pin_memory())
-    h2d = sum(v.numel() * v.element_size() for v in pin[0].values())
-    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    # ---- end to end through the public API with host buffers. Step i's
+    # inputs go host -> device on a copy stream, its compute runs on the main
+    # stream and its outputs go device -> host on a second copy stream, with
+    # inputs and outputs double-buffered: the copies of neighbouring steps
+    # overlap the compute, and every byte still crosses PCIe inside the timed
+    # region.
+    pins = [[{k: v.pin_memory() for k, v in h.items()} for h in L.host] for L in layers]
+    outs = [[dict(Y=L.Y, dX=L.dX, dA=L.dA, dB=L.dB),
+             dict(Y=torch.empty_like(L.Y), dX=torch.empty_like(L.dX), dA=torch.empty_like(L.dA),
+                  dB=torch.empty_like(L.dB))] for L in layers]
+    out_host = [[{k: torch.empty_like(v, device="cpu").pin_memory() for k, v in o.items()} for o in lo]
+                for lo in outs]
+    h2d = sum(v.numel() * v.element_size() for p in pins for v in p[0].values())
+    d2h = sum(v.numel() * v.element_size() for lo in out_host for v in lo[0].values())
+    main = torch.cuda.current_stream(dev)
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready, in_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
+    out_ready, out_free = [torch.cuda.Event() for _ in range(2)], [torch.cuda.Event() for _ in range(2)]
+    for j in range(2):  # every buffer starts free
+        in_free[j].record(main)
+        out_free[j].record(main)
 
     def e2e_step(i):
-        s, p = sets[i % 2], pin[i % 2]
-        for k in s:
-            s[k].copy_(p[k], non_blocking=True)
-        step(i)
-        out_host["Y"].copy_(Y, non_blocking=True)
-        out_host["dX"].copy_(dX, non_blocking=True)
-        out_host["dA"].copy_(dA, non_blocking=True)
-        out_host["dB"].copy_(dB, non_blocking=True)
-        out_host["Wbf"].copy_(Wbf, non_blocking=True)
+        j = i % 2
+        with torch.cuda.stream(h2d_s):
+            h2d_s.wait_event(in_free[j])  # the step two back has finished reading set j
+            for li, L in enumerate(layers):
+                for k, v in L.sets[j].items():
+                    v.copy_(pins[li][j][k], non_blocking=True)
+            in_ready[j].record(h2d_s)
+        main.wait_event(in_ready[j])
+        main.wait_event(out_free[j])  # the step two back has left output set j
+        for li, L in enumerate(layers):
+            o = outs[li][j]
+            s = L.sets[j]
+            q.quantize_nf4(s["W"], out=L.w, ws=L.ws_q)
+            q.linear_fwd(s["X"], L.w, s["A"], s["B"], L.cfg.alpha, Y=o["Y"], sT=L.sT, ws=L.ws_f)
+            q.linear_bwd(s["dY"], s["X"], L.w, s["A"], s["B"], L.cfg.alpha, sT=L.sT, dX=o["dX"], dA=o["dA"],
+                         dB=o["dB"], ws=L.ws_b)
+        in_free[j].record(main)
+        out_ready[j].record(main)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(out_ready[j])
+            for li in range(len(layers)):
+                for k, v in outs[li][j].items():
+                    out_host[li][j][k].copy_(v, non_blocking=True)
+            out_free[j].record(d2h_s)
 
-    e2e_steps = max(3, min(args.steps, 30))
+    e2e_steps = max(3, min(args.steps, 20))
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(main)
+    h2d_s.wait_event(e0)
+    d2h_s.wait_event(e0)
     for i in range(e2e_steps):
         e2e_step(i)
-    e1.record()
+    main.wait_stream(h2d_s)
+    main.wait_stream(d2h_s)
+    e1.record(main)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
+    for L in layers:
+        assert_device_ok(q, L.workspaces(), "end to end")
+    del pins, out_host, outs
 
-    # ---- the other rows of the path on their own workloads (graph-timed,
-    # outside the timed region): the small-batch sweep forward and the
-    # quantiser / dequantiser on the large weights
-    sweep = other_rows(q, dev) if (not args.no_sweep and rank == 0) else {}
+    # dequantise the headline weights (a3 standalone; not part of the step)
+    deq = {}
+    for L in layers:
+        Wbf = torch.empty(L.cfg.N, L.cfg.K, dtype=torch.bfloat16, device=dev)
+        t = timed(lambda i: q.dequantize_nf4(L.w, out=Wbf))
+        deq[L.cfg.name] = (L.cfg.N * L.cfg.K * (0.5 + 1 / 64 + 4 / 16384 + 2)) / (t * 1e-3) / 1e9
+        del Wbf
+    flops_step = step_flops(HEADLINE)
+    M = HEADLINE[0].M
+    del layers
+    torch.cuda.empty_cache()
 
-    flops = fwd_bwd_flops(M, N, K, r)
-    value = job_tflops(flops, world, ms)
+    # ---- the other configurations' fwd+bwd and the other rows of the path
+    # on their own workloads (graph-timed, outside the timed region)
+    extra = {} if (args.no_sweep or rank != 0) else fwd_bwd_rows(q, dev)
+    sweep = {} if (args.no_sweep or rank != 0) else other_rows(q, dev)
+
+    value = job_tflops(flops_step, world, ms)
     pk, pk_kind = peaks()
-    # dominant kernel: the fused matmul with the larger time per step
-    kern = {"fused_forward": (fwd_ms, 2 * M * N * (K + r)), "fused_dx": (dx_ms, 2 * M * K * (N + r))}
-    dom = max(kern, key=lambda k: kern[k][0])
-    d_ms, d_flops = kern[dom]
-    achieved = d_flops / (d_ms * 1e-3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    deq_bytes = N * K * (0.5 + 1 / 64 + 4 / 16384 + 2)
+    # dominant kernel: the fused matmul (every launch of it in the timed
+    # region: forward and dX of both linears)
+    f_ms = statistics.mean(t for _, t, _ in fused)
+    f_flops = statistics.mean(f for _, _, f in fused)
+    achieved = f_flops / (f_ms * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    by_launch = {}
+    for name, t, f in fused:
+        by_launch.setdefault(name, []).append((t, f))
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(),
         "tokens_per_s": M * world / (ms * 1e-3),
-        "dequant_gbs": deq_bytes / (rows_ms["dequantize"] * 1e-3) / 1e9,
+        "dequant_gbs": statistics.mean(deq.values()),
+        "dequant_gbs_by_weight": deq,
         "rows_ms": rows_ms,
         "timing": "timed steps replayed from one CUDA graph holding all K steps",
         "eager_ms_per_step": eager_ms,
         "host_enqueue_ms_per_step": host_ms,
-        "kernels_ms": {"fused_forward": fwd_ms, "fused_dx": dx_ms},
-        "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": NCU_TRAFFIC.get(dom),
+        "fused_launches_us": {k: statistics.mean(t for t, _ in v) * 1e3 for k, v in by_launch.items()},
+        "roofline": {"kernel": "fused_nf4_gemm (forward and dX of both linears)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": NCU_TRAFFIC.get("fused_nf4_gemm"),
                      "traffic_source": "ncu capture of one launch: dram__bytes_read.sum + dram__bytes_write.sum"
-                     if dom in NCU_TRAFFIC else None,
-                     "peak_kind": f"bf16 sustained ({pk_kind})"},
-        "e2e": {"value": job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                     if "fused_nf4_gemm" in NCU_TRAFFIC else None,
+                     "peak_kind": f"bf16 burst ({pk_kind}; the timed graph lasts well under a second)",
+                     "frac_of_sustained": achieved / pk.get("bf16_tflops_sustained", 1400.0),
+                     "frac_of_datasheet_dense": achieved / DATASHEET_BF16_TFLOPS},
+        "e2e": {"value": job_tflops(flops_step, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "H2D of step i+1 and D2H of step i-1 on two copy streams beside step i's compute"},
         "gpu_launches": launches,
+        "device_status": "ok",
+        "fwd_bwd_rows": extra,
         "other_rows": sweep,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = OracleSample(cfg).sample_line(args.cpu_seconds)
+        line["cpu_baseline"] = OracleSample(HEADLINE).sample_line(args.cpu_seconds)
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
@@ -525,17 +670,61 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One call of the library repeated (for profiler captures): `step` is the
+    headline step; `fwd:<workload>` etc. one entry point on one named
+    workload (synth names), its weight quantised once beforehand."""
+    import bit_nf4_quantized_09_b200 as q
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.case == "step":
+        layers = [Linear(q, c, dev) for c in HEADLINE]
+        for i in range(args.reps):
+            for L in layers:
+                L.step(i)
+        torch.cuda.synchronize()
+        for L in layers:
+            assert_device_ok(q, L.workspaces(), "case step")
+        return
+    kind, _, name = args.case.partition(":")
+    cfg = synth.by_name(name)
+    L = Linear(q, cfg, dev, sets=1, w_fp32=kind == "quantize")
+    if kind == "quantize":
+        fn = L.quantize
+    elif kind == "fwd":
+        fn = L.fwd
+    elif kind == "bwd":
+        L.fwd(0)
+        fn = L.bwd
+    elif kind == "dequantize":
+        Wbf = torch.empty(cfg.N, cfg.K, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: q.dequantize_nf4(L.w, out=Wbf)  # noqa: E731
+    elif kind == "merge":
+        Wbf = torch.empty(cfg.N, cfg.K, dtype=torch.bfloat16, device=dev)
+        s = L.sets[0]
+        fn = lambda i: q.merge_lora(L.w, s["A"], s["B"], cfg.alpha, out=Wbf)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    for i in range(args.reps):
+        fn(i)
+    torch.cuda.synchronize()
+    assert_device_ok(q, L.workspaces(), f"case {args.case}")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--no-sweep", action="store_true", help="skip the small-batch / quantiser rows")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the other configurations' rows")
     ap.add_argument("--rows-only", action="store_true",
                     help="only the small-batch / quantiser rows (one JSON line with other_rows), for profiling")
+    ap.add_argument("--case", default=None, help="repeat one call for a profiler capture (see above)")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -544,11 +733,13 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.case:
+        run_case(args)
     elif args.rows_only:
         import bit_nf4_quantized_09_b200 as q
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
-        print(json.dumps({"other_rows": other_rows(q, dev)}), flush=True)
+        print(json.dumps({"fwd_bwd_rows": fwd_bwd_rows(q, dev), "other_rows": other_rows(q, dev)}), flush=True)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -59,6 +59,14 @@ _SIGNATURES = {
     "qlora_merge_lora": (_int, [_wp, _vp, _vp, _int, _f32, _vp, _vp]),
     "qlora_linear_fwd": (_int, [_vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_int, [_vp, _vp, _i64, _wp, _vp, _vp, _int, _f32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_workspace_bytes_multi": (_sz, [_int, _i64, _i64, _i64, _int, _int]),
+    "qlora_linear_fwd_multi": (_int, [_vp, _i64, _wp, _vp, _vp, _int, _int, _vp, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd_multi": (_int, [_vp, _vp, _i64, _wp, _vp, _vp, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp,
+                                      _vp, _sz, _vp]),
+    "qlora_workspace_bytes_group": (_sz, [_int, _i64, ctypes.POINTER(_i64), _int, _i64, _int]),
+    "qlora_linear_fwd_group": (_int, [_vp, _i64, _wp, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd_group": (_int, [_vp, _vp, _i64, _wp, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp, _vp, _vp,
+                                      _sz, _vp]),
     "qlora_nf4_tables": (_int, [ctypes.POINTER(_f32), ctypes.POINTER(_f32)]),
     "qlora_device_status": (_int, [_vp, ctypes.POINTER(_int), _vp]),
     "qlora_status_string": (ctypes.c_char_p, [_int]),
@@ -90,6 +98,26 @@ def _check(status: int, where: str):
     if status != QLORA_OK:
         detail = lib().qlora_last_error().decode(errors="replace")
         raise QLoraError(status, where, detail)
+
+
+_check_device_status = False
+
+
+def set_check_device_status(on: bool):
+    """When on, every forward/backward wrapper call reads its workspace's
+    device status word back (a synchronisation) and raises if a bounded wait
+    of a pipelined kernel ran out, so an unwritten tile cannot pass silently.
+    Off by default: the calls stay asynchronous."""
+    global _check_device_status
+    _check_device_status = bool(on)
+
+
+def _after_call(ws: torch.Tensor, where: str, M: int = 1):
+    # an empty batch launches nothing and leaves the workspace untouched
+    if _check_device_status and M > 0:
+        st = device_status(ws)
+        if st != QLORA_OK:
+            raise QLoraError(st, where, "device status after the call")
 
 
 try:
@@ -245,8 +273,12 @@ def quantize_nf4_noalloc(W: torch.Tensor, out: NF4Weight) -> NF4Weight:
     """Quantise without any workspace: for callers that cannot allocate device
     memory at call time. The library keeps its scratch in one static device
     array (N*K up to 67,108,864 weights); `out` must be allocated beforehand."""
-    assert W.dtype == torch.float32 and W.is_cuda and W.dim() == 2
+    assert W.dtype == torch.float32 and W.is_cuda and W.dim() == 2 and W.is_contiguous()
     N, K = W.shape
+    sz = nf4_bytes(N, K)
+    assert out.absmax is None and (out.N, out.K) == (N, K), "out must be an NF4Weight with double quantisation of W's shape"
+    assert out.codes.numel() >= sz["codes"] and out.qabsmax.numel() >= sz["qabsmax"], "out is too small"
+    assert out.s2.numel() * 4 >= sz["s2"] and out.mean.numel() >= 1, "out is too small"
     _check(lib().qlora_quantize_nf4_noalloc(_ptr(W), N, K, _ptr(out.codes), _ptr(out.qabsmax), _ptr(out.s2),
                                             _ptr(out.mean), _stream(W.device)), "qlora_quantize_nf4_noalloc")
     return out
@@ -274,6 +306,7 @@ def linear_fwd(X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, 
     _check(lib().qlora_linear_fwd(_ptr(X), M, ctypes.byref(v), _ptr(A), _ptr(B), r, float(alpha), _ptr(Y),
                                   _ptr(sT) if save_sT else None, _ptr(ws), ws.numel(), _stream(dev)),
            "qlora_linear_fwd")
+    _after_call(ws, "qlora_linear_fwd", M)
     return Y, (sT if save_sT else None)
 
 
@@ -292,6 +325,135 @@ def linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.Tensor,
     _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(v), _ptr(A), _ptr(B), r, float(alpha),
                                   _ptr(sT), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(dev)),
            "qlora_linear_bwd")
+    _after_call(ws, "qlora_linear_bwd", M)
+    return dX, dA, dB
+
+
+# ------------------------------------------ several adapters over one base ---
+
+def workspace_bytes_multi(op: int, M: int, N: int, K: int, r: int, P: int) -> int:
+    return int(lib().qlora_workspace_bytes_multi(op, M, N, K, r, P))
+
+
+def linear_fwd_multi(X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, ids: torch.Tensor, P: int,
+                     alpha: float, Y: torch.Tensor | None = None, sT: torch.Tensor | None = None,
+                     save_sT: bool = True, ws: torch.Tensor | None = None):
+    """(Y, sT) of a batch whose token row m uses adapter ids[m] (int32; an id
+    outside [0, P) uses none). A: bf16 [P r, K] (the A_k stacked); B: bf16
+    [N, P r] (the B_k side by side); sT: bf16 [M, P r], zero outside the
+    row's own adapter."""
+    M, K = X.shape
+    R = A.shape[0]
+    r = R // P
+    assert ids.dtype == torch.int32 and ids.numel() == M and B.shape == (w.N, R)
+    dev = X.device
+    Y = Y if Y is not None else torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+    if save_sT and sT is None:
+        sT = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+    ws = _ws(workspace_bytes_multi(OP_FWD, M, w.N, w.K, r, P), dev, ws)
+    v = w.c_view()
+    _check(lib().qlora_linear_fwd_multi(_ptr(X), M, ctypes.byref(v), _ptr(A), _ptr(B), r, P, _ptr(ids),
+                                        float(alpha), _ptr(Y), _ptr(sT) if save_sT else None, _ptr(ws), ws.numel(),
+                                        _stream(dev)), "qlora_linear_fwd_multi")
+    _after_call(ws, "qlora_linear_fwd_multi", M)
+    return Y, (sT if save_sT else None)
+
+
+def linear_bwd_multi(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                     ids: torch.Tensor, P: int, alpha: float, sT: torch.Tensor | None = None,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                     dB: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """(dX, dA fp32 [P r, K], dB fp32 [N, P r]) of linear_fwd_multi: every
+    adapter's gradients from the rows that use it."""
+    M, K = X.shape
+    R = A.shape[0]
+    r = R // P
+    dev = X.device
+    dX = dX if dX is not None else torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty(R, K, dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty(w.N, R, dtype=torch.float32, device=dev)
+    ws = _ws(workspace_bytes_multi(OP_BWD, M, w.N, w.K, r, P), dev, ws)
+    v = w.c_view()
+    _check(lib().qlora_linear_bwd_multi(_ptr(dY), _ptr(X), M, ctypes.byref(v), _ptr(A), _ptr(B), r, P, _ptr(ids),
+                                        float(alpha), _ptr(sT), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                                        _stream(dev)), "qlora_linear_bwd_multi")
+    _after_call(ws, "qlora_linear_bwd_multi", M)
+    return dX, dA, dB
+
+
+# ------------------------------------------ projections sharing one input ---
+
+def empty_group(Ns, K: int, device) -> list:
+    """Buffers for the NF4 weights of a group (N_i x K each, double
+    quantisation): one codes allocation sliced back to back, as the group
+    calls require; each weight is quantised into its own view."""
+    szs = [nf4_bytes(n, K) for n in Ns]
+    codes = torch.empty(sum(s["codes"] for s in szs), dtype=torch.uint8, device=device)
+    out, at = [], 0
+    for n, sz in zip(Ns, szs):
+        out.append(NF4Weight(codes[at:at + sz["codes"]], torch.empty(sz["qabsmax"], dtype=torch.uint8, device=device),
+                             torch.empty(sz["s2"] // 4, dtype=torch.float32, device=device),
+                             torch.empty(1, dtype=torch.float32, device=device), n, K))
+        at += sz["codes"]
+    return out
+
+
+def _group_view(ws_: list):
+    arr = (Nf4WeightC * len(ws_))()
+    for i, w in enumerate(ws_):
+        arr[i] = w.c_view()
+    return arr
+
+
+def workspace_bytes_group(op: int, M: int, Ns, K: int, r: int) -> int:
+    n = (_i64 * len(Ns))(*Ns)
+    return int(lib().qlora_workspace_bytes_group(op, M, n, len(Ns), K, r))
+
+
+def linear_fwd_group(X: torch.Tensor, group: list, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     Y: torch.Tensor | None = None, sT: torch.Tensor | None = None, save_sT: bool = True,
+                     ws: torch.Tensor | None = None):
+    """(Y, sT) of projections sharing X: Y = [Y_0 | Y_1 | ...] bf16 [M, sum N_i].
+    A: bf16 [P r, K] (the A_i stacked); B: bf16 [sum N_i, r] (the B_i stacked);
+    sT: bf16 [M, P r]."""
+    M, K = X.shape
+    P = len(group)
+    R = A.shape[0]
+    r = R // P
+    Ns = [w.N for w in group]
+    Nt = sum(Ns)
+    dev = X.device
+    Y = Y if Y is not None else torch.empty(M, Nt, dtype=torch.bfloat16, device=dev)
+    if save_sT and sT is None:
+        sT = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+    ws = _ws(workspace_bytes_group(OP_FWD, M, Ns, K, r), dev, ws)
+    arr = _group_view(group)
+    _check(lib().qlora_linear_fwd_group(_ptr(X), M, arr, P, _ptr(A), _ptr(B), r, float(alpha), _ptr(Y),
+                                        _ptr(sT) if save_sT else None, _ptr(ws), ws.numel(), _stream(dev)),
+           "qlora_linear_fwd_group")
+    _after_call(ws, "qlora_linear_fwd_group", M)
+    return Y, (sT if save_sT else None)
+
+
+def linear_bwd_group(dY: torch.Tensor, X: torch.Tensor, group: list, A: torch.Tensor, B: torch.Tensor,
+                     alpha: float, sT: torch.Tensor | None = None, dX: torch.Tensor | None = None,
+                     dA: torch.Tensor | None = None, dB: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """(dX, dA fp32 [P r, K], dB fp32 [sum N_i, r]) of linear_fwd_group."""
+    M, K = X.shape
+    P = len(group)
+    R = A.shape[0]
+    r = R // P
+    Ns = [w.N for w in group]
+    dev = X.device
+    dX = dX if dX is not None else torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty(R, K, dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty(sum(Ns), r, dtype=torch.float32, device=dev)
+    ws = _ws(workspace_bytes_group(OP_BWD, M, Ns, K, r), dev, ws)
+    arr = _group_view(group)
+    _check(lib().qlora_linear_bwd_group(_ptr(dY), _ptr(X), M, arr, P, _ptr(A), _ptr(B), r, float(alpha), _ptr(sT),
+                                        _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(dev)),
+           "qlora_linear_bwd_group")
+    _after_call(ws, "qlora_linear_bwd_group", M)
     return dX, dA, dB
 
 

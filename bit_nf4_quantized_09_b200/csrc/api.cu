@@ -234,7 +234,6 @@ inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
-int rank_pad(int r) { return r < 16 ? 16 : r; }
 
 // Reduction splits of a skinny matmul: enough CTAs for two per SM of a
 // 148-SM B200 (fixed so workspace sizes do not depend on the device).
@@ -275,15 +274,49 @@ Split gemv_split(int64_t M, int64_t N, int64_t K) {
     return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
 }
 
+// ------------------------------------------------------- the low-rank side --
+// The adapter side of a forward or backward call. One adapter (P = 1);
+// several adapters over one frozen base, each token row using the one its id
+// names (ids set; rank R = P r, adapter k in columns [k r, (k + 1) r) of the
+// rank-r inputs); or the projections of a group, which share the input and
+// sit side by side in the output (group set; projection i in columns
+// [i r, (i + 1) r)).
+struct Lora {
+    int r = 0;
+    int P = 1;
+    bool group = false;
+    const int* ids = nullptr;
+    int R() const { return r * P; }
+    // 64-column chunks of the concatenated rank-r inputs
+    int chunks() const { return static_cast<int>((R() + 63) / 64); }
+    // problems of the backward down-projection (a group: one per projection)
+    int down_bwd() const { return group ? P : chunks(); }
+    // problems of dB (a group: one per projection)
+    int grad_b() const { return group ? P : chunks(); }
+};
+
+constexpr int kMaxMultiRank = 256;  // P r of several adapters: four 64-column chunks
+
+// A weight, or the weights of a group read as one weight of sum(N_i) rows,
+// whose codes lie back to back in one buffer.
+struct Weights {
+    const qlora_nf4_weight* w = nullptr;
+    int P = 1;
+    int64_t N = 0, K = 0;
+    int64_t off[kMaxGroups + 1] = {};  // first row of each weight; off[P] = N
+    int64_t rows(int i) const { return off[i + 1] - off[i]; }
+};
+
 // ------------------------------------------------------- workspace layout --
 // Head of every fwd/bwd workspace: the device status word, then the split
-// tickets of the skinny matmuls; cleared by one memset at the start of each
-// call (the kernels also leave their tickets at zero).
+// tickets of the skinny matmuls and the stream-K flags of the fused ones;
+// cleared by one memset at the start of each call (the kernels also leave
+// their tickets at zero).
 struct Layout {
     size_t header = 0;                                   // bytes cleared per call
     size_t status = 0, ctrT = 0, ctrU = 0, ctrA = 0, ctrB = 0, ctrY = 0, flags = 0;
     size_t skpart = 0;                                    // fused matmul: partial tiles of stream-K contributors
-    size_t cT = 0, partT = 0, sT = 0, partY = 0;          // forward
+    size_t cT = 0, cflat = 0, partT = 0, sT = 0, partY = 0;  // forward
     size_t partU = 0, sU = 0, partA = 0;                  // backward (partA holds dA and dB partials)
     size_t total = 0;
     int64_t ldc = 0;
@@ -291,18 +324,33 @@ struct Layout {
     GemvMmaPlan reg_gemv{1, 1, 4, 1};
 };
 
-Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
+// UMMA N of a rank-r problem of `w` columns (at most 64).
+int rank_pad(int w) { return w <= 16 ? 16 : (w <= 32 ? 32 : 64); }
+
+// Column tiles of the fused forward: 256-column tiles per weight of a group.
+int64_t fwd_tiles_n(const Weights& W, bool group) {
+    if (!group) return cdiv(W.N, 256);
+    int64_t t = 0;
+    for (int i = 0; i < W.P; ++i) t += cdiv(W.rows(i), 256);
+    return t;
+}
+
+Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
     Layout L;
-    const int NR = rank_pad(r);
+    const int64_t N = W.N, K = W.K;
+    const int R = lo.R();
+    const int NRc = rank_pad(std::min(R, 64));            // chunked rank problems
+    const int NRu = lo.group ? rank_pad(lo.r) : NRc;      // backward down-projection
+    const int nch = lo.chunks(), ndu = lo.down_bwd(), ndb = lo.grad_b();
     L.ldc = (N + 3) / 4 * 4;  // constants row pitch: a multiple of 16 bytes
     const int64_t mtiles = std::max<int64_t>(1, cdiv(M, 128));
     const int64_t ktiles = cdiv(K, 128), ntiles = cdiv(N, 128);
     L.status = 0;
     L.ctrT = 256;
-    L.ctrU = L.ctrT + 4 * static_cast<size_t>(mtiles);
-    L.ctrA = L.ctrU + 4 * static_cast<size_t>(mtiles);
-    L.ctrB = L.ctrA + 4 * static_cast<size_t>(ktiles);
-    L.ctrY = L.ctrB + 4 * static_cast<size_t>(ntiles);
+    L.ctrU = L.ctrT + 4 * static_cast<size_t>(nch * mtiles);
+    L.ctrA = L.ctrU + 4 * static_cast<size_t>(ndu * mtiles);
+    L.ctrB = L.ctrA + 4 * static_cast<size_t>(nch * ktiles);
+    L.ctrY = L.ctrB + 4 * static_cast<size_t>(ndb * ntiles);
     L.flags = L.ctrY + 4 * static_cast<size_t>(ntiles);
     L.header = up256(L.flags + 4 * static_cast<size_t>(kPlanSms));
     size_t off = L.header;
@@ -313,13 +361,15 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
     };
     L.cT = take(static_cast<size_t>(K / kBlock) * L.ldc * 4);
     // the fused matmul's partial tiles, one per CTA, when it splits tiles
-    L.skpart = take(static_cast<size_t>(fused_partial_ctas(M, op == QLORA_OP_FWD ? N : K, op == QLORA_OP_FWD ? K : N,
-                                                           kPlanSms)) *
+    const bool fwd = op == QLORA_OP_FWD;
+    L.skpart = take(static_cast<size_t>(fused_partial_ctas(M, fwd ? fwd_tiles_n(W, lo.group) : cdiv(K, 256),
+                                                           fwd ? K : N, kPlanSms)) *
                     kFusedBM * kFusedBN * 4);
-    L.sT_split = split_for(mtiles, K);
-    L.sT = take(static_cast<size_t>(M) * r * 2);
-    if (op == QLORA_OP_FWD) {
-        L.partT = take(static_cast<size_t>(L.sT_split.splits) * M * NR * 4);
+    L.sT_split = split_for(mtiles * nch, K);
+    L.sT = take(static_cast<size_t>(M) * R * 2);
+    const size_t partT_bytes = static_cast<size_t>(nch) * L.sT_split.splits * M * NRc * 4;
+    if (fwd) {
+        L.partT = take(partT_bytes);
         if (M <= kGemvMaxM) {
             // either small-batch kernel may run (the choice is a runtime option)
             L.gemv = gemv_split(M, N, K);
@@ -329,15 +379,23 @@ Layout layout_for(int op, int64_t M, int64_t N, int64_t K, int r) {
                 part = std::max(part, static_cast<size_t>(L.reg_gemv.max_parts) * M * N * 4);
             }
             L.partY = take(part);
+            // a group's block constants decoded in block order for the
+            // register-fed kernel (its weights keep their own mean and s2)
+            if (lo.group) L.cflat = take(static_cast<size_t>(N * K / kBlock) * 4);
         }
     } else {
-        L.sU_split = split_for(mtiles, N);
-        L.grad_split = split_for(ktiles + ntiles, M);
-        const int64_t part_down = std::max(L.sU_split.splits, L.sT_split.splits);
-        L.partU = take(static_cast<size_t>(part_down) * M * NR * 4);
+        int64_t red_max = N;
+        if (lo.group) {
+            red_max = 0;
+            for (int i = 0; i < W.P; ++i) red_max = std::max(red_max, W.rows(i));
+        }
+        L.sU_split = split_for(mtiles * ndu, red_max);
+        L.grad_split = split_for(nch * ktiles + ndb * ntiles, M);
+        L.partU = take(std::max(static_cast<size_t>(ndu) * L.sU_split.splits * M * NRu * 4, partT_bytes));
         L.partT = L.partU;
-        L.sU = take(static_cast<size_t>(M) * r * 2);
-        L.partA = take(static_cast<size_t>(L.grad_split.splits) * (K + N) * NR * 4);
+        L.sU = take(static_cast<size_t>(M) * R * 2);
+        const int64_t b_rows = lo.group ? N : ndb * N;
+        L.partA = take(static_cast<size_t>(L.grad_split.splits) * (nch * K + b_rows) * NRc * 4);
     }
     L.total = off;
     return L;
@@ -366,6 +424,32 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
     return QLORA_OK;
 }
 
+// The weights of a call: one, or the P weights of a group, which must share
+// K and the storage form and keep their codes back to back in one buffer.
+qlora_status check_weights(const qlora_nf4_weight* w, int P, Weights* out) {
+    if (!w || P < 1 || P > kMaxGroups) return QLORA_ERR_INVALID_ARG;
+    out->w = w;
+    out->P = P;
+    out->K = w[0].K;
+    out->off[0] = 0;
+    for (int i = 0; i < P; ++i) {
+        const qlora_status s = check_weight(w + i);
+        if (s != QLORA_OK) return s;
+        if (w[i].K != out->K) return QLORA_ERR_BAD_SHAPE;
+        if ((w[i].absmax == nullptr) != (w[0].absmax == nullptr)) {
+            g_last_error = "the weights of a group must all use the same storage (with or without double quantisation)";
+            return QLORA_ERR_INVALID_ARG;
+        }
+        if (i > 0 && w[i].codes != w[i - 1].codes + w[i - 1].N * w[i - 1].K / 2) {
+            g_last_error = "the codes of the weights of a group must lie back to back in one buffer";
+            return QLORA_ERR_INVALID_ARG;
+        }
+        out->off[i + 1] = out->off[i] + w[i].N;
+    }
+    out->N = out->off[P];
+    return QLORA_OK;
+}
+
 BlockConstants constants_of(const qlora_nf4_weight* w) {
     if (w->absmax) return BlockConstants{nullptr, nullptr, nullptr, w->absmax};
     return BlockConstants{w->qabsmax, w->s2, w->mean, nullptr};
@@ -377,11 +461,13 @@ CUtensorMapSwizzle swizzle_for_rank(int NR) {
     return NR == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : (NR == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Map of a row-major [rows, r] bf16 matrix read as an MN-major [64, NR] tile
-// per 64 rows (B, sU, sT).
-qlora_status make_rank_map(CUtensorMap* m, const uint16_t* base, int64_t rows, int r, const char* what) {
-    const int NR = rank_pad(r);
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, r, rows, static_cast<uint64_t>(r) * 2, NR, 64,
+// Map of `cols` columns of a row-major bf16 matrix of `rows` rows and row
+// pitch `ld` elements, starting at `base`, read as MN-major [64 rows, NR
+// columns] tiles (B, sU, sT and their chunks); columns past `cols` read as
+// zeros.
+qlora_status make_rank_map(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols, int64_t ld, int NR,
+                           const char* what) {
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, static_cast<uint64_t>(ld) * 2, NR, 64,
                     swizzle_for_rank(NR), what);
 }
 
@@ -394,43 +480,438 @@ Split capped(const Split& sp, int64_t red) {
     return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
 }
 
-// out = bf16(scale * act[M, red] . W_r^T) as [M, r]. W_r is the rank-r
-// operand: A [r, red] read K-major, or (w_is_red_major) B [red, r] read
-// MN-major.
-qlora_status lora_down(const uint16_t* act, int64_t M, int64_t red, const uint16_t* wr, bool w_is_red_major, int r,
-                       float scale, const Split& sp_layout, float* part, int* counter, uint16_t* out, int* status,
-                       cudaStream_t st) {
-    const int NR = rank_pad(r);
-    const Split sp = capped(sp_layout, red);
-    CUtensorMap ta, tb;
-    QLORA_MAP(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, red, M, red * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "act");
-    if (w_is_red_major) {
-        qlora_status s = make_rank_map(&tb, wr, red, r, "B");
-        if (s != QLORA_OK) return s;
-    } else {
-        QLORA_MAP(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wr, red, r, red * 2, 64, NR, CU_TENSOR_MAP_SWIZZLE_128B, "A");
-    }
+// A split of a shorter reduction within the layout's partial buffers: at
+// most the layout's number of splits.
+Split split_within(const Split& sp, int64_t red) {
+    const Split c = capped(sp, red);
+    const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
+    const int64_t steps = cdiv(KT, c.splits);
+    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
+}
+
+SkinnyProblem skinny_problem(int64_t rows, int64_t red, const Split& sp, int a_mn, int b_mn, int mode, int ncols,
+                             int64_t out_ld, float* part, int* counter) {
+    SkinnyProblem p{};
+    p.rows = rows;
+    p.red = red;
+    p.splits = sp.splits;
+    p.steps_per_split = sp.steps;
+    p.a_mn_major = a_mn;
+    p.b_mn_major = b_mn;
+    p.mode = mode;
+    p.ncols = ncols;
+    p.out_ld = out_ld;
+    p.scale = 1.0f;
+    p.part = part;
+    p.counter = counter;
+    return p;
+}
+
+// sT = bf16(s X A^T) [M, R] in 64-column chunks (one skinny problem each);
+// with row ids, the columns of every adapter but the row's own are zero.
+qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A, const Lora& lo, float scale,
+                      const Split& sp_layout, float* part, int* ctr, uint16_t* sT, int* status, cudaStream_t st) {
+    const int R = lo.R(), nch = lo.chunks(), NR = rank_pad(std::min(R, 64));
+    const Split sp = capped(sp_layout, K);
+    const int64_t mtiles = cdiv(M, 128);
+    SkinnyMaps maps;
     SkinnyArgs a{};
     a.NR = NR;
-    a.r = r;
-    SkinnyProblem& P = a.p[0];
-    P.rows = M;
-    P.red = red;
-    P.splits = sp.splits;
-    P.steps_per_split = sp.steps;
-    P.a_mn_major = 0;
-    P.b_mn_major = w_is_red_major ? 1 : 0;
-    P.mode = kSkinnyOutBf16;
-    P.scale = scale;
-    P.part = part;
-    P.counter = counter;
-    P.out_bf16 = out;
-    a.p[1] = P;
+    CUtensorMap tx;
+    QLORA_MAP(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "X");
+    for (int c = 0; c < nch; ++c) {
+        const int w = std::min(64, R - 64 * c);
+        maps.a[c] = tx;
+        QLORA_MAP(&maps.b[c], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A + static_cast<int64_t>(64 * c) * K, K, w, K * 2, 64,
+                  NR, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+        SkinnyProblem& p = a.p[c];
+        p = skinny_problem(M, K, sp, 0, 0, kSkinnyOutBf16, w, R,
+                           part + static_cast<int64_t>(c) * sp_layout.splits * M * NR, ctr + c * mtiles);
+        p.scale = scale;
+        p.out_bf16 = sT + 64 * c;
+        p.row_ids = lo.ids;
+        p.ids_col0 = 64 * c;
+        p.ids_r = lo.r;
+    }
     a.status = status;
     a.timeout_ns = timeout_ns();
     if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_skinny(ta, tb, ta, tb, a, 1, st), 1, "skinny(lora down)");
+    QLORA_LAUNCH(launch_skinny(maps, a, nch, st), 1, "skinny(sT)");
     return QLORA_OK;
+}
+
+// sU = bf16(s dY B) [M, R]: 64-column chunks of B [N, R] (row ids mask as
+// above), or for a group one problem per projection, sU_i = s dY_i B_i with
+// dY_i the projection's columns of dY and B_i its rows of B [N, r].
+qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uint16_t* B, const Lora& lo, float scale,
+                      const Split& sp_layout, float* part, int* ctr, uint16_t* sU, int* status, cudaStream_t st) {
+    const int R = lo.R(), np = lo.down_bwd();
+    const int NR = lo.group ? rank_pad(lo.r) : rank_pad(std::min(R, 64));
+    const int64_t N = W.N, mtiles = cdiv(M, 128);
+    SkinnyMaps maps;
+    SkinnyArgs a{};
+    a.NR = NR;
+    int64_t poff = 0;
+    for (int c = 0; c < np; ++c) {
+        const int64_t n0 = lo.group ? W.off[c] : 0, red = lo.group ? W.rows(c) : N;
+        const int w = lo.group ? lo.r : std::min(64, R - 64 * c);
+        QLORA_MAP(&maps.a[c], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY + n0, red, M, N * 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "dY");
+        qlora_status s = lo.group ? make_rank_map(&maps.b[c], B + n0 * lo.r, red, lo.r, lo.r, NR, "B")
+                                  : make_rank_map(&maps.b[c], B + 64 * c, N, w, R, NR, "B");
+        if (s != QLORA_OK) return s;
+        const Split sp = split_within(sp_layout, red);
+        SkinnyProblem& p = a.p[c];
+        p = skinny_problem(M, red, sp, 0, 1, kSkinnyOutBf16, w, R, part + poff, ctr + c * mtiles);
+        poff += static_cast<int64_t>(sp_layout.splits) * M * NR;
+        p.scale = scale;
+        p.out_bf16 = sU + (lo.group ? c * lo.r : 64 * c);
+        p.row_ids = lo.ids;
+        p.ids_col0 = 64 * c;
+        p.ids_r = lo.r;
+    }
+    a.status = status;
+    a.timeout_ns = timeout_ns();
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_skinny(maps, a, np, st), 1, "skinny(sU)");
+    return QLORA_OK;
+}
+
+// The projections of a group as column groups of one fused forward; a
+// single weight is one group.
+void set_groups(FusedArgs* fa, const Weights& W, const Lora& lo) {
+    if (!lo.group) {
+        fa->ngroups = 1;
+        fa->group_end[0] = W.N;
+        fa->group_rank_x[0] = 0;
+        return;
+    }
+    fa->ngroups = W.P;
+    for (int i = 0; i < W.P; ++i) {
+        fa->group_end[i] = W.off[i + 1];
+        fa->group_rank_x[i] = i * lo.r;
+    }
+}
+
+// ------------------------------------------- forward and backward bodies --
+// Checks shared by every forward and backward call form.
+qlora_status check_lora(const Lora& lo, int64_t M) {
+    if (!rank_ok(lo.r)) return QLORA_ERR_UNSUPPORTED_RANK;
+    if (lo.P < 1) return QLORA_ERR_INVALID_ARG;
+    if (lo.group && lo.P > kMaxGroups) return QLORA_ERR_INVALID_ARG;
+    if (lo.R() > kMaxMultiRank) return QLORA_ERR_UNSUPPORTED_RANK;
+    if (lo.P > 1 && !lo.group && M > 0 && (!lo.ids || (reinterpret_cast<uintptr_t>(lo.ids) & 3u)))
+        return lo.ids ? QLORA_ERR_MISALIGNED : QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+// cT (the transposed decoded constants the fused matmuls read): each weight
+// of a group at its own column offset.
+qlora_status decode_constants_t(const Weights& W, const Layout& L, float* cT, cudaStream_t st) {
+    for (int i = 0; i < W.P; ++i) {
+        const int64_t cols = i == W.P - 1 ? L.ldc - W.off[i] : W.rows(i);
+        QLORA_LAUNCH(launch_decode_constants_t(constants_of(W.w + i), W.rows(i), W.K, L.ldc, cols, cT + W.off[i], st), 1,
+                     "decode constants");
+    }
+    return QLORA_OK;
+}
+
+qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint16_t* A, const uint16_t* B,
+                      const Lora& lo, float alpha, uint16_t* Y, uint16_t* sT_save, void* ws, size_t ws_bytes,
+                      void* stream) {
+    qlora_status s = check_lora(lo, M);
+    if (s != QLORA_OK) return s;
+    if (M < 0) return QLORA_ERR_BAD_SHAPE;
+    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    if (M == 0) return QLORA_OK;
+    if (!X || !A || !B || !Y || !ws) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(ws) ||
+        (sT_save && !aligned16(sT_save)))
+        return QLORA_ERR_MISALIGNED;
+    const int64_t N = W.N, K = W.K;
+    const int r = lo.r, R = lo.R();
+    const Layout L = layout_for(QLORA_OP_FWD, M, W, lo);
+    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(base + L.status);
+    float* cT = reinterpret_cast<float*>(base + L.cT);
+    float* partT = reinterpret_cast<float*>(base + L.partT);
+    uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
+    const float scale = alpha / static_cast<float>(r);
+    const bool plain = lo.P == 1 && !lo.group;
+
+    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
+    if (M <= small && M <= std::min<int64_t>(g_reg_gemv_max_m.load(), kGemvMmaMaxM)) {
+        // few tokens: rank-r down-projection, then the register-fed GEMV,
+        // launched as its programmatic dependent so the weight stream starts
+        // while sT is still being computed
+        const float* cflat = nullptr;
+        if (lo.group) {
+            // each weight's block constants, decoded into one array in block order
+            cflat = reinterpret_cast<const float*>(base + L.cflat);
+            for (int i = 0; i < W.P; ++i)
+                QLORA_LAUNCH(launch_decode_constants(constants_of(W.w + i), W.rows(i) * K / kBlock,
+                                                     const_cast<float*>(cflat) + W.off[i] * K / kBlock, sms, st),
+                             1, "decode constants");
+        }
+        if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
+                          st)) != QLORA_OK)
+            return s;
+        GemvMmaArgs ga{};
+        ga.X = X;
+        ga.codes = W.w[0].codes;
+        ga.qabsmax = W.w[0].qabsmax;
+        ga.s2 = W.w[0].s2;
+        ga.mean = W.w[0].mean;
+        ga.absmax = lo.group ? cflat : W.w[0].absmax;
+        ga.M = M;
+        ga.N = N;
+        ga.K = K;
+        ga.rank_cols = lo.group ? r : R;
+        ga.sT_ld = R;
+        ga.B_ld = lo.group ? r : R;
+        ga.ngroups = lo.group ? W.P : 1;
+        for (int i = 0; i < ga.ngroups; ++i) {
+            ga.group_end[i] = lo.group ? W.off[i + 1] : N;
+            ga.group_rank_x[i] = lo.group ? i * r : 0;
+        }
+        ga.ctas = L.reg_gemv.ctas;
+        ga.units = L.reg_gemv.units;
+        ga.max_chunks = L.reg_gemv.max_chunks;
+        ga.part = reinterpret_cast<float*>(base + L.partY);
+        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
+        ga.sT = sT;
+        ga.B = B;
+        ga.Y = Y;
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        cudaEvent_t ev0, ev1;
+        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
+        // an event record between the two launches would break the
+        // programmatic edge, so a profiled call launches in plain order
+        QLORA_LAUNCH(launch_gemv_mma(ga, tables(), ev0 == nullptr, st), 1, "register gemv");
+        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
+        return QLORA_OK;
+    }
+    if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
+    if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
+                      st)) != QLORA_OK)
+        return s;
+
+    if (M <= small && plain) {
+        // few tokens: weight-streaming swap-AB kernel, split over K
+        const int Mp = static_cast<int>((M + 15) / 16 * 16);
+        CUtensorMap t_x, t_codes, t_c;
+        QLORA_MAP(&t_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, Mp, CU_TENSOR_MAP_SWIZZLE_128B, "X");
+        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_32B, "codes");
+        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
+        GemvArgs ga{};
+        ga.M = M;
+        ga.N = N;
+        ga.K = K;
+        ga.Mp = Mp;
+        ga.r = r;
+        ga.splits = L.gemv.splits;
+        ga.steps_per_split = L.gemv.steps;
+        ga.part = reinterpret_cast<float*>(base + L.partY);
+        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
+        ga.sT = sT;
+        ga.B = B;
+        ga.Y = Y;
+        ga.status = status;
+        ga.timeout_ns = timeout_ns();
+        if (injected_failure()) return QLORA_ERR_CUDA;
+        cudaEvent_t ev0, ev1;
+        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
+        QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
+        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
+        return QLORA_OK;
+    }
+
+    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
+    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");
+    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 256,
+              CU_TENSOR_MAP_SWIZZLE_32B, "codes");
+    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+              "constants");
+    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sT, R, M, R * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sT");
+    // B [N, R] (one adapter or several side by side), or the stacked B_i [N, r] of a group
+    const int bcols = lo.group ? r : R;
+    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, bcols, N, bcols * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "B");
+    FusedArgs fa{};
+    fa.M = M;
+    fa.out_cols = N;
+    fa.red = K;
+    fa.rank_cols = lo.group ? r : R;
+    fa.rank_steps = lo.group ? 1 : lo.chunks();
+    set_groups(&fa, W, lo);
+    fa.ctas = fused_ctas(M, fused_tiles_n(fa), K, std::min(sms, kPlanSms));
+    fa.out = Y;
+    fa.part = reinterpret_cast<float*>(base + L.skpart);
+    fa.flags = reinterpret_cast<int*>(base + L.flags);
+    fa.status = status;
+    fa.timeout_ns = timeout_ns();
+    fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
+    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
+    // programmatic dependent of the sT launch: the main loop overlaps it
+    // (a profiled call keeps plain stream order)
+    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
+                 "fused forward");
+    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
+    return QLORA_OK;
+}
+
+qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const Weights& W, const uint16_t* A,
+                      const uint16_t* B, const Lora& lo, float alpha, const uint16_t* sT_in, uint16_t* dX, float* dA,
+                      float* dB, void* ws, size_t ws_bytes, void* stream) {
+    qlora_status s = check_lora(lo, M);
+    if (s != QLORA_OK) return s;
+    if (M < 0) return QLORA_ERR_BAD_SHAPE;
+    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+    if (!dA || !dB || !A || !B || !ws) return QLORA_ERR_INVALID_ARG;
+    if (M > 0 && (!dY || !X || !dX)) return QLORA_ERR_INVALID_ARG;
+    if ((M > 0 && (!aligned16(dY) || !aligned16(X) || !aligned16(dX))) || !aligned16(A) || !aligned16(B) ||
+        !aligned16(dA) || !aligned16(dB) || !aligned16(ws) || (sT_in && !aligned16(sT_in)))
+        return QLORA_ERR_MISALIGNED;
+    const int64_t N = W.N, K = W.K;
+    const int r = lo.r, R = lo.R();
+    const Layout L = layout_for(QLORA_OP_BWD, M, W, lo);
+    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    int sms = 0;
+    if ((s = device_ready(&sms)) != QLORA_OK) return s;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t dB_cols = lo.group ? r : R;
+    if (M == 0) {  // an empty batch: the adapter gradients are exactly zero
+        QLORA_TRY(cudaMemsetAsync(dA, 0, static_cast<size_t>(R) * K * 4, st), "zero dA");
+        QLORA_TRY(cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * dB_cols * 4, st), "zero dB");
+        return QLORA_OK;
+    }
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int* status = reinterpret_cast<int*>(base + L.status);
+    float* cT = reinterpret_cast<float*>(base + L.cT);
+    float* partU = reinterpret_cast<float*>(base + L.partU);
+    uint16_t* sU = reinterpret_cast<uint16_t*>(base + L.sU);
+    const uint16_t* sT = sT_in ? sT_in : reinterpret_cast<uint16_t*>(base + L.sT);
+    float* partA = reinterpret_cast<float*>(base + L.partA);
+    const float scale = alpha / static_cast<float>(r);
+    const int NRc = rank_pad(std::min(R, 64));
+    const int nch = lo.chunks(), ndb = lo.grad_b();
+
+    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
+    // sU = s dY B, with B read in place (MN-major)
+    if ((s = down_bwd(dY, M, W, B, lo, scale, L.sU_split, partU, reinterpret_cast<int*>(base + L.ctrU), sU, status,
+                      st)) != QLORA_OK)
+        return s;
+    // sT from the forward, or recomputed
+    if (!sT_in) {
+        if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partU, reinterpret_cast<int*>(base + L.ctrT),
+                          reinterpret_cast<uint16_t*>(base + L.sT), status, st)) != QLORA_OK)
+            return s;
+    }
+
+    // dX = dY deq(W) + sU A
+    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
+    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "dY");
+    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 128, 64,
+              CU_TENSOR_MAP_SWIZZLE_128B, "codes");
+    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 4, CU_TENSOR_MAP_SWIZZLE_NONE,
+              "constants");
+    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sU, R, M, R * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sU");
+    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, R, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+    FusedArgs fa{};
+    fa.M = M;
+    fa.out_cols = K;
+    fa.red = N;
+    fa.rank_cols = R;
+    fa.rank_steps = nch;
+    fa.ngroups = 1;
+    fa.group_end[0] = K;
+    fa.group_rank_x[0] = 0;
+    fa.ctas = fused_ctas(M, fused_tiles_n(fa), N, std::min(sms, kPlanSms));
+    fa.out = dX;
+    fa.part = reinterpret_cast<float*>(base + L.skpart);
+    fa.flags = reinterpret_cast<int*>(base + L.flags);
+    fa.status = status;
+    fa.timeout_ns = timeout_ns();
+    fa.stall_producer = 0;
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
+    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
+    // plain stream order after the rank-r launches: the adapter gradients,
+    // dX's programmatic dependent, read sU and sT from their first step
+    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
+    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
+
+    // dA = sU^T X (as dA^T[K, R] = X^T sU, in 64-column chunks) and dB = dY^T sT
+    // (chunks of sT, or per projection of a group dB_i = dY_i^T sT_i), split
+    // over tokens
+    SkinnyMaps maps;
+    SkinnyArgs ga{};
+    ga.NR = NRc;
+    const Split gsp = capped(L.grad_split, M);
+    const int64_t ktiles = cdiv(K, 128), ntiles = cdiv(N, 128);
+    CUtensorMap t_xt;
+    QLORA_MAP(&t_xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
+    int np = 0;
+    int64_t poff = 0;
+    for (int c = 0; c < nch; ++c, ++np) {
+        const int w = std::min(64, R - 64 * c);
+        maps.a[np] = t_xt;
+        if ((s = make_rank_map(&maps.b[np], sU + 64 * c, M, w, R, NRc, "sU")) != QLORA_OK) return s;
+        ga.p[np] = skinny_problem(K, M, gsp, 1, 1, kSkinnyOutF32Transposed, w, K, partA + poff,
+                                  reinterpret_cast<int*>(base + L.ctrA) + c * ktiles);
+        ga.p[np].out_f32 = dA + static_cast<int64_t>(64 * c) * K;
+        poff += static_cast<int64_t>(L.grad_split.splits) * K * NRc;
+    }
+    for (int c = 0; c < ndb; ++c, ++np) {
+        const int64_t n0 = lo.group ? W.off[c] : 0, rows = lo.group ? W.rows(c) : N;
+        const int w = lo.group ? r : std::min(64, R - 64 * c);
+        QLORA_MAP(&maps.a[np], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY + n0, rows, M, N * 2, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
+        if ((s = make_rank_map(&maps.b[np], sT + (lo.group ? c * r : 64 * c), M, w, R, NRc, "sT")) != QLORA_OK)
+            return s;
+        ga.p[np] = skinny_problem(rows, M, gsp, 1, 1, kSkinnyOutF32, w, dB_cols, partA + poff,
+                                  reinterpret_cast<int*>(base + L.ctrB) + c * ntiles);
+        ga.p[np].out_f32 = dB + (lo.group ? n0 * r : 64 * c);
+        poff += static_cast<int64_t>(L.grad_split.splits) * rows * NRc;
+    }
+    ga.status = status;
+    ga.timeout_ns = timeout_ns();
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    // dA and dB need only sU and sT: launched as dX's programmatic
+    // dependent they start once every dX tile has started, on the SMs dX's
+    // last wave leaves idle (a profiled call keeps plain stream order)
+    QLORA_LAUNCH(launch_skinny(maps, ga, np, st, ev1 == nullptr), 1, "skinny(grads)");
+    return QLORA_OK;
+}
+
+Weights single_weight(const qlora_nf4_weight* w) {
+    Weights W;
+    W.w = w;
+    W.P = 1;
+    W.N = w->N;
+    W.K = w->K;
+    W.off[0] = 0;
+    W.off[1] = w->N;
+    return W;
 }
 
 }  // namespace
@@ -458,7 +939,12 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     }
     if (op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
     if (M < 0 || !rank_ok(r)) return 0;
-    return layout_for(op, M, N, K, r).total;
+    qlora_nf4_weight w{};
+    w.N = N;
+    w.K = K;
+    Lora lo;
+    lo.r = r;
+    return layout_for(op, M, single_weight(&w), lo).total;
 }
 
 const char* qlora_status_string(qlora_status s) {
@@ -629,136 +1115,9 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_weig
                               size_t ws_bytes, void* stream) {
     qlora_status s = check_weight(w);
     if (s != QLORA_OK) return s;
-    if (M < 0) return QLORA_ERR_BAD_SHAPE;
-    if (!rank_ok(r)) return QLORA_ERR_UNSUPPORTED_RANK;
-    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-    if (M == 0) return QLORA_OK;
-    if (!X || !A || !B || !Y || !ws) return QLORA_ERR_INVALID_ARG;
-    if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(ws) ||
-        (sT_save && !aligned16(sT_save)))
-        return QLORA_ERR_MISALIGNED;
-    const int64_t N = w->N, K = w->K;
-    const Layout L = layout_for(QLORA_OP_FWD, M, N, K, r);
-    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    int sms = 0;
-    if ((s = device_ready(&sms)) != QLORA_OK) return s;
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t* base = static_cast<uint8_t*>(ws);
-    int* status = reinterpret_cast<int*>(base + L.status);
-    float* cT = reinterpret_cast<float*>(base + L.cT);
-    float* partT = reinterpret_cast<float*>(base + L.partT);
-    uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
-    const float scale = alpha / static_cast<float>(r);
-
-    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
-    if (M <= small && M <= std::min<int64_t>(g_reg_gemv_max_m.load(), kGemvMmaMaxM)) {
-        // few tokens: rank-r down-projection, then the register-fed GEMV,
-        // launched as its programmatic dependent so the weight stream starts
-        // while sT is still being computed
-        if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
-                           status, st)) != QLORA_OK)
-            return s;
-        GemvMmaArgs ga{};
-        ga.X = X;
-        ga.codes = w->codes;
-        ga.qabsmax = w->qabsmax;
-        ga.s2 = w->s2;
-        ga.mean = w->mean;
-        ga.absmax = w->absmax;
-        ga.M = M;
-        ga.N = N;
-        ga.K = K;
-        ga.r = r;
-        ga.ctas = L.reg_gemv.ctas;
-        ga.units = L.reg_gemv.units;
-        ga.max_chunks = L.reg_gemv.max_chunks;
-        ga.part = reinterpret_cast<float*>(base + L.partY);
-        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
-        ga.sT = sT;
-        ga.B = B;
-        ga.Y = Y;
-        if (injected_failure()) return QLORA_ERR_CUDA;
-        cudaEvent_t ev0, ev1;
-        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-        // an event record between the two launches would break the
-        // programmatic edge, so a profiled call launches in plain order
-        QLORA_LAUNCH(launch_gemv_mma(ga, tables(), ev0 == nullptr, st), 1, "register gemv");
-        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
-        return QLORA_OK;
-    }
-    QLORA_LAUNCH(launch_decode_constants_t(constants_of(w), N, K, L.ldc, cT, st), 1, "decode constants");
-    if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT,
-                       status, st)) != QLORA_OK)
-        return s;
-
-    if (M <= small) {
-        // few tokens: weight-streaming swap-AB kernel, split over K
-        const int Mp = static_cast<int>((M + 15) / 16 * 16);
-        CUtensorMap t_x, t_codes, t_c;
-        QLORA_MAP(&t_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, Mp, CU_TENSOR_MAP_SWIZZLE_128B, "X");
-        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 32, 128,
-                  CU_TENSOR_MAP_SWIZZLE_32B, "codes");
-        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
-        GemvArgs ga{};
-        ga.M = M;
-        ga.N = N;
-        ga.K = K;
-        ga.Mp = Mp;
-        ga.r = r;
-        ga.splits = L.gemv.splits;
-        ga.steps_per_split = L.gemv.steps;
-        ga.part = reinterpret_cast<float*>(base + L.partY);
-        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
-        ga.sT = sT;
-        ga.B = B;
-        ga.Y = Y;
-        ga.status = status;
-        ga.timeout_ns = timeout_ns();
-        if (injected_failure()) return QLORA_ERR_CUDA;
-        cudaEvent_t ev0, ev1;
-        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-        QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
-        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
-        return QLORA_OK;
-    }
-
-    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
-    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");
-    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 32, 256, CU_TENSOR_MAP_SWIZZLE_32B,
-              "codes");
-    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
-              "constants");
-    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sT, r, M, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sT");
-    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, r, N, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "B");
-    FusedArgs fa{};
-    fa.M = M;
-    fa.out_cols = N;
-    fa.red = K;
-    fa.r = r;
-    fa.ctas = fused_ctas(M, N, K, std::min(sms, kPlanSms));
-    fa.out = Y;
-    fa.part = reinterpret_cast<float*>(base + L.skpart);
-    fa.flags = reinterpret_cast<int*>(base + L.flags);
-    fa.status = status;
-    fa.timeout_ns = timeout_ns();
-    fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    cudaEvent_t ev0, ev1;
-    take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-    // programmatic dependent of the sT launch: the main loop overlaps it
-    // (a profiled call keeps plain stream order)
-    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
-                 "fused forward");
-    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
-    return QLORA_OK;
+    Lora lo;
+    lo.r = r;
+    return fwd_impl(X, M, single_weight(w), A, B, lo, alpha, Y, sT_save, ws, ws_bytes, stream);
 }
 
 qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
@@ -766,113 +1125,96 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, 
                               uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
     qlora_status s = check_weight(w);
     if (s != QLORA_OK) return s;
-    if (M < 0) return QLORA_ERR_BAD_SHAPE;
-    if (!rank_ok(r)) return QLORA_ERR_UNSUPPORTED_RANK;
-    if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-    if (!dA || !dB || !A || !B || !ws) return QLORA_ERR_INVALID_ARG;
-    if (M > 0 && (!dY || !X || !dX)) return QLORA_ERR_INVALID_ARG;
-    if ((M > 0 && (!aligned16(dY) || !aligned16(X) || !aligned16(dX))) || !aligned16(A) || !aligned16(B) ||
-        !aligned16(dA) || !aligned16(dB) || !aligned16(ws) || (sT_in && !aligned16(sT_in)))
-        return QLORA_ERR_MISALIGNED;
-    const int64_t N = w->N, K = w->K;
-    const Layout L = layout_for(QLORA_OP_BWD, M, N, K, r);
-    if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE_TOO_SMALL;
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    int sms = 0;
-    if ((s = device_ready(&sms)) != QLORA_OK) return s;
+    Lora lo;
+    lo.r = r;
+    return bwd_impl(dY, X, M, single_weight(w), A, B, lo, alpha, sT_in, dX, dA, dB, ws, ws_bytes, stream);
+}
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (M == 0) {  // an empty batch: the adapter gradients are exactly zero
-        QLORA_TRY(cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 4, st), "zero dA");
-        QLORA_TRY(cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 4, st), "zero dB");
-        return QLORA_OK;
+size_t qlora_workspace_bytes_multi(int op, int64_t M, int64_t N, int64_t K, int r, int P) {
+    if (N <= 0 || K <= 0 || K % kBlock != 0) return 0;
+    if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || M < 0 || !rank_ok(r) || P < 1 || P * r > kMaxMultiRank)
+        return 0;
+    qlora_nf4_weight w{};
+    w.N = N;
+    w.K = K;
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    return layout_for(op, M, single_weight(&w), lo).total;
+}
+
+qlora_status qlora_linear_fwd_multi(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
+                                    const uint16_t* B, int r, int P, const int32_t* ids, float alpha, uint16_t* Y,
+                                    uint16_t* sT_save, void* ws, size_t ws_bytes, void* stream) {
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    lo.ids = ids;
+    return fwd_impl(X, M, single_weight(w), A, B, lo, alpha, Y, sT_save, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_multi(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                                    const uint16_t* A, const uint16_t* B, int r, int P, const int32_t* ids,
+                                    float alpha, const uint16_t* sT, uint16_t* dX, float* dA, float* dB, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    qlora_status s = check_weight(w);
+    if (s != QLORA_OK) return s;
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    lo.ids = ids;
+    return bwd_impl(dY, X, M, single_weight(w), A, B, lo, alpha, sT, dX, dA, dB, ws, ws_bytes, stream);
+}
+
+size_t qlora_workspace_bytes_group(int op, int64_t M, const int64_t* N, int P, int64_t K, int r) {
+    if (!N || P < 1 || P > kMaxGroups || K <= 0 || K % kBlock != 0) return 0;
+    if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || M < 0 || !rank_ok(r)) return 0;
+    qlora_nf4_weight w[kMaxGroups] = {};
+    Weights W;
+    W.w = w;
+    W.P = P;
+    W.K = K;
+    for (int i = 0; i < P; ++i) {
+        if (N[i] <= 0) return 0;
+        w[i].N = N[i];
+        w[i].K = K;
+        W.off[i + 1] = W.off[i] + N[i];
     }
-    uint8_t* base = static_cast<uint8_t*>(ws);
-    int* status = reinterpret_cast<int*>(base + L.status);
-    float* cT = reinterpret_cast<float*>(base + L.cT);
-    float* partU = reinterpret_cast<float*>(base + L.partU);
-    uint16_t* sU = reinterpret_cast<uint16_t*>(base + L.sU);
-    const uint16_t* sT = sT_in ? sT_in : reinterpret_cast<uint16_t*>(base + L.sT);
-    float* partA = reinterpret_cast<float*>(base + L.partA);
-    const float scale = alpha / static_cast<float>(r);
-    const int NR = rank_pad(r);
+    W.N = W.off[P];
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    lo.group = true;
+    return layout_for(op, M, W, lo).total;
+}
 
-    QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_decode_constants_t(constants_of(w), N, K, L.ldc, cT, st), 1, "decode constants");
-    // sU = s dY B, with B [N, r] read in place (MN-major)
-    if ((s = lora_down(dY, M, N, B, true, r, scale, L.sU_split, partU, reinterpret_cast<int*>(base + L.ctrU), sU,
-                       status, st)) != QLORA_OK)
-        return s;
-    // sT from the forward, or recomputed
-    if (!sT_in) {
-        if ((s = lora_down(X, M, K, A, false, r, scale, L.sT_split, partU, reinterpret_cast<int*>(base + L.ctrT),
-                           reinterpret_cast<uint16_t*>(base + L.sT), status, st)) != QLORA_OK)
-            return s;
-    }
+qlora_status qlora_linear_fwd_group(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, int P,
+                                    const uint16_t* A, const uint16_t* B, int r, float alpha, uint16_t* Y,
+                                    uint16_t* sT_save, void* ws, size_t ws_bytes, void* stream) {
+    Weights W;
+    qlora_status s = check_weights(w, P, &W);
+    if (s != QLORA_OK) return s;
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    lo.group = true;
+    return fwd_impl(X, M, W, A, B, lo, alpha, Y, sT_save, ws, ws_bytes, stream);
+}
 
-    // dX = dY deq(W) + sU A
-    CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
-    QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "dY");
-    QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B,
-              "codes");
-    QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 4, CU_TENSOR_MAP_SWIZZLE_NONE,
-              "constants");
-    QLORA_MAP(&t_lact, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sU, r, M, r * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "sU");
-    QLORA_MAP(&t_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, r, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "A");
-    FusedArgs fa{};
-    fa.M = M;
-    fa.out_cols = K;
-    fa.red = N;
-    fa.r = r;
-    fa.ctas = fused_ctas(M, K, N, std::min(sms, kPlanSms));
-    fa.out = dX;
-    fa.part = reinterpret_cast<float*>(base + L.skpart);
-    fa.flags = reinterpret_cast<int*>(base + L.flags);
-    fa.status = status;
-    fa.timeout_ns = timeout_ns();
-    fa.stall_producer = 0;
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    cudaEvent_t ev0, ev1;
-    take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
-    if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-    // plain stream order after the rank-r launches: the adapter gradients,
-    // dX's programmatic dependent, read sU and sT from their first step
-    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
-    if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
-
-    // dA = sU^T X (as dA^T[K, r] = X^T sU) and dB = dY^T sT, split over tokens
-    CUtensorMap ta0, tb0, ta1, tb1;
-    QLORA_MAP(&ta0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
-    if ((s = make_rank_map(&tb0, sU, M, r, "sU")) != QLORA_OK) return s;
-    QLORA_MAP(&ta1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
-    if ((s = make_rank_map(&tb1, sT, M, r, "sT")) != QLORA_OK) return s;
-    SkinnyArgs ga{};
-    ga.NR = NR;
-    ga.r = r;
-    const Split gsp = capped(L.grad_split, M);
-    for (int p = 0; p < 2; ++p) {
-        SkinnyProblem& P = ga.p[p];
-        P.rows = p == 0 ? K : N;
-        P.red = M;
-        P.splits = gsp.splits;
-        P.steps_per_split = gsp.steps;
-        P.a_mn_major = 1;
-        P.b_mn_major = 1;
-        P.mode = p == 0 ? kSkinnyOutF32Transposed : kSkinnyOutF32;
-        P.scale = 1.0f;
-        P.part = partA + (p == 0 ? 0 : static_cast<int64_t>(L.grad_split.splits) * K * NR);
-        P.counter = reinterpret_cast<int*>(base + (p == 0 ? L.ctrA : L.ctrB));
-        P.out_f32 = p == 0 ? dA : dB;
-    }
-    ga.status = status;
-    ga.timeout_ns = timeout_ns();
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    // dA and dB need only sU and sT: launched as dX's programmatic
-    // dependent they start once every dX tile has started, on the SMs dX's
-    // last wave leaves idle (a profiled call keeps plain stream order)
-    QLORA_LAUNCH(launch_skinny(ta0, tb0, ta1, tb1, ga, 2, st, ev1 == nullptr), 1, "skinny(grads)");
-    return QLORA_OK;
+qlora_status qlora_linear_bwd_group(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                                    int P, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                                    const uint16_t* sT, uint16_t* dX, float* dA, float* dB, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    Weights W;
+    qlora_status s = check_weights(w, P, &W);
+    if (s != QLORA_OK) return s;
+    Lora lo;
+    lo.r = r;
+    lo.P = P;
+    lo.group = true;
+    return bwd_impl(dY, X, M, W, A, B, lo, alpha, sT, dX, dA, dB, ws, ws_bytes, stream);
 }
 
 qlora_status qlora_device_status(const void* ws, int* status_host, void* stream) {

@@ -67,48 +67,71 @@ __device__ __forceinline__ void dequant_block(const Nf4Tables& tab, float cprime
 // Stream-K schedule. The work is the list of (output tile, 64-deep reduction
 // step) units, tile-major; CTA c (one per SM) takes the contiguous range
 // [c W / P, (c + 1) W / P). Cut at tile boundaries, a range is a list of
-// segments. A segment that starts at step 0 makes its CTA the tile's owner:
-// it also runs the rank-r step and writes the tile. A segment that starts
-// later is a contributor: it writes its fp32 partial tile and raises a flag.
-// Contributions come first in a CTA's range and ownership last, so an owner
-// finds its partials ready, adds them in CTA order (deterministic) and
-// writes the bf16 tile.
+// segments. The CTA that holds a tile's last step owns the tile: it also runs
+// the rank-r steps and writes the tile. A segment that ends before the tile's
+// last step is a contributor: it writes its fp32 partial tile and raises a
+// flag. Every CTA walks its segments from last to first, so its contribution
+// (the head of the next tile, at the end of its range) comes first and its
+// ownership (the tail of a tile, at the start of its range) last: an owner
+// finds the partials of the lower-indexed CTAs ready, adds them in CTA order
+// (deterministic) and writes the bf16 tile. An owner waits only for CTAs with
+// lower indices, which the hardware has dispatched before it.
 struct Sched {
     int64_t W;    // tiles * KT
     int P;        // CTAs
     int KT;       // reduction steps per tile
-    int tiles_n;  // tiles along the output columns
     __device__ int64_t begin(int c) const { return static_cast<int64_t>(c) * W / P; }
     __device__ int cta_of(int64_t u) const { return static_cast<int>(((u + 1) * P - 1) / W); }
 };
 
-// Walks the segments of one CTA's range. Without splitting (kSplit false:
-// one CTA per tile) the range is exactly tile c, all of its steps.
+// Walks the segments of one CTA's range, last to first. Without splitting
+// (kSplit false: one CTA per tile) the range is exactly tile c, all of its
+// steps.
 template <bool kSplit>
 struct SegIter {
     const Sched& sc;
-    int64_t u, end;
+    int64_t lo, hi;  // units not yet walked: [lo, hi)
     int64_t tile;
     int k_lo, k_hi;
     __device__ SegIter(const Sched& s, int c)
-        : sc(s), u(kSplit ? s.begin(c) : static_cast<int64_t>(c) * s.KT),
-          end(kSplit ? s.begin(c + 1) : static_cast<int64_t>(c + 1) * s.KT), tile(0), k_lo(0), k_hi(0) {}
+        : sc(s), lo(kSplit ? s.begin(c) : static_cast<int64_t>(c) * s.KT),
+          hi(kSplit ? s.begin(c + 1) : static_cast<int64_t>(c + 1) * s.KT), tile(0), k_lo(0), k_hi(0) {}
     __device__ bool next() {
-        if (u >= end) return false;
+        if (hi <= lo) return false;
         if (!kSplit) {
-            tile = u / sc.KT;
+            tile = lo / sc.KT;
             k_lo = 0;
             k_hi = sc.KT;
-            u = end;
+            hi = lo;
             return true;
         }
-        tile = u / sc.KT;
-        k_lo = static_cast<int>(u - tile * sc.KT);
-        k_hi = static_cast<int>(min(static_cast<int64_t>(sc.KT), end - tile * sc.KT));
-        u = tile * sc.KT + k_hi;
+        tile = (hi - 1) / sc.KT;
+        const int64_t t0 = tile * sc.KT;
+        const int64_t start = max(lo, t0);
+        k_lo = static_cast<int>(start - t0);
+        k_hi = static_cast<int>(hi - t0);
+        hi = start;
         return true;
     }
+    __device__ bool owner() const { return k_hi == sc.KT; }
 };
+
+// The output columns of column tile j: [n0, n_lim), and the act-side column
+// of its rank input. Tiles are 256 columns, counted group by group.
+struct TileCols {
+    int64_t n0, n_lim;
+    int rank_x;
+};
+__device__ __forceinline__ TileCols tile_cols(const FusedArgs& a, int64_t j) {
+    int64_t start = 0;
+    for (int g = 0; g < a.ngroups; ++g) {
+        const int64_t cnt = (a.group_end[g] - start + kFusedBN - 1) / kFusedBN;
+        if (j < cnt || g == a.ngroups - 1) return TileCols{start + j * kFusedBN, a.group_end[g], a.group_rank_x[g]};
+        j -= cnt;
+        start = a.group_end[g];
+    }
+    return TileCols{0, 0, 0};
+}
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -144,11 +167,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = static_cast<int>((args.red + kFusedBK - 1) / kFusedBK);
-    const int tiles_n = static_cast<int>((args.out_cols + kFusedBN - 1) / kFusedBN);
+    int tiles_n = 0;
+    {
+        int64_t start = 0;
+        for (int g = 0; g < args.ngroups; ++g) {
+            tiles_n += static_cast<int>((args.group_end[g] - start + kFusedBN - 1) / kFusedBN);
+            start = args.group_end[g];
+        }
+    }
     const int tiles_m = static_cast<int>((args.M + kFusedBM - 1) / kFusedBM);
-    const Sched sc{static_cast<int64_t>(tiles_m) * tiles_n * KT, static_cast<int>(gridDim.x), KT, tiles_n};
+    const Sched sc{static_cast<int64_t>(tiles_m) * tiles_n * KT, static_cast<int>(gridDim.x), KT};
     const int cta = blockIdx.x;
-    const bool has_lora = args.r > 0;
+    const int rank_steps = args.rank_cols > 0 ? args.rank_steps : 0;
     const uint64_t tmo = args.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -188,9 +218,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             SegIter<kSplit> it(sc, cta);
             while (!args.stall_producer && !*abort_flag && it.next()) {
                 ++seg;
-                const int64_t m0 = (it.tile / tiles_n) * kFusedBM, n0 = (it.tile % tiles_n) * kFusedBN;
+                const int64_t m0 = (it.tile / tiles_n) * kFusedBM;
+                const TileCols tc = tile_cols(args, it.tile % tiles_n);
+                const int64_t n0 = tc.n0;
                 const int nk = it.k_hi - it.k_lo;
-                const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+                const int steps = nk + (it.owner() ? rank_steps : 0);
                 for (int i = 0; i < steps; ++i, ++g) {
                     const int s = g % kFusedStages;
                     const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
@@ -214,22 +246,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                             tma_load_2d(st + kOffC, &tm_c, full + s, kt * kFusedBK, static_cast<int>(n0 / kBlock));
                         }
                     } else {
-                        // the rank-r input (sT or sU) comes from the preceding
-                        // launch, of which this one may be a programmatic dependent
-                        asm volatile("griddepcontrol.wait;" ::: "memory");
-                        // the rank-r step lands in a weight-tile region, which the
-                        // previous segment's epilogue uses as scratch: wait for it
-                        if (seg > 0 && !mbar_wait(tmem_free, static_cast<uint32_t>(seg - 1) & 1u, tmo, args.status)) {
-                            *abort_flag = 1;
-                            break;
+                        const int c = i - nk;  // rank step: columns 64c .. 64c + 63 of the rank term
+                        if (c == 0) {
+                            // the rank-r input (sT or sU) comes from the preceding
+                            // launch, of which this one may be a programmatic dependent
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                            // the rank steps land in weight-tile regions, one of which
+                            // the previous segment's epilogue uses as scratch: wait for it
+                            if (seg > 0 &&
+                                !mbar_wait(tmem_free, static_cast<uint32_t>(seg - 1) & 1u, tmo, args.status)) {
+                                *abort_flag = 1;
+                                break;
+                            }
                         }
                         mbar_arrive_expect_tx(full + s, kActBytes + kWBytes);
-                        tma_load_2d(st, &tm_lact, full + s, 0, static_cast<int>(m0));
+                        tma_load_2d(st, &tm_lact, full + s, tc.rank_x + 64 * c, static_cast<int>(m0));
                         if (!kTransW) {
-                            tma_load_2d(st + kOffW, &tm_lw, full + s, 0, static_cast<int>(n0));
+                            tma_load_2d(st + kOffW, &tm_lw, full + s, 64 * c, static_cast<int>(n0));
                         } else {
                             for (int a = 0; a < 4; ++a)
-                                tma_load_2d(st + kOffW + a * 8192, &tm_lw, full + s, static_cast<int>(n0) + 64 * a, 0);
+                                tma_load_2d(st + kOffW + a * 8192, &tm_lw, full + s, static_cast<int>(n0) + 64 * a,
+                                            64 * c);
                         }
                     }
                     last_use[s] = static_cast<int>(u);
@@ -255,7 +292,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 }
                 tc_fence_after();
                 const int nk = it.k_hi - it.k_lo;
-                const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+                const int steps = nk + (it.owner() ? rank_steps : 0);
                 for (int i = 0; i < steps; ++i, ++g) {
                     const int s = g % kFusedStages;
                     const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
@@ -266,7 +303,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                     tc_fence_after();
                     const uint32_t act = smem_u32(smem + s * kStageBytes);
                     const uint32_t wt = act + kOffW;
-                    const int ksub = (i < nk) ? (kFusedBK / 16) : (args.r + 15) / 16;
+                    const int ksub = (i < nk) ? (kFusedBK / 16) : (min(64, args.rank_cols - 64 * (i - nk)) + 15) / 16;
                     for (int kk = 0; kk < ksub; ++kk) {
                         const uint64_t bdesc = kTransW ? sw128_desc(wt + kk * 2048, 8192, 1024)
                                                        : sw128_desc(wt + kk * 32, 16, 1024);
@@ -297,9 +334,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         int g = 0, seg = 0;
         SegIter<kSplit> it(sc, cta);
         while (it.next()) {
-            const int64_t m0 = (it.tile / tiles_n) * kFusedBM, n0 = (it.tile % tiles_n) * kFusedBN;
+            const int64_t m0 = (it.tile / tiles_n) * kFusedBM;
+            const TileCols tc = tile_cols(args, it.tile % tiles_n);
+            const int64_t n0 = tc.n0;
             const int nk = it.k_hi - it.k_lo;
-            const int steps = nk + ((it.k_lo == 0 && has_lora) ? 1 : 0);
+            const int steps = nk + (it.owner() ? rank_steps : 0);
             for (int i = 0; ok && i < steps; ++i, ++g) {
                 const int s = g % kFusedStages;
                 const uint32_t u = static_cast<uint32_t>(g / kFusedStages);
@@ -345,7 +384,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             // ((c * 8 + i) * 256 + t), so each warp instruction moves 512
             // contiguous bytes.
             const int64_t tile_floats = static_cast<int64_t>(kFusedBM) * kFusedBN;
-            if (kSplit && it.k_lo > 0) {
+            if (kSplit && !it.owner()) {
                 // contributor: the fp32 partial tile, then the flag
                 float4* my_part = reinterpret_cast<float4*>(args.part + static_cast<int64_t>(cta) * tile_floats) + t;
                 const bool live = m0 + row_l < args.M;  // rows past M are never read back
@@ -367,9 +406,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 epi_bar();
                 if (t == 0 && good) st_release(args.flags + cta, 1);
             } else {
-                // owner: wait for the contributors of the tile's later steps
-                const int first = cta + 1;
-                const int last = (kSplit && it.k_hi < KT) ? sc.cta_of(it.tile * KT + KT - 1) : cta;
+                // owner: wait for the contributors of the tile's earlier steps
+                const int first = (kSplit && it.k_lo > 0) ? sc.cta_of(it.tile * KT) : cta;
+                const int last = cta - 1;
                 if (first <= last) {  // only a split tile waits and fences
                 if (t == 0) {
                     int okp = good ? 1 : 0;
@@ -433,7 +472,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                             const int64_t orow = m0 + row_l - lane + rr;
                             const int64_t ocol = n0 + 32 * c + 8 * pc;
                             const uint4 d = lds128(scratch + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4));
-                            if (orow < args.M && ocol < args.out_cols)
+                            if (orow < args.M && ocol < tc.n_lim)
                                 *reinterpret_cast<uint4*>(args.out + orow * args.out_cols + ocol) = d;
                         }
                     }
@@ -477,7 +516,7 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, a.out_cols))
+    if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, fused_tiles_n(a)))
         return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, false>, act, codes, cT, lact, lw, a, tab);
     return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, true>, act, codes, cT, lact, lw, a, tab);
 }

@@ -13,7 +13,11 @@
 //         place with a 32/64/128-byte swizzle matching NR).
 // The reduction is split over CTAs; each CTA writes fp32 partials and the last
 // CTA of a row tile (atomic ticket, no waiting) adds them in split order and
-// writes the result, so outputs are deterministic.
+// writes the result, so outputs are deterministic. One launch carries up to
+// eight such problems (grid.z), each with its own pair of operand maps: the
+// 64-column chunks of a rank above 64 (several adapters side by side), the
+// projections of a group, or dA and dB together. A bf16 output may zero, per
+// token row, the columns of the adapters that the row does not use.
 //   warp 0 TMA producer, warp 1 TMEM owner + UMMA issuer, warps 2-5 epilogue.
 #include <algorithm>
 
@@ -49,9 +53,7 @@ __device__ __forceinline__ uint64_t mn_b_desc(uint32_t addr, int NR) {
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
-    skinny_gemm(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
-                const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
-                const SkinnyArgs args) {
+    skinny_gemm(const __grid_constant__ SkinnyMaps maps, const __grid_constant__ SkinnyArgs args) {
     // a launch that depends on this one programmatically may be scheduled
     // now; it waits for this grid's completion before reading its output
     asm volatile("griddepcontrol.launch_dependents;");
@@ -59,8 +61,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     const SkinnyProblem P = args.p[prob];
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
     if (row0 >= P.rows || static_cast<int>(blockIdx.y) >= P.splits) return;  // whole CTA idle
-    const CUtensorMap* ta = prob ? &tm_a1 : &tm_a0;
-    const CUtensorMap* tb = prob ? &tm_b1 : &tm_b0;
+    const CUtensorMap* ta = &maps.a[prob];
+    const CUtensorMap* tb = &maps.b[prob];
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,11 +119,12 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                 const int k = (k_begin + i) * 64;
                 uint8_t* st = smem + s * kStage;
                 mbar_arrive_expect_tx(full + s, kABytes + b_bytes);
+                const int ar = static_cast<int>(row0);
                 if (!P.a_mn_major) {
-                    tma_load_2d(st, ta, full + s, k, static_cast<int>(row0));
+                    tma_load_2d(st, ta, full + s, k, ar);
                 } else {
-                    tma_load_2d(st, ta, full + s, static_cast<int>(row0), k);
-                    tma_load_2d(st + 8192, ta, full + s, static_cast<int>(row0) + 64, k);
+                    tma_load_2d(st, ta, full + s, ar, k);
+                    tma_load_2d(st + 8192, ta, full + s, ar + 64, k);
                 }
                 if (!P.b_mn_major)
                     tma_load_2d(st + kABytes, tb, full + s, k, 0);
@@ -234,23 +237,28 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             }
         }
         if (last && row < P.rows) {
-            const int r = args.r;
+            const int nc = P.ncols;
             if (P.mode == kSkinnyOutBf16) {
-                uint16_t* o = P.out_bf16 + row * r;
+                uint16_t* o = P.out_bf16 + row * P.out_ld;
+                // the adapter of this token row (row_ids set): columns of
+                // other adapters are written as zeros
+                const int id = P.row_ids ? __ldg(P.row_ids + row) : 0;
 #pragma unroll
                 for (int j = 0; j < 64; j += 2)
-                    if (j < r)
+                    if (j < nc) {
+                        const bool keep = !P.row_ids || (P.ids_col0 + j) / P.ids_r == id;
                         *reinterpret_cast<uint32_t*>(o + j) =
-                            pack_bf16x2(__fmul_rn(P.scale, v[j]), __fmul_rn(P.scale, v[j + 1]));
+                            keep ? pack_bf16x2(__fmul_rn(P.scale, v[j]), __fmul_rn(P.scale, v[j + 1])) : 0u;
+                    }
             } else if (P.mode == kSkinnyOutF32Transposed) {
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (j < r) P.out_f32[static_cast<int64_t>(j) * P.rows + row] = v[j];
+                    if (j < nc) P.out_f32[static_cast<int64_t>(j) * P.out_ld + row] = v[j];
             } else {
-                float4* o = reinterpret_cast<float4*>(P.out_f32 + row * r);
+                float4* o = reinterpret_cast<float4*>(P.out_f32 + row * P.out_ld);
 #pragma unroll
                 for (int j = 0; j < 64; j += 4)
-                    if (j < r) o[j / 4] = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    if (j < nc) o[j / 4] = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
     }
@@ -271,8 +279,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
 size_t skinny_smem_bytes() { return kSmem; }
 
-cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1, const CUtensorMap& b1,
-                          const SkinnyArgs& args, int nproblems, cudaStream_t st, bool pdl) {
+cudaError_t launch_skinny(const SkinnyMaps& maps, const SkinnyArgs& args, int nproblems, cudaStream_t st, bool pdl) {
+    if (nproblems < 1 || nproblems > kSkinnyMaxProblems) return cudaErrorInvalidValue;
     int64_t max_tiles = 0;
     int max_splits = 0;
     for (int p = 0; p < nproblems; ++p) {
@@ -290,7 +298,7 @@ cudaError_t launch_skinny(const CUtensorMap& a0, const CUtensorMap& b0, const CU
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, skinny_gemm, a0, b0, a1, b1, args);
+    return cudaLaunchKernelEx(&cfg, skinny_gemm, maps, args);
 }
 
 cudaError_t skinny_init_device() {

@@ -71,38 +71,39 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// sum_{j < R} sT[j] * B[j] over bf16 operands, fp32 products and sums in
-// order; all loads are issued before the first product.
-template <int R>
-__device__ __forceinline__ float rank_dot(const uint16_t* sT, const uint16_t* b) {
-    uint4 tv[R / 8], bv[R / 8];
-#pragma unroll
-    for (int i = 0; i < R / 8; ++i) {
-        tv[i] = __ldg(reinterpret_cast<const uint4*>(sT) + i);
-        bv[i] = __ldg(reinterpret_cast<const uint4*>(b) + i);
-    }
+// sum_{j < cols} sT[j] * B[j] over bf16 operands, fp32 products and sums in
+// order (cols a multiple of 8, both rows 16-byte aligned); the loads of each
+// 32 columns are issued before their first product.
+__device__ __forceinline__ float rank_dot(const uint16_t* sT, const uint16_t* b, int cols) {
     float acc = 0.0f;
+    for (int c0 = 0; c0 < cols; c0 += 32) {
+        uint4 tv[4], bv[4];
 #pragma unroll
-    for (int i = 0; i < R / 8; ++i) {
-        const uint32_t tw[4] = {tv[i].x, tv[i].y, tv[i].z, tv[i].w};
-        const uint32_t bw[4] = {bv[i].x, bv[i].y, bv[i].z, bv[i].w};
+        for (int i = 0; i < 4; ++i) {
+            const bool in = c0 + 8 * i < cols;
+            tv[i] = in ? __ldg(reinterpret_cast<const uint4*>(sT + c0) + i) : make_uint4(0u, 0u, 0u, 0u);
+            bv[i] = in ? __ldg(reinterpret_cast<const uint4*>(b + c0) + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            acc = __fmaf_rn(__uint_as_float(tw[j] << 16), __uint_as_float(bw[j] << 16), acc);
-            acc = __fmaf_rn(__uint_as_float(tw[j] & 0xFFFF0000u), __uint_as_float(bw[j] & 0xFFFF0000u), acc);
+        for (int i = 0; i < 4; ++i) {
+            if (c0 + 8 * i >= cols) break;
+            const uint32_t tw[4] = {tv[i].x, tv[i].y, tv[i].z, tv[i].w};
+            const uint32_t bw[4] = {bv[i].x, bv[i].y, bv[i].z, bv[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc = __fmaf_rn(__uint_as_float(tw[j] << 16), __uint_as_float(bw[j] << 16), acc);
+                acc = __fmaf_rn(__uint_as_float(tw[j] & 0xFFFF0000u), __uint_as_float(bw[j] & 0xFFFF0000u), acc);
+            }
         }
     }
     return acc;
 }
 
-// r is one of 8, 16, 32, 64 (checked on the host); rows are 16-byte aligned
-__device__ __forceinline__ float rank_dot_r(const uint16_t* sT, const uint16_t* b, int r) {
-    switch (r) {
-        case 8: return rank_dot<8>(sT, b);
-        case 16: return rank_dot<16>(sT, b);
-        case 32: return rank_dot<32>(sT, b);
-        default: return rank_dot<64>(sT, b);
-    }
+// Column of sT holding the rank-r input of output row n.
+__device__ __forceinline__ int rank_col(const GemvMmaArgs& a, int64_t n) {
+    for (int g = 0; g < a.ngroups - 1; ++g)
+        if (n < a.group_end[g]) return a.group_rank_x[g];
+    return a.group_rank_x[a.ngroups - 1];
 }
 
 // The weight stream goes through a per-lane ring of kStages step slots in
@@ -308,7 +309,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
         }
     }
     __syncthreads();
-    const int r = a.r;
     for (int j = 0; j < nseg; ++j) {
         if (!last_of[j]) continue;
         __threadfence();  // see the other CTAs' partials
@@ -321,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
             if (n >= N) continue;
             // every load of this output goes out before the first use: the
             // rank-r operands, then the partials in CTA order, 16 at a time
-            const float lr = rank_dot_r(a.sT + m * r, a.B + static_cast<int64_t>(n) * r, r);
+            const float lr = rank_dot(a.sT + static_cast<int64_t>(m) * a.sT_ld + rank_col(a, n),
+                                      a.B + static_cast<int64_t>(n) * a.B_ld, a.rank_cols);
             float s = 0.0f;
             for (int s0 = 0; s0 < np; s0 += 16) {
                 float v[16];

@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(256) decode_constants_t_kernel(const uint8_t* 
                                                                   const float* __restrict__ s2,
                                                                   const float* __restrict__ mean,
                                                                   const float* __restrict__ absmax, int64_t N,
-                                                                  int64_t KB, int64_t ldc,
+                                                                  int64_t KB, int64_t ldc, int64_t cols,
                                                                   float* __restrict__ cT) {
     __shared__ float tile[32][33];
     const float mu = kNoDq ? 0.0f : *mean;
@@ -368,8 +368,21 @@ __global__ void __launch_bounds__(256) decode_constants_t_kernel(const uint8_t* 
     __syncthreads();
     for (int i = ty; i < 32; i += 8) {
         const int64_t kb = kb0 + i, n = n0 + tx;
-        if (kb < KB && n < ldc) cT[kb * ldc + n] = (n < N) ? tile[tx][i] : 0.0f;
+        if (kb < KB && n < cols) cT[kb * ldc + n] = (n < N) ? tile[tx][i] : 0.0f;
     }
+}
+
+// c'_b of every block, in block order (fp32 [nb]).
+template <bool kNoDq>
+__global__ void __launch_bounds__(256) decode_constants_kernel(const uint8_t* __restrict__ q,
+                                                                const float* __restrict__ s2,
+                                                                const float* __restrict__ mean,
+                                                                const float* __restrict__ absmax, int64_t nb,
+                                                                float* __restrict__ c) {
+    const float mu = kNoDq ? 0.0f : *mean;
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nb;
+         b += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        c[b] = kNoDq ? absmax[b] : decode_constant(q, s2, mu, b);
 }
 
 // Test hook: the double quantisation's E4M3 conversion on arbitrary floats.
@@ -455,14 +468,24 @@ cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes,
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_constants_t(const BlockConstants& c, int64_t N, int64_t K, int64_t ldc, float* cT,
-                                      cudaStream_t st) {
+cudaError_t launch_decode_constants_t(const BlockConstants& c, int64_t N, int64_t K, int64_t ldc, int64_t cols,
+                                      float* cT, cudaStream_t st) {
     const int64_t KB = K / kBlock;
-    dim3 grid(static_cast<unsigned>((KB + 31) / 32), static_cast<unsigned>((ldc + 31) / 32));
+    dim3 grid(static_cast<unsigned>((KB + 31) / 32), static_cast<unsigned>((cols + 31) / 32));
     if (c.absmax)
-        decode_constants_t_kernel<true><<<grid, 256, 0, st>>>(nullptr, nullptr, nullptr, c.absmax, N, KB, ldc, cT);
+        decode_constants_t_kernel<true><<<grid, 256, 0, st>>>(nullptr, nullptr, nullptr, c.absmax, N, KB, ldc, cols, cT);
     else
-        decode_constants_t_kernel<false><<<grid, 256, 0, st>>>(c.qabsmax, c.s2, c.mean, nullptr, N, KB, ldc, cT);
+        decode_constants_t_kernel<false><<<grid, 256, 0, st>>>(c.qabsmax, c.s2, c.mean, nullptr, N, KB, ldc, cols,
+                                                               cT);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_constants(const BlockConstants& c, int64_t nb, float* out, int num_sms, cudaStream_t st) {
+    const int grid = grid_for(nb, 256, 8 * num_sms);
+    if (c.absmax)
+        decode_constants_kernel<true><<<grid, 256, 0, st>>>(nullptr, nullptr, nullptr, c.absmax, nb, out);
+    else
+        decode_constants_kernel<false><<<grid, 256, 0, st>>>(c.qabsmax, c.s2, c.mean, nullptr, nb, out);
     return cudaGetLastError();
 }
 

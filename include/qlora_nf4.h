@@ -209,6 +209,69 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M,
                               uint16_t* dX, float* dA, float* dB,
                               void* ws, size_t ws_bytes, void* stream);
 
+/* Several adapters over one frozen base in one call ["waylandz LLM book
+ * ch.26", 26.7.3: one base model hosts many adapters and switches between
+ * them at run time; "agentlenshq" summary, 利用ケース: one 4-bit base serves
+ * several adapters]. Token row m uses adapter k = ids[m]:
+ *   Y[m] = X[m] deq(W)^T + (alpha/r) (X[m] A_k^T) B_k^T.
+ * P adapters of one rank r in {8, 16, 32, 64}, P r <= 256; all share alpha.
+ *   A:   bf16 [P r, K], adapter k in rows [k r, (k + 1) r) (the A_k stacked)
+ *   B:   bf16 [N, P r], adapter k in columns [k r, (k + 1) r) (the B_k side by side)
+ *   ids: int32 [M] (device, 4-byte aligned); a row whose id is outside
+ *        [0, P) uses no adapter (the frozen base layer only).
+ * The rank-r inputs are those of a layer of rank P r whose columns other
+ * than the row's own adapter are zero: sT_save (bf16 [M, P r], may be NULL)
+ * holds s X A_k^T in the row's own columns and zeros elsewhere. The
+ * backward returns every adapter's gradients at once, each from the rows
+ * that use it (an adapter no row uses gets exactly zero):
+ *   dA: fp32 [P r, K] (dA_k in rows [k r, (k + 1) r)), dB: fp32 [N, P r].
+ * sT: the forward's sT_save, or NULL to recompute it. The workspace size
+ * comes from qlora_workspace_bytes_multi (same op codes, P adapters of rank
+ * r). Errors, asynchrony and ownership as for qlora_linear_fwd/bwd; ids is
+ * read on the device only. */
+size_t qlora_workspace_bytes_multi(int op, int64_t M, int64_t N, int64_t K, int r, int P);
+qlora_status qlora_linear_fwd_multi(const uint16_t* X, int64_t M, const qlora_nf4_weight* w,
+                                    const uint16_t* A, const uint16_t* B, int r, int P,
+                                    const int32_t* ids, float alpha, uint16_t* Y, uint16_t* sT_save,
+                                    void* ws, size_t ws_bytes, void* stream);
+qlora_status qlora_linear_bwd_multi(const uint16_t* dY, const uint16_t* X, int64_t M,
+                                    const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
+                                    int r, int P, const int32_t* ids, float alpha, const uint16_t* sT,
+                                    uint16_t* dX, float* dA, float* dB,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* Projections that share one input, each with its own frozen NF4 weight and
+ * adapter, in one call: q, k, v of attention or gate and up of the MLP
+ * ["ta-paperlens QLoRA explainer", コードで見る: target_modules names every
+ * linear layer; 落とし穴: adapters on attention alone leave a gap].
+ * w[0..P-1] (1 <= P <= 4): weights N_i x K, all with the same K and the same
+ * storage (all with or all without double quantisation), each quantised on
+ * its own (its own mean and s2), and with their codes back to back in one
+ * buffer: w[i+1].codes == w[i].codes + N_i K / 2 (quantise each into its
+ * slice of one allocation). N = sum N_i.
+ *   A:  bf16 [P r, K], projection i's A_i in rows [i r, (i + 1) r)
+ *   B:  bf16 [N, r], the B_i [N_i, r] stacked (projection i in rows
+ *       [n_i, n_i + N_i), n_i = N_0 + ... + N_{i-1})
+ *   Y:  bf16 [M, N] = [Y_0 | Y_1 | ...], Y_i = X deq(W_i)^T + (alpha/r) (X A_i^T) B_i^T
+ *   sT_save: bf16 [M, P r] = [s X A_0^T | s X A_1^T | ...] (may be NULL)
+ * Backward, with dY bf16 [M, N] = [dY_0 | dY_1 | ...]:
+ *   dX = sum_i (dY_i deq(W_i) + (alpha/r) (dY_i B_i) A_i)   bf16 [M, K]
+ *   dA: fp32 [P r, K] (dA_i in rows [i r, (i + 1) r))
+ *   dB: fp32 [N, r]   (dB_i in rows [n_i, n_i + N_i))
+ * r in {8, 16, 32, 64}. The workspace size comes from
+ * qlora_workspace_bytes_group (N: host array of the P row counts). Errors,
+ * asynchrony and ownership as for qlora_linear_fwd/bwd. */
+size_t qlora_workspace_bytes_group(int op, int64_t M, const int64_t* N, int P, int64_t K, int r);
+qlora_status qlora_linear_fwd_group(const uint16_t* X, int64_t M, const qlora_nf4_weight* w, int P,
+                                    const uint16_t* A, const uint16_t* B, int r, float alpha,
+                                    uint16_t* Y, uint16_t* sT_save,
+                                    void* ws, size_t ws_bytes, void* stream);
+qlora_status qlora_linear_bwd_group(const uint16_t* dY, const uint16_t* X, int64_t M,
+                                    const qlora_nf4_weight* w, int P, const uint16_t* A,
+                                    const uint16_t* B, int r, float alpha, const uint16_t* sT,
+                                    uint16_t* dX, float* dA, float* dB,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* Host copies of the library's own NF4 tables: levels[16] (fp32, ascending)
  * and thresholds[15] (the fp32 decision points between neighbouring levels).
  * Computed on the host at load time, independently of any test code. */

@@ -18,3 +18,19 @@ def golden():
     import json
     with open(os.path.join(ROOT, "tests", "golden", "page_numbers.json")) as f:
         return json.load(f)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_checked(request):
+    """GPU tests run with the binding reading back the device status word
+    after every forward and backward call: a bounded wait that ran out
+    inside a kernel (leaving a tile unwritten) turns the test red."""
+    if request.node.get_closest_marker("gpu") is None:
+        yield
+        return
+    import bit_nf4_quantized_09_b200 as q
+    q.set_check_device_status(True)
+    try:
+        yield
+    finally:
+        q.set_check_device_status(True)

@@ -201,3 +201,74 @@ def test_missing_library_fails_loudly():
             "    print('raised', 'no CPU fallback' in str(e))\n")
     out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert out.stdout.strip() == "raised True", out.stdout + out.stderr
+
+
+def test_host_validation_several_adapters(q):
+    """qlora_linear_{fwd,bwd}_multi: P adapters of rank r (P r <= 256) and a
+    per-row id array, checked on the host before any CUDA call."""
+    L = q.lib()
+    w = _weight(q)
+    P = 0x7000000
+    ws = q.workspace_bytes_multi(q.OP_FWD, 64, 512, 512, 16, 3)
+    assert ws > 0
+    assert q.workspace_bytes_multi(q.OP_FWD, 64, 512, 512, 16, 17) == 0   # P r > 256
+    assert q.workspace_bytes_multi(q.OP_FWD, 64, 512, 512, 12, 2) == 0    # rank
+    assert q.workspace_bytes_multi(q.OP_BWD, 64, 512, 512, 64, 4) > q.workspace_bytes(q.OP_BWD, 64, 512, 512, 64)
+
+    def fwd(**kw):
+        return L.qlora_linear_fwd_multi(P, kw.get("M", 64), ctypes.byref(w), P, P, kw.get("r", 16), kw.get("P", 3),
+                                        kw.get("ids", P), 16.0, P, None, P, kw.get("wsb", ws), None)
+    assert fwd(P=0) == -1
+    assert fwd(P=17) == -4
+    assert fwd(r=24) == -4
+    assert fwd(ids=None) == -1
+    assert fwd(ids=P + 2) == -3
+    assert fwd(M=0, ids=None) == 0
+    assert fwd(wsb=ws - 1) == -5
+    bws = q.workspace_bytes_multi(q.OP_BWD, 64, 512, 512, 16, 3)
+
+    def bwd(**kw):
+        return L.qlora_linear_bwd_multi(P, P, 64, ctypes.byref(w), P, P, 16, kw.get("P", 3), kw.get("ids", P), 16.0,
+                                        None, P, P, P, P, kw.get("wsb", bws), None)
+    assert bwd(ids=None) == -1
+    assert bwd(P=20) == -4
+    assert bwd(wsb=bws - 256) == -5
+
+
+def test_host_validation_projection_group(q):
+    """qlora_linear_{fwd,bwd}_group: up to four weights with one K and one
+    storage form whose codes lie back to back in one buffer."""
+    L = q.lib()
+    P = 0x7000000
+    K = 512
+
+    def group(Ns, gap=0, Ks=None, nodq=()):
+        arr = (q.Nf4WeightC * len(Ns))()
+        at = P
+        for i, n in enumerate(Ns):
+            k = Ks[i] if Ks else K
+            arr[i] = q.Nf4WeightC(at, P + 0x1000000 * (i + 1), P + 0x1100000 * (i + 1), P + 0x1200000 * (i + 1), n, k,
+                                  P + 0x1300000 * (i + 1) if i in nodq else None)
+            at += n * k // 2 + gap
+        return arr
+    Ns = [512, 256, 264]
+    n_arr = (ctypes.c_int64 * 3)(*Ns)
+    ws = L.qlora_workspace_bytes_group(q.OP_FWD, 64, n_arr, 3, K, 16)
+    assert ws > 0
+    assert L.qlora_workspace_bytes_group(q.OP_FWD, 64, n_arr, 5, K, 16) == 0
+    assert L.qlora_workspace_bytes_group(q.OP_FWD, 64, n_arr, 3, K, 12) == 0
+
+    def fwd(arr, nw=3, wsb=ws):
+        return L.qlora_linear_fwd_group(P, 64, arr, nw, P, P, 16, 16.0, P, None, P, wsb, None)
+    assert fwd(group(Ns), wsb=ws - 1) == -5
+    assert fwd(group(Ns, gap=16)) == -1                       # codes not back to back
+    assert b"back to back" in L.qlora_last_error()
+    assert fwd(group(Ns, Ks=[512, 512, 448])) == -2           # K differs
+    assert fwd(group(Ns, nodq=(1,))) == -1                    # storage differs
+    assert fwd(group([512, 256, 12])) == -2                   # N % 8
+    assert fwd(group(Ns), nw=0) == -1
+    assert fwd(group(Ns + [256, 256]), nw=5) == -1            # at most four projections
+    bws = L.qlora_workspace_bytes_group(q.OP_BWD, 64, n_arr, 3, K, 16)
+    assert L.qlora_linear_bwd_group(P, P, 64, group(Ns, gap=16), 3, P, P, 16, 16.0, None, P, P, P, P, bws,
+                                    None) == -1
+    assert L.qlora_linear_bwd_group(P, P, 64, group(Ns), 3, P, P, 16, 16.0, None, P, None, P, P, bws, None) == -1

@@ -78,3 +78,20 @@ def test_largest_accepted_size_and_rejection(q):
     assert q.lib().qlora_status_string(rc) == b"QLORA_ERR_EXCEEDS_STATIC_SCRATCH"
     assert q.launch_count() == n0
     assert np.isfinite(q.dequantize_nf4(without_allocation(q, W)).float().cpu().numpy()).all()
+
+
+def test_python_wrapper_checks_its_outputs(q):
+    """The torch wrapper of the same entry point: it matches the workspace
+    entry point, and refuses an output sized for another shape before any
+    launch (an undersized output would be written past its end)."""
+    W = synth.weight(synth.custom(N=520, K=320, M=1, r=8, seed_base=94)).cuda()
+    out = q.NF4Weight.empty(520, 320, W.device)
+    same(q.quantize_nf4_noalloc(W, out), with_workspace(q, W))
+    torch.cuda.synchronize()
+    n0 = q.launch_count()
+    with pytest.raises(AssertionError):
+        q.quantize_nf4_noalloc(W, q.NF4Weight.empty(512, 320, W.device))
+    strided = torch.empty(520, 640, dtype=torch.float32, device=W.device)[:, :320]   # not contiguous
+    with pytest.raises(AssertionError):
+        q.quantize_nf4_noalloc(strided, q.NF4Weight.empty(520, 320, W.device))
+    assert q.launch_count() == n0
