@@ -25,7 +25,6 @@ std::atomic<int64_t> g_timeout_us{1000000};
 std::atomic<int64_t> g_stall_producer{0};
 std::atomic<int64_t> g_launch_count{0};
 std::atomic<int64_t> g_skinny_max_splits{0};
-std::atomic<int64_t> g_reg_gemv_max_m{16};
 thread_local std::string g_last_error;
 
 // One-shot event requests of qlora_profile_next_launch, per kernel id.
@@ -157,7 +156,7 @@ qlora_status device_ready(int* sms_out) {
                            std::to_string(minor) + ")";
             d.status = QLORA_ERR_UNSUPPORTED_DEVICE;
         } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess ||
-                   (e = gemv_init_device()) != cudaSuccess || (e = gemv_mma_init_device()) != cudaSuccess) {
+                   (e = gemv_mma_init_device()) != cudaSuccess) {
             d.status = cuda_fail(e, "cudaFuncSetAttribute");
         } else if (!g_encode) {
             void* fn = nullptr;
@@ -253,27 +252,6 @@ Split split_for(int64_t tiles, int64_t red) {
     return Split{static_cast<int>(s), static_cast<int>(steps)};
 }
 
-// K splits of the small-batch kernel: at most two waves of three CTAs per SM
-// (on 148 SMs), the best wave fill, and fp32 partials no larger than a
-// quarter of the packed weight.
-Split gemv_split(int64_t M, int64_t N, int64_t K) {
-    const int64_t KT = K / 64, tiles = cdiv(N, 128), slots = 3 * 148;
-    const int64_t smax = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(KT, 64), K / (32 * std::max<int64_t>(M, 1))));
-    int64_t best = 1;
-    double best_eff = -1.0;
-    for (int64_t s = 1; s <= smax; ++s) {
-        const int64_t units = tiles * s;
-        if (s > 1 && units > 2 * slots) break;
-        const double eff = static_cast<double>(units) / static_cast<double>(cdiv(units, slots) * slots);
-        if (eff > best_eff + 1e-9) {
-            best = s;
-            best_eff = eff;
-        }
-    }
-    const int64_t steps = cdiv(KT, best);
-    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
-}
-
 // ------------------------------------------------------- the low-rank side --
 // The adapter side of a forward or backward call. One adapter (P = 1);
 // several adapters over one frozen base, each token row using the one its id
@@ -320,8 +298,8 @@ struct Layout {
     size_t partU = 0, sU = 0, partA = 0;                  // backward (partA holds dA and dB partials)
     size_t total = 0;
     int64_t ldc = 0;
-    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1}, gemv{1, 1};
-    GemvMmaPlan reg_gemv{1, 1, 4, 1};
+    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1};
+    GemvMmaPlan reg_gemv{1, 1, 2, 1};
 };
 
 // UMMA N of a rank-r problem of `w` columns (at most 64).
@@ -370,15 +348,10 @@ Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
     const size_t partT_bytes = static_cast<size_t>(nch) * L.sT_split.splits * M * NRc * 4;
     if (fwd) {
         L.partT = take(partT_bytes);
-        if (M <= kGemvMaxM) {
-            // either small-batch kernel may run (the choice is a runtime option)
-            L.gemv = gemv_split(M, N, K);
-            size_t part = static_cast<size_t>(L.gemv.splits) * M * N * 4;
-            if (M <= kGemvMmaMaxM) {
-                L.reg_gemv = gemv_mma_plan(M, N, K, kPlanSms);
-                part = std::max(part, static_cast<size_t>(L.reg_gemv.max_parts) * M * N * 4);
-            }
-            L.partY = take(part);
+        if (M <= kGemvMmaMaxM) {
+            // the small-batch kernel may run (its token limit is a runtime option)
+            L.reg_gemv = gemv_mma_plan(M, N, K, kPlanSms);
+            L.partY = take(static_cast<size_t>(L.reg_gemv.max_parts) * M * N * 4);
             // a group's block constants decoded in block order for the
             // register-fed kernel (its weights keep their own mean and s2)
             if (lo.group) L.cflat = take(static_cast<size_t>(N * K / kBlock) * 4);
@@ -643,15 +616,13 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
     float* partT = reinterpret_cast<float*>(base + L.partT);
     uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
     const float scale = alpha / static_cast<float>(r);
-    const bool plain = lo.P == 1 && !lo.group;
 
     QLORA_TRY(cudaMemsetAsync(base, 0, L.header, st), "clear status and tickets");
     if (injected_failure()) return QLORA_ERR_CUDA;
-    const int64_t small = std::min<int64_t>(g_small_m_max.load(), kGemvMaxM);
-    if (M <= small && M <= std::min<int64_t>(g_reg_gemv_max_m.load(), kGemvMmaMaxM)) {
-        // few tokens: rank-r down-projection, then the register-fed GEMV,
-        // launched as its programmatic dependent so the weight stream starts
-        // while sT is still being computed
+    if (M <= std::min<int64_t>(g_small_m_max.load(), kGemvMmaMaxM)) {
+        // few tokens: rank-r down-projection, then the weight-streaming
+        // small-batch kernel, launched as its programmatic dependent so the
+        // weight stream starts while sT is still being computed
         const float* cflat = nullptr;
         if (lo.group) {
             // each weight's block constants, decoded into one array in block order
@@ -664,9 +635,12 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
         if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
                           st)) != QLORA_OK)
             return s;
+        CUtensorMap t_codes, t_x;
+        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 128, 256,
+                  CU_TENSOR_MAP_SWIZZLE_128B, "codes");
+        QLORA_MAP(&t_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, static_cast<uint32_t>(M),
+                  CU_TENSOR_MAP_SWIZZLE_128B, "X");
         GemvMmaArgs ga{};
-        ga.X = X;
-        ga.codes = W.w[0].codes;
         ga.qabsmax = W.w[0].qabsmax;
         ga.s2 = W.w[0].s2;
         ga.mean = W.w[0].mean;
@@ -684,44 +658,7 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
         }
         ga.ctas = L.reg_gemv.ctas;
         ga.units = L.reg_gemv.units;
-        ga.max_chunks = L.reg_gemv.max_chunks;
-        ga.part = reinterpret_cast<float*>(base + L.partY);
-        ga.counter = reinterpret_cast<int*>(base + L.ctrY);
-        ga.sT = sT;
-        ga.B = B;
-        ga.Y = Y;
-        if (injected_failure()) return QLORA_ERR_CUDA;
-        cudaEvent_t ev0, ev1;
-        take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
-        if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-        // an event record between the two launches would break the
-        // programmatic edge, so a profiled call launches in plain order
-        QLORA_LAUNCH(launch_gemv_mma(ga, tables(), ev0 == nullptr, st), 1, "register gemv");
-        if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
-        return QLORA_OK;
-    }
-    if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
-    if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
-                      st)) != QLORA_OK)
-        return s;
-
-    if (M <= small && plain) {
-        // few tokens: weight-streaming swap-AB kernel, split over K
-        const int Mp = static_cast<int>((M + 15) / 16 * 16);
-        CUtensorMap t_x, t_codes, t_c;
-        QLORA_MAP(&t_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, Mp, CU_TENSOR_MAP_SWIZZLE_128B, "X");
-        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 128,
-                  CU_TENSOR_MAP_SWIZZLE_32B, "codes");
-        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
-        GemvArgs ga{};
-        ga.M = M;
-        ga.N = N;
-        ga.K = K;
-        ga.Mp = Mp;
-        ga.r = r;
-        ga.splits = L.gemv.splits;
-        ga.steps_per_split = L.gemv.steps;
+        ga.stages = L.reg_gemv.stages;
         ga.part = reinterpret_cast<float*>(base + L.partY);
         ga.counter = reinterpret_cast<int*>(base + L.ctrY);
         ga.sT = sT;
@@ -733,10 +670,16 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
         cudaEvent_t ev0, ev1;
         take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
         if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-        QLORA_LAUNCH(launch_gemv(t_x, t_codes, t_c, ga, tables(), st), 1, "gemv");
+        // an event record between the two launches would break the
+        // programmatic edge, so a profiled call launches in plain order
+        QLORA_LAUNCH(launch_gemv_mma(t_codes, t_x, ga, tables(), ev0 == nullptr, st), 1, "register gemv");
         if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
         return QLORA_OK;
     }
+    if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
+    if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
+                      st)) != QLORA_OK)
+        return s;
 
     CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
     QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");
@@ -979,7 +922,6 @@ qlora_status qlora_set_option(int option, int64_t value) {
             if (value < 0) return QLORA_ERR_INVALID_ARG;
             g_skinny_max_splits = value;
             return QLORA_OK;
-        case QLORA_OPT_REG_GEMV_MAX_M: g_reg_gemv_max_m = value; return QLORA_OK;
         default: return QLORA_ERR_INVALID_ARG;
     }
 }
@@ -992,7 +934,6 @@ int64_t qlora_get_option(int option) {
         case QLORA_OPT_STALL_PRODUCER: return g_stall_producer.load();
         case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
         case QLORA_OPT_SKINNY_MAX_SPLITS: return g_skinny_max_splits.load();
-        case QLORA_OPT_REG_GEMV_MAX_M: return g_reg_gemv_max_m.load();
         default: return -1;
     }
 }

@@ -1,30 +1,57 @@
-// Small-batch forward for up to 32 tokens: Y = X . deq(W)^T + sT . B^T.
+// Small-batch forward for up to 64 tokens: Y = X . deq(W)^T + sT . B^T.
 //
 // With a few tokens every weight is used a few times only, so the step is
-// bound by streaming the packed weight (about half a byte per weight) and by
-// decoding it; "ta-paperlens QLoRA explainer", 落とし穴, names this
-// small-batch regime as the one where 4-bit weights pay off.
+// bound by streaming the packed weight (about half a byte per weight);
+// "ta-paperlens QLoRA explainer", 落とし穴, names this small-batch regime as
+// the one where 4-bit weights pay off. The kernel is shaped so that the
+// decode and its bookkeeping cost fewer instructions than the stream allows:
+// per two weights one byte permute, one integer multiply-add and one
+// shared-memory load.
 //
-// Design: no shared-memory staging of the weight at all. Each warp owns 16
-// weight rows and walks K in steps of four NF4 blocks (256 weights per row).
-// Lane (g, q) loads the 32 packed bytes of block q of rows g and g + 8 with
-// 16-byte global loads one step ahead, builds the two per-block bf16 lookup
-// tables, decodes straight into the A fragments of mma.m16n8k16 (weight rows
-// = MMA rows) and multiplies them with X fragments read from shared memory
-// (tokens = MMA columns, n8 tiles). The reduction index inside an MMA is
-// permuted: lane q's slots 2q, 2q + 1, 2q + 8, 2q + 9 of MMA step s hold
-// weights 4s .. 4s + 3 of its block, and the X fragment uses the same order,
-// so no data is moved between lanes.
+// Factored dequantisation. Within a 64-weight block every weight is
+// level[code] * c'_b, so for output row n
+//   Y[m, n] = sum_b c'_{n,b} * sum_{k in b} level[code_{n,k}] * X[m, k].
+// The inner sums run on the tensor core (mma.m16n8k16, bf16 operands, fp32
+// accumulation) over the unscaled levels rounded to bf16, one block at a time
+// into a zeroed fragment; c'_{n,b} (fp32) is applied with one FMA per
+// accumulator per block. The weight the product sees is bf16(level) * c', not
+// the exactly dequantised bf16(level * c'): at most 2^-8 relative apart per
+// weight, far inside the forward's tolerance.
 //
-// CTA = 8 warps = 128 weight rows. The (row tile, block column) units are
-// dealt out in equal contiguous ranges, one per CTA slot (stream-K), so no
-// wave is left part-empty; a range may cross into the next row tile. Every
-// CTA that touches a tile writes its fp32 partial sums for it; the last one
-// to finish (atomic ticket) adds them in CTA order, adds the rank-r term and
-// writes Y in bf16. The rank-r input sT comes from the preceding launch;
-// the kernel may be launched as its programmatic dependent and waits for it
-// (griddepcontrol.wait) only before the epilogue, so the weight stream
-// overlaps the down-projection.
+// Decoding. A code byte holds two consecutive weights (the first in the high
+// nibble), so one 256-entry table of bf16 pairs turns a byte into the 32-bit
+// operand register of two weights. The table lives in shared memory with one
+// copy per lane (entry e of lane l at word 32 e + l): every lookup of a warp
+// hits 32 distinct banks.
+//
+// Data movement. A producer warp stages, per pipeline step of four block
+// columns, the packed codes of the CTA's 256 weight rows (one 128 x 256-byte
+// TMA box: 128 contiguous bytes of every row, so each DRAM access is a whole
+// line; 128-byte swizzle) and the matching X columns of every token (one
+// 64 x M box per block column, 128-byte swizzle) into a ring of stages guarded by
+// mbarriers; every wait is bounded. Four producer warps take the steps in
+// turn: each issues its step's copies and decodes the step's block constants
+// c' (E4M3 code, second-level scale and mean, or the fp32 constant; every
+// load issued before the first use) into the stage, so four steps' load
+// latencies overlap and a consumer reads the four constants of a row with
+// one 16-byte load.
+//
+// Fragment layout. Lane (g, q) of a consumer warp that owns 16 weight rows
+// reads the 8 code bytes 8q .. 8q + 7 of rows g and g + 8 of each block.
+// Inside MMA step s (0..3) of a block its A-operand slots 2q, 2q + 1 hold
+// weights 16q + 4s, +1 (code byte 8q + 2s) and slots 2q + 8, 2q + 9 hold
+// weights 16q + 4s + 2, +3 (byte 8q + 2s + 1); its X fragment uses the same
+// order, X[m][16q .. 16q + 15] of the block (two swizzled 16-byte chunks).
+//
+// Work split. A CTA of 16 consumer warps owns 256 weight rows; the (row tile,
+// block column) units are dealt out in equal contiguous ranges, one per CTA,
+// one CTA per SM (stream-K), so no wave is left part-empty; a range may cross
+// into the next row tile. Every CTA that touches a tile writes its fp32
+// partial sums for it; the last one to finish (atomic ticket, no waiting)
+// adds them in CTA order, adds the rank-r term and writes Y in bf16. The
+// rank-r input sT comes from the preceding launch; the kernel may be launched
+// as its programmatic dependent and waits for it (griddepcontrol.wait) only
+// in that epilogue, so the weight stream overlaps the down-projection.
 #include <algorithm>
 
 #include "common.cuh"
@@ -34,29 +61,21 @@ namespace qlora {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kRowsCta = kWarps * 16;
-constexpr uint32_t kChunk = 144;  // bytes per 64 X elements in shared memory (128 + 16 pad)
+constexpr int kWarps = 16;                    // consumer warps
+constexpr int kProdWarps = 4;                 // producer warps: TMA (one lane) and the block constants
+constexpr int kThreads = (kWarps + kProdWarps) * 32;
+constexpr int kRowsCta = kWarps * 16;         // 256 weight rows
+constexpr int kStep = 4;                      // block columns per pipeline step
+constexpr int kMaxStages = 6;
+constexpr uint32_t kLutBytes = 256 * 32 * 4;  // 256 entries x 32 lane copies
+constexpr uint32_t kCodeStage = 32 * kStep * kRowsCta;  // 128 contiguous bytes of each of the 256 rows
 
-// Row pitch of the staged X slice: 144-byte chunks and a pitch congruent to
-// 64 mod 128 bytes, so the 16-byte fragment reads of a quarter warp (2 token
-// rows x 4 lanes q) fall on 8 distinct groups of 4 banks.
-__host__ __device__ constexpr uint32_t x_pitch(int chunks) {
-    const uint32_t raw = static_cast<uint32_t>(chunks) * kChunk;
-    return (raw + 63u) / 128u * 128u + 64u;
+__host__ __device__ constexpr uint32_t x_box_bytes(int64_t M) {
+    return static_cast<uint32_t>((M * 128 + 1023) / 1024 * 1024);  // 1024-aligned for the 128-byte swizzle
 }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+constexpr uint32_t kConstBytes = kRowsCta * kStep * 4;  // c' of the step: [256 rows][4 blocks] fp32
+__host__ __device__ constexpr uint32_t stage_bytes(int64_t M) {
+    return kCodeStage + kStep * x_box_bytes(M) + kConstBytes;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -65,11 +84,31 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory"); }
+
+// The bf16 pair of code byte k of w, from this lane's copy of the table.
+__device__ __forceinline__ uint32_t lut(uint32_t lane_base, uint32_t w, uint32_t k) {
+    const uint32_t e = __byte_perm(w, 0u, 0x4440u + k);
+    return lds32(lane_base + e * 128u);
+}
 
 // sum_{j < cols} sT[j] * B[j] over bf16 operands, fp32 products and sums in
 // order (cols a multiple of 8, both rows 16-byte aligned); the loads of each
@@ -106,25 +145,6 @@ __device__ __forceinline__ int rank_col(const GemvMmaArgs& a, int64_t n) {
     return a.group_rank_x[a.ngroups - 1];
 }
 
-// The weight stream goes through a per-lane ring of kStages step slots in
-// shared memory, filled by cp.async kStages - 1 steps ahead. A slot holds one
-// step's inputs for lane (g, q): the 32 packed bytes of rows g and g + 8, the
-// aligned words holding their E4M3 constants, and their second-level scales.
-// Only the lane that copies a slot reads it, so a per-thread wait_group is
-// the only synchronisation. 80-byte slots keep the 16-byte reads of eight
-// consecutive lanes on distinct banks.
-constexpr uint32_t kSlot = 80;
-
-// Per instantiation (MT n8 token tiles): ring depth and CTAs per SM. One
-// token tile runs three CTAs per SM with a two-step ring; wider ones two
-// CTAs with a three-step ring (their staged X slice is larger).
-template <int MT>
-struct Cfg {
-    static constexpr int kStages = MT == 1 ? 2 : 3;
-    static constexpr int kCtasPerSm = MT == 1 ? 3 : 2;
-    static constexpr uint32_t kRing = kStages * kSlot * kThreads;  // bytes per CTA
-};
-
 // The work is the list of (row tile, NF4 block column) units in tile-major
 // order, U = tiles * KB; CTA c takes units [c U / P, (c + 1) U / P) (stream-K).
 // With P >= tiles a range touches at most two row tiles: its segments. The
@@ -139,17 +159,34 @@ struct Sched {
     __device__ int parts(int tile) const { return cta_of(min((tile + 1) * KB, U) - 1) - cta_of(tile * KB) + 1; }
 };
 
+// Pipeline step k of a CTA's range: its segment, first block column and the
+// number of its block columns inside the segment (steps never straddle two
+// segments; the last step of a segment may be short).
+struct Step {
+    int seg, col0, nb;
+};
+__device__ __forceinline__ Step step_of(int k, int nst0, int blo0, int len0, int len1) {
+    Step s;
+    s.seg = k >= nst0 ? 1 : 0;
+    const int kk = s.seg ? k - nst0 : k;
+    s.col0 = (s.seg ? 0 : blo0) + kStep * kk;
+    s.nb = min(kStep, (s.seg ? len1 : len0) - kStep * kk);
+    return s;
+}
+
 template <int MT, bool kNoDq>
-__global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
-    gemv_mma_kernel(const GemvMmaArgs a, const Nf4Tables tab) {
-    constexpr int kStages = Cfg<MT>::kStages;
-    constexpr uint32_t kRing = Cfg<MT>::kRing;
-    extern __shared__ __align__(16) uint8_t smem[];
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                    const GemvMmaArgs a, const Nf4Tables tab) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
     __shared__ int last_of[2];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    __shared__ float levels[16];
+    __shared__ volatile int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int M = static_cast<int>(a.M);
     const int N = static_cast<int>(a.N), KB = static_cast<int>(a.K / kBlock);
-    const int64_t K = a.K;
     const Sched sc{static_cast<int>(a.units), static_cast<int>(gridDim.x), KB};
     const int c = blockIdx.x;
     const int u0 = static_cast<int>(static_cast<int64_t>(c) * sc.U / sc.P);
@@ -160,125 +197,133 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
     const int blo0 = u0 - t0 * KB;
     const int len0 = min(u1, (t0 + 1) * KB) - u0;
     const int len1 = u1 - u0 - len0;
-    const int it0 = (len0 + 3) / 4, it_all = it0 + (len1 + 3) / 4;
-    const uint32_t PX = x_pitch(a.max_chunks);
-    const uint32_t ring = smem_u32(smem) + threadIdx.x * kSlot;  // this lane's slot 0
-    const uint32_t xs = smem_u32(smem) + kRing;
+    const int nst0 = (len0 + kStep - 1) / kStep, nst = nst0 + (len1 + kStep - 1) / kStep;
+    const int S = a.stages;
+    const uint32_t xbox = x_box_bytes(M), stage = stage_bytes(M);
+    const uint32_t lut_base = smem_u32(smem);
+    const uint32_t st_base = lut_base + kLutBytes;
+    const uint64_t tmo = a.timeout_ns;
 
-    // This lane's rows and first block column in each segment: unit indices
-    // (row * KB + column) of rows g and g + 8, the last column offset, and the
-    // bit offsets of the E4M3 constants in their aligned words (the same for
-    // every step of a segment, since steps advance by 4 columns). A lane past
-    // its segment's end or past N copies a valid neighbour (clamped row and
-    // column) instead: its X chunk is zero or its output row is dropped, so
-    // nothing it decodes reaches Y (decoded weights are always finite).
-    struct LaneSeg {
-        int64_t ia, ib;
-        int kmax;
-        uint32_t sh;  // byte offset of row g's constant * 8 | (row g + 8's) << 8
-    };
-    auto lane_seg = [&](int j) {
-        const int r0 = (t0 + j) * kRowsCta + warp * 16 + g;
-        LaneSeg ls;
-        const int blo = j ? 0 : blo0;
-        ls.ia = static_cast<int64_t>(min(r0, N - 1)) * KB + blo;
-        ls.ib = static_cast<int64_t>(min(r0 + 8, N - 1)) * KB + blo;
-        ls.kmax = (j ? len1 : len0) - 1;
-        ls.sh = static_cast<uint32_t>((ls.ia + q) & 3) * 8 | static_cast<uint32_t>((ls.ib + q) & 3) * 8 << 8;
-        return ls;
-    };
-    const LaneSeg seg0 = lane_seg(0), seg1 = lane_seg(1);
-
-    // copies of step gi into slot gi % kStages
-    auto issue = [&](int gi) {
-        if (gi < it_all) {
-            const bool s1 = gi >= it0;
-            const int off = min(4 * (gi - (s1 ? it0 : 0)) + q, s1 ? seg1.kmax : seg0.kmax);
-            const int64_t ia = (s1 ? seg1.ia : seg0.ia) + off, ib = (s1 ? seg1.ib : seg0.ib) + off;
-            const uint32_t d = ring + (gi % kStages) * (kSlot * kThreads);
-            cp_async16(d, a.codes + ia * 32);
-            cp_async16(d + 16, a.codes + ia * 32 + 16);
-            cp_async16(d + 32, a.codes + ib * 32);
-            cp_async16(d + 48, a.codes + ib * 32 + 16);
-            if (kNoDq) {  // the two fp32 constants
-                cp_async4(d + 64, a.absmax + ia);
-                cp_async4(d + 68, a.absmax + ib);
-            } else {
-                cp_async4(d + 64, a.qabsmax + (ia & ~int64_t(3)));
-                cp_async4(d + 68, a.qabsmax + (ib & ~int64_t(3)));
-                cp_async4(d + 72, a.s2 + (ia >> 8));
-                cp_async4(d + 76, a.s2 + (ib >> 8));
-            }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full + s, 32);       // one arrive per lane of the step's producer warp
+            mbar_init(empty + s, kWarps);  // one arrive per consumer warp
         }
-        cp_async_commit();  // possibly empty: keeps one group per step
-    };
-    // ---- stage X (its loads go out ahead of the weight stream's): step i's
-    // four 64-column chunks at chunk 4i .. 4i + 3, zeros for columns past a
-    // segment's end
-    for (int i = threadIdx.x; i < M * it_all * 32; i += kThreads) {
-        const int cc = i & 7, ch = (i >> 3) % (4 * it_all), m = (i >> 3) / (4 * it_all);
-        const int seg = ch >= 4 * it0;
-        const int lb = ch - (seg ? 4 * it0 : 0);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (lb < (seg ? len1 : len0))
-            v = __ldg(reinterpret_cast<const uint4*>(a.X + m * K + ((seg ? 0 : blo0) + lb) * kBlock) + cc);
-        const uint32_t at = xs + m * PX + ch * kChunk + cc * 16;
-        sts64(at, v.x, v.y);
-        sts64(at + 8, v.z, v.w);
+        abort_flag = 0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) levels[k] = tab.level[k];
+        fence_mbar_init();
     }
+    __syncthreads();
 
-
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) issue(i);
-
-    const float mean = kNoDq ? 0.0f : __ldg(a.mean);
-    float acc[MT][4];
-#pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
-    // X fragment rows: token g + 8t, clamped to the last token (the MMA
-    // columns past M then hold copies whose sums are never written)
-    uint32_t xtok[MT];
-#pragma unroll
-    for (int t = 0; t < MT; ++t) xtok[t] = kRing + min(g + 8 * t, M - 1) * PX + q * kChunk;
-    __syncthreads();  // X staged
-
-#pragma unroll 1
-    for (int gi = 0; gi < it_all; ++gi) {
-        issue(gi + kStages - 1);
-        cp_async_wait<kStages - 1>();  // this lane's copies of step gi have landed
-        const uint32_t d = ring + (gi % kStages) * (kSlot * kThreads);
-        const uint4 a0 = lds128(d), a1 = lds128(d + 16), b0 = lds128(d + 32), b1 = lds128(d + 48);
-        const uint4 cq = lds128(d + 64);  // q words A, B; s2 A, B (kNoDq: constants A, B)
-        const uint32_t sh = gi >= it0 ? seg1.sh : seg0.sh;
-        const float cpa = kNoDq ? __uint_as_float(cq.x)
-                                : __fmaf_rn(e4m3_to_f32(cq.x >> (sh & 31u)), __uint_as_float(cq.z), mean);
-        const float cpb = kNoDq ? __uint_as_float(cq.y)
-                                : __fmaf_rn(e4m3_to_f32(cq.y >> (sh >> 8)), __uint_as_float(cq.w), mean);
-        const Nf4BlockLut la = make_block_lut(tab.level, cpa);
-        const Nf4BlockLut lb = make_block_lut(tab.level, cpb);
-        const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        const uint8_t* xstep = smem + 4 * gi * kChunk;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            uint32_t oa[4], ob[4];
-            lut_decode8_sx(la, wa[w], oa);
-            lut_decode8_sx(lb, wb[w], ob);
-            // X fragments of MMA steps 2w and 2w + 1: 16 contiguous bytes
-            uint4 bx[MT];
-#pragma unroll
-            for (int t = 0; t < MT; ++t) bx[t] = *reinterpret_cast<const uint4*>(xstep + xtok[t] + 16 * w);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t af[4] = {oa[2 * h], ob[2 * h], oa[2 * h + 1], ob[2 * h + 1]};
-#pragma unroll
-                for (int t = 0; t < MT; ++t) mma_bf16(acc[t], af, h ? bx[t].z : bx[t].x, h ? bx[t].w : bx[t].y);
-            }
+    if (warp >= kWarps) {
+        // ----------------------------------------------------- producers --
+        if (warp == kWarps && lane == 0) {
+            tma_prefetch_desc(&tm_codes);
+            tma_prefetch_desc(&tm_x);
         }
-        if (gi == it0 - 1 || gi == it_all - 1) {
-            // segment done: its partial sums, c0, c1 = (row g, tokens 2q,
-            // 2q + 1) and c2, c3 = (row g + 8, the same tokens)
-            const int tile = t0 + (gi >= it0);
+        const float mean = kNoDq ? 0.0f : __ldg(a.mean);
+        const uint32_t tx = kCodeStage + kStep * static_cast<uint32_t>(M) * 128u;
+        const int pw = warp - kWarps;  // producer warp pw owns steps pw, pw + kProdWarps, ...
+        constexpr int kRowsPerLane = kRowsCta / 32;
+        int last_k = -1;  // this warp's last step whose copies were issued
+        for (int k = pw; k < nst; k += kProdWarps) {
+            const int s = k % S;
+            const uint32_t u = static_cast<uint32_t>(k / S);
+            if (k >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(empty + s, (u - 1) & 1u, tmo, a.status))) {
+                abort_flag = 1;
+                break;
+            }
+            if (abort_flag) break;
+            const Step sp = step_of(k, nst0, blo0, len0, len1);
+            const int row0 = (t0 + sp.seg) * kRowsCta;
+            uint8_t* st = smem + kLutBytes + s * stage;
+            if (lane == 0) {
+                mbar_expect_tx(full + s, tx);
+                // whole steps even past a segment's end: the extra columns are
+                // valid memory or zero-filled past K, and never used
+                tma_load_2d(st, &tm_codes, full + s, sp.col0 * 32, row0);
+#pragma unroll
+                for (int b = 0; b < kStep; ++b)
+                    tma_load_2d(st + kCodeStage + b * xbox, &tm_x, full + s, (sp.col0 + b) * kBlock, 0);
+            }
+            last_k = k;
+            // the step's constants: lane l decodes rows l, l + 32, ... (clamped
+            // to valid rows and columns; unused ones are never read); every
+            // load is issued before the first use
+            float4* cst = reinterpret_cast<float4*>(st + kCodeStage + kStep * xbox);
+            constexpr int kBatch = 4;  // rows whose loads are in flight together
+#pragma unroll 1
+            for (int j0 = 0; j0 < kRowsPerLane; j0 += kBatch) {
+                uint32_t qv[kBatch][kStep];
+                float sv[kBatch][kStep];
+#pragma unroll
+                for (int j = 0; j < kBatch; ++j) {
+                    const int64_t rb = static_cast<int64_t>(min(row0 + lane + 32 * (j0 + j), N - 1)) * KB;
+#pragma unroll
+                    for (int b = 0; b < kStep; ++b) {
+                        const int64_t ib = rb + min(sp.col0 + b, KB - 1);
+                        if (kNoDq) {
+                            sv[j][b] = __ldg(a.absmax + ib);
+                        } else {
+                            qv[j][b] = __ldg(a.qabsmax + ib);
+                            sv[j][b] = __ldg(a.s2 + (ib >> 8));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kBatch; ++j) {
+                    float c4[kStep];
+#pragma unroll
+                    for (int b = 0; b < kStep; ++b)
+                        c4[b] = kNoDq ? sv[j][b] : __fmaf_rn(e4m3_to_f32(qv[j][b]), sv[j][b], mean);
+                    cst[lane + 32 * (j0 + j)] = make_float4(c4[0], c4[1], c4[2], c4[3]);
+                }
+            }
+            mbar_arrive(full + s);  // release this lane's constants (the copies complete the phase)
+        }
+        // make sure no copy of this warp's is still landing in shared memory at exit
+        if (lane == 0)
+            for (int k = last_k; k >= 0 && k > last_k - S; k -= kProdWarps)
+                mbar_wait(full + k % S, static_cast<uint32_t>(k / S) & 1u, tmo, nullptr);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ consumers --
+        const int g = lane >> 2, q = lane & 3;
+        const uint32_t lane_lut = lut_base + 4u * static_cast<uint32_t>(lane);
+        // the table: entry e = bf16(level[e >> 4]) | bf16(level[e & 15]) << 16,
+        // four lane copies per 16-byte store
+        for (int i = threadIdx.x; i < 256 * 8; i += kWarps * 32) {
+            const int e = i >> 3;
+            const uint32_t v = pack_bf16x2(levels[e >> 4], levels[e & 15]);
+            sts128(lut_base + static_cast<uint32_t>(e) * 128u + static_cast<uint32_t>(i & 7) * 16u, v, v, v, v);
+        }
+        consumer_bar();
+
+        float acc[MT][4];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+        // X fragment rows in a stage's box: token g + 8t (clamped to the last
+        // token: the MMA columns past M hold copies whose sums are never
+        // written), chunks 2q and 2q + 1 of its 128-byte row, swizzled
+        uint32_t xoff[MT][2];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            const uint32_t m = static_cast<uint32_t>(min(g + 8 * t, M - 1));
+            xoff[t][0] = m * 128u + (((2u * q) ^ (m & 7u)) << 4);
+            xoff[t][1] = m * 128u + (((2u * q + 1u) ^ (m & 7u)) << 4);
+        }
+        // this lane's code bytes in a stage's box: rows g and g + 8 of the warp
+        // (a row past N is decoded from zero-filled codes and its sums dropped);
+        // the 8 bytes of block b sit in 16-byte chunk 2b + q/2 of the row's 128,
+        // stored at chunk (2b + q/2) ^ (row & 7)
+        const uint32_t crow_sw = static_cast<uint32_t>(g & 7);
+        const uint32_t coff = static_cast<uint32_t>(warp * 16 + g) * 128u + 8u * (q & 1);
+        const uint32_t crow = static_cast<uint32_t>(warp * 16 + g);  // its row of the constants
+        auto flush = [&](int seg) {
+            // segment done: its partial sums, acc[t][0..1] = (row g, tokens
+            // 8t + 2q, +1) and acc[t][2..3] = (row g + 8, the same tokens)
+            const int tile = t0 + seg;
             const int sl = sc.slot(tile, c);
             const int rowA = tile * kRowsCta + warp * 16 + g, rowB = rowA + 8;
 #pragma unroll
@@ -294,14 +339,69 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
                 }
                 acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
             }
+        };
+
+        bool ok = true;
+        for (int k = 0; k < nst && ok; ++k) {
+            const int s = k % S;
+            const uint32_t u = static_cast<uint32_t>(k / S);
+            const Step sp = step_of(k, nst0, blo0, len0, len1);
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(full + s, u & 1u, tmo, a.status));
+            if (!ok) break;
+            const uint32_t stc = st_base + static_cast<uint32_t>(s) * stage;
+            // the step's block constants of rows g and g + 8
+            const uint4 ca4 = lds128(stc + kCodeStage + kStep * xbox + crow * 16u);
+            const uint4 cb4 = lds128(stc + kCodeStage + kStep * xbox + crow * 16u + 128u);
+            const float cA[kStep] = {__uint_as_float(ca4.x), __uint_as_float(ca4.y), __uint_as_float(ca4.z),
+                                     __uint_as_float(ca4.w)};
+            const float cB[kStep] = {__uint_as_float(cb4.x), __uint_as_float(cb4.y), __uint_as_float(cb4.z),
+                                     __uint_as_float(cb4.w)};
+#pragma unroll
+            for (int b = 0; b < kStep; ++b) {
+                if (b >= sp.nb) break;
+                const uint32_t ch = ((2u * b + (q >> 1)) ^ crow_sw) << 4;
+                const uint2 wa = lds64(stc + coff + ch), wb = lds64(stc + coff + ch + 1024u);
+                // A fragments of the block's four MMA steps (unscaled levels)
+                uint32_t af[4][4];
+#pragma unroll
+                for (int st4 = 0; st4 < 4; ++st4) {
+                    const uint32_t xa = st4 < 2 ? wa.x : wa.y, xb = st4 < 2 ? wb.x : wb.y;
+                    const uint32_t kk = (st4 & 1) * 2;
+                    af[st4][0] = lut(lane_lut, xa, kk);
+                    af[st4][1] = lut(lane_lut, xb, kk);
+                    af[st4][2] = lut(lane_lut, xa, kk + 1);
+                    af[st4][3] = lut(lane_lut, xb, kk + 1);
+                }
+                const uint32_t xb0 = stc + kCodeStage + b * xbox;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const uint4 x0 = lds128(xb0 + xoff[t][0]), x1 = lds128(xb0 + xoff[t][1]);
+                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    // two independent two-step chains per block
+                    float t0v[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    mma_bf16(t0v, af[0], xw[0], xw[1]);
+                    mma_bf16(t1v, af[2], xw[4], xw[5]);
+                    mma_bf16(t0v, af[1], xw[2], xw[3]);
+                    mma_bf16(t1v, af[3], xw[6], xw[7]);
+                    acc[t][0] = __fmaf_rn(t0v[0] + t1v[0], cA[b], acc[t][0]);
+                    acc[t][1] = __fmaf_rn(t0v[1] + t1v[1], cA[b], acc[t][1]);
+                    acc[t][2] = __fmaf_rn(t0v[2] + t1v[2], cB[b], acc[t][2]);
+                    acc[t][3] = __fmaf_rn(t0v[3] + t1v[3], cB[b], acc[t][3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);
+            if (k == nst0 - 1) flush(0);
+            else if (k == nst - 1) flush(1);
         }
+        if (!ok) abort_flag = 1;
     }
-    cp_async_wait<0>();
 
     // ---- tickets: the last CTA to finish a row tile reduces it
     const int nseg = len1 > 0 ? 2 : 1;
     __threadfence();  // publish this CTA's partials before taking tickets
     __syncthreads();
+    if (abort_flag) return;  // a wait ran out (status recorded): no tickets, no output
     if (threadIdx.x == 0) {
         for (int j = 0; j < nseg; ++j) {
             const int tile = t0 + j;
@@ -338,87 +438,83 @@ __global__ void __launch_bounds__(kThreads, Cfg<MT>::kCtasPerSm)
     }
 }
 
+// dynamic shared memory of one CTA: the 227 KB per block less room for the
+// kernel's static shared variables
+constexpr size_t kSmemLimit = 226 * 1024;
+
+size_t smem_bytes(int64_t M, int stages) { return kLutBytes + static_cast<size_t>(stages) * stage_bytes(M) + 1024; }
+
 template <int MT, bool kNoDq>
-cudaError_t launch_mt(const GemvMmaArgs& a, const Nf4Tables& tab, size_t smem, bool pdl, cudaStream_t st) {
+cudaError_t launch_mt(const CUtensorMap& codes, const CUtensorMap& x, const GemvMmaArgs& a, const Nf4Tables& tab,
+                      bool pdl, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(a.ctas));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = smem_bytes(a.M, a.stages);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_mma_kernel<MT, kNoDq>, a, tab);
+    return cudaLaunchKernelEx(&cfg, gemv_mma_kernel<MT, kNoDq>, codes, x, a, tab);
 }
 
-constexpr int kMaxMt = 4;
-
-// n8 token tiles of the instantiation that serves M tokens (1, 2 or 4)
-int token_tiles(int64_t M) { return M <= 8 ? 1 : (M <= 16 ? 2 : kMaxMt); }
+// n8 token tiles of the instantiation that serves M tokens
+int token_tiles(int64_t M) { return M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8)); }
 
 }  // namespace
 
-size_t gemv_mma_smem_bytes(int64_t M, int max_chunks) {
-    const uint32_t ring = token_tiles(M) == 1 ? Cfg<1>::kRing : Cfg<2>::kRing;
-    return ring + static_cast<size_t>(M) * x_pitch(max_chunks);
-}
-
 GemvMmaPlan gemv_mma_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
     const int64_t KB = K / kBlock, tiles = (N + kRowsCta - 1) / kRowsCta, U = tiles * KB;
-    const bool one = token_tiles(M) == 1;
-    const int per_sm = one ? Cfg<1>::kCtasPerSm : Cfg<2>::kCtasPerSm;
-    // staged X per CTA: what the SM's 227 KB leave beside the rings
-    const size_t budget = (227 * 1024) / per_sm - 1024 - (one ? Cfg<1>::kRing : Cfg<2>::kRing);
-    const int64_t slots = static_cast<int64_t>(per_sm) * std::max(num_sms, 1);
-    // whole waves of CTA slots, at least one CTA per row tile (so a range
-    // touches at most two tiles), at most one CTA per unit
-    int64_t P = std::min(U, (tiles + slots - 1) / slots * slots);
-    // staged X chunks: the range's blocks plus up to 3 pad blocks per segment
-    auto chunks = [&](int64_t p) { return ((U + p - 1) / p + 6 + 3) / 4 * 4; };
-    while (P < U && static_cast<size_t>(M) * x_pitch(static_cast<int>(chunks(P))) > budget) P = std::min(U, P + slots);
+    const int64_t slots = std::max(num_sms, 1);  // one CTA per SM
+    // whole waves, at least one CTA per row tile (so a range touches at most
+    // two tiles), at most one CTA per unit
+    const int64_t P = std::min(U, (tiles + slots - 1) / slots * slots);
     GemvMmaPlan plan;
     plan.ctas = static_cast<int>(P);
     plan.units = U;
-    plan.max_chunks = static_cast<int>(chunks(P));
+    plan.stages = static_cast<int>(std::min<size_t>(kMaxStages, (kSmemLimit - kLutBytes - 1024) / stage_bytes(M)));
     plan.max_parts = static_cast<int>((KB + U / P - 1) / (U / P) + 1);
     return plan;
 }
 
 namespace {
-template <bool kNoDq>
-cudaError_t gemv_mma_opt_in(int smax) {
-    cudaError_t e;
-    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<1, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) !=
-        cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(gemv_mma_kernel<2, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)) !=
-        cudaSuccess)
-        return e;
-    return cudaFuncSetAttribute(gemv_mma_kernel<4, kNoDq>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
+template <int MT>
+cudaError_t opt_in(int smax) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_mma_kernel<MT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smax);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemv_mma_kernel<MT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
 }
 }  // namespace
 
 cudaError_t gemv_mma_init_device() {
-    const int smax = 220 * 1024;  // above any plan (the plan keeps two or three CTAs per SM)
-    const cudaError_t e = gemv_mma_opt_in<false>(smax);
-    return e != cudaSuccess ? e : gemv_mma_opt_in<true>(smax);
+    const int smax = static_cast<int>(kSmemLimit);
+    cudaError_t e;
+    if ((e = opt_in<1>(smax)) != cudaSuccess || (e = opt_in<2>(smax)) != cudaSuccess ||
+        (e = opt_in<4>(smax)) != cudaSuccess)
+        return e;
+    return opt_in<8>(smax);
 }
 
-cudaError_t launch_gemv_mma(const GemvMmaArgs& a, const Nf4Tables& tab, bool pdl, cudaStream_t st) {
-    if (a.M < 1 || a.M > kGemvMmaMaxM || a.ctas < 1) return cudaErrorInvalidValue;
-    const size_t smem = gemv_mma_smem_bytes(a.M, a.max_chunks);
+cudaError_t launch_gemv_mma(const CUtensorMap& codes, const CUtensorMap& x, const GemvMmaArgs& a,
+                            const Nf4Tables& tab, bool pdl, cudaStream_t st) {
+    if (a.M < 1 || a.M > kGemvMmaMaxM || a.ctas < 1 || a.stages < 2 || a.stages > kMaxStages)
+        return cudaErrorInvalidValue;
+    if (smem_bytes(a.M, a.stages) > kSmemLimit) return cudaErrorInvalidValue;
     const int mt = token_tiles(a.M);
-    static_assert(kMaxMt * 8 == kGemvMmaMaxM, "token tiles");
+    static_assert(8 * 8 == kGemvMmaMaxM, "token tiles");
     if (a.absmax) {
-        if (mt == 1) return launch_mt<1, true>(a, tab, smem, pdl, st);
-        if (mt == 2) return launch_mt<2, true>(a, tab, smem, pdl, st);
-        return launch_mt<4, true>(a, tab, smem, pdl, st);
+        if (mt == 1) return launch_mt<1, true>(codes, x, a, tab, pdl, st);
+        if (mt == 2) return launch_mt<2, true>(codes, x, a, tab, pdl, st);
+        if (mt == 4) return launch_mt<4, true>(codes, x, a, tab, pdl, st);
+        return launch_mt<8, true>(codes, x, a, tab, pdl, st);
     }
-    if (mt == 1) return launch_mt<1, false>(a, tab, smem, pdl, st);
-    if (mt == 2) return launch_mt<2, false>(a, tab, smem, pdl, st);
-    return launch_mt<4, false>(a, tab, smem, pdl, st);
+    if (mt == 1) return launch_mt<1, false>(codes, x, a, tab, pdl, st);
+    if (mt == 2) return launch_mt<2, false>(codes, x, a, tab, pdl, st);
+    if (mt == 4) return launch_mt<4, false>(codes, x, a, tab, pdl, st);
+    return launch_mt<8, false>(codes, x, a, tab, pdl, st);
 }
 
 }  // namespace qlora

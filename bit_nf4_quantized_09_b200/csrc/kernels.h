@@ -119,38 +119,10 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
                             const Nf4Tables& tab, bool pdl, cudaStream_t st);
 
-// ------------------------------------------------ small-batch dequant GEMV --
-constexpr int kGemvThreads = 320;  // 8 dequant warps (4 also epilogue), TMA warp, MMA warp
-constexpr int kGemvMaxM = 64;      // tokens that fit the UMMA N side of one tile (largest small-batch M)
-size_t gemv_smem_bytes();
-cudaError_t gemv_init_device();
-
-struct GemvArgs {
-    int64_t M, N, K;
-    int Mp;              // M rounded up to a multiple of 16
-    int r;               // LoRA rank
-    int splits;          // K splits (grid.y)
-    int steps_per_split;
-    float* part;         // fp32 [splits][M][N] partials (splits > 1)
-    int* counter;        // [N/128 row tiles] tickets, zero before the launch; left zero
-    const uint16_t* sT;  // bf16 [M, r]
-    const uint16_t* B;   // bf16 [N, r]
-    uint16_t* Y;         // bf16 [M, N]
-    int* status;
-    uint64_t timeout_ns;
-};
-
-// Maps: x = X {K, M} box {64, Mp} SW128; codes {K/2, N} box {32, 128} SW32;
-// cT {ldc, K/64} box {128, 1}.
-cudaError_t launch_gemv(const CUtensorMap& x, const CUtensorMap& codes, const CUtensorMap& cT, const GemvArgs& a,
-                        const Nf4Tables& tab, cudaStream_t st);
-
 // ------------------------------------- small-batch register-fed MMA GEMV --
-constexpr int kGemvMmaMaxM = 32;  // tokens: up to four n8 MMA tiles
+constexpr int kGemvMmaMaxM = 64;  // tokens: up to eight n8 MMA tiles
 
 struct GemvMmaArgs {
-    const uint16_t* X;       // bf16 [M, K]
-    const uint8_t* codes;    // packed NF4 [N, K/2]
     const uint8_t* qabsmax;  // E4M3 [N*K/64]
     const float* s2;         // [groups]
     const float* mean;       // [1]
@@ -165,28 +137,30 @@ struct GemvMmaArgs {
     int64_t group_end[kMaxGroups];
     int group_rank_x[kMaxGroups];
     int ctas;                // grid size (from the plan)
-    int64_t units;           // (N/128 row tiles) * (K/64 block columns)
-    int max_chunks;          // staged X chunks per CTA (from the plan)
+    int64_t units;           // (row tiles) * (K/64 block columns)
+    int stages;              // shared-memory pipeline stages (from the plan)
     float* part;             // fp32 [max_parts][M][N] partial sums
-    int* counter;            // [N/128 row tiles] tickets, zero before the launch; left zero
+    int* counter;            // [row tiles] tickets, zero before the launch; left zero
     const uint16_t* sT;      // bf16 [M, sT_ld], read only in the epilogue
     const uint16_t* B;       // bf16 [N, B_ld]
     uint16_t* Y;             // bf16 [M, N]
+    int* status;             // device status word
+    uint64_t timeout_ns;
 };
 
 struct GemvMmaPlan {
     int ctas;
     int64_t units;
-    int max_chunks;
+    int stages;
     int max_parts;  // partial-sum slots per row tile
 };
 
 GemvMmaPlan gemv_mma_plan(int64_t M, int64_t N, int64_t K, int num_sms);
-size_t gemv_mma_smem_bytes(int64_t M, int max_chunks);
 cudaError_t gemv_mma_init_device();
-// pdl: launch as the programmatic dependent of the previous launch on the
-// stream (the kernel waits for it before reading sT).
-cudaError_t launch_gemv_mma(const GemvMmaArgs& a, const Nf4Tables& tab, bool pdl, cudaStream_t st);
+// Maps: codes {K/2, N} box {128, 256} SW128; x = X {K, M} box {64, M} SW128. pdl: launch as the programmatic dependent of the previous launch on
+// the stream (the kernel waits for it before reading sT).
+cudaError_t launch_gemv_mma(const CUtensorMap& codes, const CUtensorMap& x, const GemvMmaArgs& a,
+                            const Nf4Tables& tab, bool pdl, cudaStream_t st);
 
 // ---------------------------------------------------------- skinny GEMMs --
 // D[rows, NR] = sum over the reduction of A_op[rows, red] * B_op[NR, red]^T,

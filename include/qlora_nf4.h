@@ -287,7 +287,7 @@ const char* qlora_status_string(qlora_status s);
 const char* qlora_last_error(void);
 
 /* Test and tuning hooks (not needed for normal use).
- *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses a
+ *   QLORA_OPT_SMALL_M_MAX   token count up to which the forward uses the
  *                           small-batch weight-streaming kernel (default 16,
  *                           maximum 64; 0 forces the tiled GEMM for every M);
  *                           above it the tiled GEMM, which splits its tiles
@@ -309,10 +309,6 @@ const char* qlora_last_error(void);
 #define QLORA_OPT_SKINNY_MAX_SPLITS 6 /* tuning: cap on the reduction splits of
                                         the rank-r matmuls (0 = no cap; a cap
                                         only lowers them, workspaces stay valid) */
-#define QLORA_OPT_REG_GEMV_MAX_M  7  /* token count up to which the small-batch
-                                        forward decodes in registers and feeds
-                                        mma.sync (default 16, maximum 32; 0 =
-                                        always the tcgen05 small-batch kernel) */
 qlora_status qlora_set_option(int option, int64_t value);
 int64_t qlora_get_option(int option);
 

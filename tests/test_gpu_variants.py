@@ -121,10 +121,9 @@ def test_nodq_forward_backward(q, cfg):
     check("dB", f64(dB), dBr)
 
 
-def test_nodq_tcgen05_small_batch_path(q):
-    """A weight without double quantisation through the tcgen05 small-batch
-    kernel (constants transposed by the same launch that decodes them with
-    double quantisation)."""
+def test_nodq_small_batch_four_token_tiles(q):
+    """A weight without double quantisation through the small-batch kernel
+    with 24 tokens (four n8 token tiles; forced past its default limit)."""
     cfg = synth.custom(N=1024, K=576, M=24, r=16)
     W, X, A, B = synth.weight(cfg), synth.activations(cfg), synth.lora_a(cfg), synth.lora_b(cfg)
     w = quantize(q, W, True)
