@@ -550,6 +550,15 @@ qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uin
     return QLORA_OK;
 }
 
+std::atomic<int64_t> g_fused_pairs{1};
+
+// Whole output tiles (at least as many as SMs) and at least two row tiles:
+// the fused matmuls run in CTA pairs that share each dequantised weight tile.
+bool use_pairs(int64_t M, int64_t tiles_n, int sms) {
+    const int64_t tiles_m = cdiv(M, kFusedBM);
+    return g_fused_pairs.load() != 0 && tiles_m >= 2 && tiles_m * tiles_n >= std::min(sms, kPlanSms);
+}
+
 // The projections of a group as column groups of one fused forward; a
 // single weight is one group.
 void set_groups(FusedArgs* fa, const Weights& W, const Lora& lo) {
@@ -706,13 +715,25 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
     if (injected_failure()) return QLORA_ERR_CUDA;
+    // whole tiles in CTA pairs that share each dequantised weight tile
+    const bool pair = use_pairs(M, fused_tiles_n(fa), sms);
+    if (pair) {
+        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_32B, "codes");
+        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
+    }
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_FWD, &ev0, &ev1);
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
     // programmatic dependent of the sT launch: the main loop overlaps it
     // (a profiled call keeps plain stream order)
-    QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
-                 "fused forward");
+    if (pair)
+        QLORA_LAUNCH(launch_fused_pair_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
+                     "fused forward (pairs)");
+    else
+        QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
+                     "fused forward");
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
     return QLORA_OK;
 }
@@ -795,12 +816,23 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = 0;
     if (injected_failure()) return QLORA_ERR_CUDA;
+    const bool pair = use_pairs(M, fused_tiles_n(fa), sms);
+    if (pair) {
+        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_64B, "codes");
+        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
+    }
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
     // plain stream order after the rank-r launches: the adapter gradients,
     // dX's programmatic dependent, read sU and sT from their first step
-    QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
+    if (pair)
+        QLORA_LAUNCH(launch_fused_pair_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1,
+                     "fused dX (pairs)");
+    else
+        QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
 
     // dA = sU^T X (as dA^T[K, R] = X^T sU, in 64-column chunks) and dB = dY^T sT
@@ -922,6 +954,7 @@ qlora_status qlora_set_option(int option, int64_t value) {
             if (value < 0) return QLORA_ERR_INVALID_ARG;
             g_skinny_max_splits = value;
             return QLORA_OK;
+        case QLORA_OPT_FUSED_PAIRS: g_fused_pairs = value ? 1 : 0; return QLORA_OK;
         default: return QLORA_ERR_INVALID_ARG;
     }
 }
@@ -934,6 +967,7 @@ int64_t qlora_get_option(int option) {
         case QLORA_OPT_STALL_PRODUCER: return g_stall_producer.load();
         case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
         case QLORA_OPT_SKINNY_MAX_SPLITS: return g_skinny_max_splits.load();
+        case QLORA_OPT_FUSED_PAIRS: return g_fused_pairs.load();
         default: return -1;
     }
 }

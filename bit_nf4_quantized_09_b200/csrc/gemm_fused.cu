@@ -495,6 +495,342 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA pairs (whole tiles). Two CTAs of a cluster take the same 256-column
+// weight tile and two neighbouring 256-row activation tiles. Each
+// dequantises only its half of the weight tile (128 of its N rows; for dX 128
+// of its output columns, 16 KB either way) into its own shared memory, and one
+// thread then copies that half into the partner's weight stage with a bulk
+// shared-to-shared copy that completes on the partner's barrier as
+// transaction bytes; every weight tile is decoded once per pair instead of
+// once per CTA. Each CTA runs the same cta_group::1 UMMAs on its own full
+// copy.
+//
+// Three rings: activation tiles (3 stages, loaded by one producer lane),
+// this CTA's half of the packed codes and constants (6 stages, another lane,
+// so codes arrive far ahead of their use) and decoded weight tiles (3
+// stages). The dequantiser warps form two groups that take the steps in
+// turn. A weight stage is rewritten only when both CTAs' UMMAs have consumed
+// it (multicast commit), because the partner copies into it; the rank-r
+// weight tile of a rank step is loaded into the weight stage by the group
+// that owns the step.
+// ---------------------------------------------------------------------------
+constexpr int kPA = 3, kPW = 3, kPC = 6;                 // ring depths: activations, weights, codes
+constexpr uint32_t kPCodeBytes = 4096;                    // this CTA's half of a step's codes
+constexpr uint32_t kPCStage = kPCodeBytes + 1024;         // + its half of the constants (512 B used)
+constexpr uint32_t kPOffW = kPA * kActBytes;              // 96 KB
+constexpr uint32_t kPOffCodes = kPOffW + kPW * kWBytes;   // 192 KB
+constexpr uint32_t kPBarOffset = kPOffCodes + kPC * kPCStage;
+constexpr uint32_t kPSmemBytes = kPBarOffset + 512 + 1024;
+
+template <bool kTransW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
+    fused_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_lact,
+                        const __grid_constant__ CUtensorMap tm_lw, const FusedArgs args, const Nf4Tables tab) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + kPBarOffset);
+    uint64_t* a_empty = a_full + kPA;
+    uint64_t* w_full = a_empty + kPA;
+    uint64_t* w_empty = w_full + kPW;
+    uint64_t* c_full = w_empty + kPW;
+    uint64_t* c_empty = c_full + kPC;
+    uint64_t* acc = c_empty + kPC;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+    const int KT = static_cast<int>((args.red + kFusedBK - 1) / kFusedBK);
+    int tiles_n = 0;
+    {
+        int64_t start = 0;
+        for (int g = 0; g < args.ngroups; ++g) {
+            tiles_n += static_cast<int>((args.group_end[g] - start + kFusedBN - 1) / kFusedBN);
+            start = args.group_end[g];
+        }
+    }
+    // the pair's column tile and this CTA's row tile (the second row tile of
+    // the last pair may lie past M: its rows are zero-filled and never written)
+    const int pair = blockIdx.x >> 1;
+    const int64_t m0 = (static_cast<int64_t>(pair / tiles_n) * 2 + rank) * kFusedBM;
+    const TileCols tc = tile_cols(args, pair % tiles_n);
+    const int64_t n0 = tc.n0;
+    const int rank_steps = args.rank_cols > 0 ? args.rank_steps : 0;
+    const int steps = KT + rank_steps;
+    const uint64_t tmo = args.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPA; ++s) {
+            mbar_init(a_full + s, 1);
+            mbar_init(a_empty + s, 1);   // this CTA's UMMAs
+        }
+        for (int s = 0; s < kPW; ++s) {
+            mbar_init(w_full + s, 4);    // the owning group's 4 warps (+ the partner's half as bytes)
+            mbar_init(w_empty + s, 2);   // both CTAs' UMMAs
+        }
+        for (int s = 0; s < kPC; ++s) {
+            mbar_init(c_full + s, 1);
+            mbar_init(c_empty + s, 4);   // the consuming group's 4 warps
+        }
+        mbar_init(acc, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tm_act);
+        tma_prefetch_desc(&tm_codes);
+        tma_prefetch_desc(&tm_c);
+        tma_prefetch_desc(&tm_lact);
+        tma_prefetch_desc(&tm_lw);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_sync();  // the partner's barriers are initialised before any remote copy
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // --------------------------------------------------- producers --
+        if (lane == 0 && !args.stall_producer) {
+            // activation tiles (X or dY; sT or sU in the rank steps), 3 ahead
+            int last = -1;
+            for (int i = 0; i < steps; ++i) {
+                const int s = i % kPA;
+                const uint32_t u = static_cast<uint32_t>(i / kPA);
+                if (i >= kPA && !mbar_wait(a_empty + s, (u - 1) & 1u, tmo, args.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                uint8_t* st = smem + s * kActBytes;
+                mbar_arrive_expect_tx(a_full + s, kActBytes);
+                if (i < KT) {
+                    tma_load_2d(st, &tm_act, a_full + s, i * kFusedBK, static_cast<int>(m0));
+                } else {
+                    const int c = i - KT;
+                    if (c == 0) asm volatile("griddepcontrol.wait;" ::: "memory");  // sT / sU of the preceding launch
+                    tma_load_2d(st, &tm_lact, a_full + s, tc.rank_x + 64 * c, static_cast<int>(m0));
+                }
+                last = i;
+            }
+            for (int i = max(0, last - kPA + 1); i <= last; ++i)
+                mbar_wait(a_full + i % kPA, static_cast<uint32_t>(i / kPA) & 1u, tmo, nullptr);
+        } else if (lane == 1 && !args.stall_producer) {
+            // this CTA's half of the codes and constants, 6 ahead
+            int last = -1;
+            for (int i = 0; i < KT; ++i) {
+                const int s = i % kPC;
+                const uint32_t u = static_cast<uint32_t>(i / kPC);
+                if (i >= kPC && !mbar_wait(c_empty + s, (u - 1) & 1u, tmo, args.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                uint8_t* st = smem + kPOffCodes + s * kPCStage;
+                mbar_arrive_expect_tx(c_full + s, kPCodeBytes + 512);
+                if (!kTransW) {
+                    tma_load_2d(st, &tm_codes, c_full + s, i * (kFusedBK / 2),
+                                static_cast<int>(n0) + 128 * static_cast<int>(rank));
+                    tma_load_2d(st + kPCodeBytes, &tm_c, c_full + s, static_cast<int>(n0) + 128 * static_cast<int>(rank),
+                                i);
+                } else {
+                    tma_load_2d(st, &tm_codes, c_full + s, static_cast<int>(n0 / 2) + 64 * static_cast<int>(rank),
+                                i * kFusedBK);
+                    tma_load_2d(st + kPCodeBytes, &tm_c, c_full + s, i * kFusedBK,
+                                static_cast<int>(n0 / kBlock) + 2 * static_cast<int>(rank));
+                }
+                last = i;
+            }
+            for (int i = max(0, last - kPC + 1); i <= last; ++i)
+                mbar_wait(c_full + i % kPC, static_cast<uint32_t>(i / kPC) & 1u, tmo, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ----------------------------------------------------------- MMA --
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, kFusedBN, false, kTransW);
+            bool ok = true;
+            tc_fence_after();
+            for (int i = 0; i < steps; ++i) {
+                const int sa = i % kPA, sw = i % kPW;
+                if (!mbar_wait(a_full + sa, static_cast<uint32_t>(i / kPA) & 1u, tmo, args.status) ||
+                    !mbar_wait_cluster(w_full + sw, static_cast<uint32_t>(i / kPW) & 1u, tmo, args.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t act = smem_u32(smem + sa * kActBytes);
+                const uint32_t wt = smem_u32(smem + kPOffW + sw * kWBytes);
+                const int ksub = (i < KT) ? (kFusedBK / 16) : (min(64, args.rank_cols - 64 * (i - KT)) + 15) / 16;
+                for (int kk = 0; kk < ksub; ++kk) {
+                    const uint64_t bdesc = kTransW ? sw128_desc(wt + kk * 2048, 8192, 1024)
+                                                   : sw128_desc(wt + kk * 32, 16, 1024);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t adesc = sw128_desc(act + h * 16384 + kk * 32, 16, 1024);
+                        umma_f16(tmem + h * 256, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(a_empty + sa);
+                umma_commit_multicast(w_empty + sw, 0x3);  // the weight stage is free in both CTAs' view
+            }
+            umma_commit(acc);  // arrives once every UMMA has completed (also after an abort)
+            if (!ok) {
+                *abort_flag = 1;
+                __threadfence_block();
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- dequantise half tiles, then epilogue --
+        // group G (warps 4G .. 4G + 3) takes the steps i with i % 2 == G;
+        // thread tl decodes N row 128 rank + tl (forward) or output-column
+        // block 2 rank + tl / 64, reduction row tl % 64 (dX)
+        const int G = warp >> 2, tl = (warp & 3) * 32 + lane;
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        const uint32_t w_full_remote = mapa_shared(smem_u32(w_full), peer);
+        constexpr uint32_t kHalf = kWBytes / 2;  // this CTA's half of the weight tile
+        bool ok = true;
+        for (int i = G; ok && i < steps; i += 2) {
+            const int sw = i % kPW;
+            // both CTAs' UMMAs are done with the weight stage's previous use
+            if (i >= kPW)
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(w_empty + sw, static_cast<uint32_t>(i / kPW - 1) & 1u,
+                                                               tmo, args.status));
+            if (!ok) break;
+            uint8_t* wst = smem + kPOffW + sw * kWBytes;
+            const uint32_t wt = smem_u32(wst);
+            if (i < KT) {
+                const int sc = i % kPC;
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(c_full + sc, static_cast<uint32_t>(i / kPC) & 1u, tmo,
+                                                       args.status));
+                if (!ok) break;
+                uint8_t* cst = smem + kPOffCodes + sc * kPCStage;
+                const uint32_t codes = smem_u32(cst);
+                const float* cs = reinterpret_cast<const float*>(cst + kPCodeBytes);
+                uint32_t c0, c1, dst;
+                float cprime;
+                int swz;
+                if (!kTransW) {
+                    // codes rows are 32 B, 32-byte swizzled; W row n = 128 rank + tl
+                    const uint32_t crow = codes + tl * 32;
+                    const uint32_t sw32 = (tl >> 2) & 1;
+                    c0 = crow + ((0 ^ sw32) << 4);
+                    c1 = crow + ((1 ^ sw32) << 4);
+                    const int n = 128 * static_cast<int>(rank) + tl;
+                    dst = static_cast<uint32_t>(n) * 128u;
+                    swz = n & 7;
+                    cprime = cs[tl];
+                } else {
+                    // codes rows are 64 B (this CTA's 128 output columns), 64-byte swizzled
+                    const int nl = tl & 63, al = tl >> 6, a = 2 * static_cast<int>(rank) + al;
+                    const uint32_t crow = codes + nl * 64;
+                    const uint32_t sw64 = (nl >> 1) & 3;
+                    c0 = crow + (((2 * al) ^ sw64) << 4);
+                    c1 = crow + (((2 * al + 1) ^ sw64) << 4);
+                    dst = static_cast<uint32_t>(a * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128);
+                    swz = nl & 7;
+                    cprime = cs[al * 64 + nl];
+                }
+                const Nf4BlockLut lutb = make_block_lut(tab.level, cprime);
+                const uint4 ca = lds128(c0), cb = lds128(c1);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(c_empty + sc);  // the codes stage has been read
+                const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t o[4];
+                    lut_decode8(lutb, words[j], o);
+                    sts128(wt + dst + ((static_cast<uint32_t>(j) ^ static_cast<uint32_t>(swz)) << 4), o);
+                }
+                fence_proxy_async_smem();  // -> visible to the tensor core and the bulk copy
+                // the group's half is complete: one thread sends it to the partner
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + G) : "memory");
+                if (leader) {
+                    mbar_arrive_expect_tx(w_full + sw, kHalf);  // the partner's half, coming the same way
+                    bulk_copy_to_cluster(mapa_shared(wt + kHalf * rank, peer), wt + kHalf * rank, kHalf,
+                                         w_full_remote + static_cast<uint32_t>(sw) * 8u);
+                } else if (lane == 0) {
+                    mbar_arrive(w_full + sw);
+                }
+            } else {
+                // rank step: the rank-r weight tile straight into the weight stage
+                if (leader) {
+                    const int c = i - KT;
+                    mbar_arrive_expect_tx(w_full + sw, kWBytes);
+                    if (!kTransW) {
+                        tma_load_2d(wst, &tm_lw, w_full + sw, 64 * c, static_cast<int>(n0));
+                    } else {
+                        for (int a = 0; a < 4; ++a)
+                            tma_load_2d(wst + a * 8192, &tm_lw, w_full + sw, static_cast<int>(n0) + 64 * a, 64 * c);
+                    }
+                } else if (lane == 0) {
+                    mbar_arrive(w_full + sw);
+                }
+            }
+        }
+        if (!ok) *abort_flag = 1;
+
+        // ------------------------------------------------------ epilogue --
+        const int q = warp & 3, h = warp >> 2;
+        const int row_l = h * 128 + q * 32 + lane;
+        const bool acc_ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0u, tmo, args.status));
+        tc_fence_after();
+        const bool write = __all_sync(0xFFFFFFFFu, acc_ok && !*abort_flag);
+        const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+        const int64_t row = m0 + row_l;
+        // 2 KB scratch of this warp in the first activation stage, idle now
+        // (every UMMA has completed and every activation copy has landed)
+        const uint32_t scratch = smem_u32(smem) + warp * 2048;
+        for (int c = 0; c < kFusedBN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(trow + 32 * c, r);
+            tmem_ld_wait();
+            if (write && row < args.M) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w4[4] = {pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                                            pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                                            pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                                            pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]))};
+                    sts128(scratch + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), w4);
+                }
+            }
+            __syncwarp();
+            if (write) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = 8 * i + (lane >> 2), pc = lane & 3;
+                    const int64_t orow = m0 + row_l - lane + rr;
+                    const int64_t ocol = n0 + 32 * c + 8 * pc;
+                    const uint4 d = lds128(scratch + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4));
+                    if (orow < args.M && ocol < tc.n_lim)
+                        *reinterpret_cast<uint4*>(args.out + orow * args.out_cols + ocol) = d;
+                }
+            }
+            __syncwarp();
+        }
+        tc_fence_before();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // the partner may still copy into this CTA's shared memory until it has
+    // passed its own main loop
+    cluster_sync();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 template <bool kTransW>
 cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
                          const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
@@ -521,9 +857,44 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
     return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, true>, act, codes, cT, lact, lw, a, tab);
 }
 
+template <bool kTransW>
+cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,
+                        const CUtensorMap& lact, const CUtensorMap& lw, const FusedArgs& a, const Nf4Tables& tab,
+                        bool pdl, cudaStream_t st) {
+    int least = 0, greatest = 0;
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles_m = (a.M + kFusedBM - 1) / kFusedBM;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * fused_tiles_n(a) * ((tiles_m + 1) / 2)));
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = kPSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributePriority;
+    attr[0].val.priority = greatest;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, fused_nf4_gemm_pair<kTransW>, act, codes, cT, lact, lw, a, tab);
+}
+
 }  // namespace
 
 size_t fused_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_fused_pair_fwd(const CUtensorMap& act, const CUtensorMap& codes_half, const CUtensorMap& cT_half,
+                                  const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                                  const Nf4Tables& tab, bool pdl, cudaStream_t st) {
+    return launch_pair<false>(act, codes_half, cT_half, lora_act, lora_w, a, tab, pdl, st);
+}
+
+cudaError_t launch_fused_pair_dx(const CUtensorMap& act, const CUtensorMap& codes_half, const CUtensorMap& cT_half,
+                                 const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                                 const Nf4Tables& tab, bool pdl, cudaStream_t st) {
+    return launch_pair<true>(act, codes_half, cT_half, lora_act, lora_w, a, tab, pdl, st);
+}
 
 cudaError_t fused_init_device() {
     cudaError_t e;
@@ -534,8 +905,13 @@ cudaError_t fused_init_device() {
         (e = cudaFuncSetAttribute(fused_nf4_gemm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(kSmemBytes))) != cudaSuccess)
         return e;
-    return cudaFuncSetAttribute(fused_nf4_gemm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(kSmemBytes));
+    if ((e = cudaFuncSetAttribute(fused_nf4_gemm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kSmemBytes))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fused_nf4_gemm_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kPSmemBytes))) != cudaSuccess)
+        return e;
+    return cudaFuncSetAttribute(fused_nf4_gemm_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kPSmemBytes));
 }
 
 cudaError_t launch_fused_fwd(const CUtensorMap& act, const CUtensorMap& codes, const CUtensorMap& cT,

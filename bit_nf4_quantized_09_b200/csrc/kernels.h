@@ -119,6 +119,18 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
                             const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
                             const Nf4Tables& tab, bool pdl, cudaStream_t st);
 
+// CTA-pair forms of the two launches (whole tiles, clusters of two CTAs along
+// M that share each dequantised weight tile; each CTA decodes its half). The
+// grid is 2 * (column tiles) * ceil(row tiles / 2).
+// Maps as above except: forward codes box {32, 128}, cT box {128, 1}; dX
+// codes box {64, 64} SW64, cT box {64, 2}.
+cudaError_t launch_fused_pair_fwd(const CUtensorMap& act, const CUtensorMap& codes_half, const CUtensorMap& cT_half,
+                                  const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                                  const Nf4Tables& tab, bool pdl, cudaStream_t st);
+cudaError_t launch_fused_pair_dx(const CUtensorMap& act, const CUtensorMap& codes_half, const CUtensorMap& cT_half,
+                                 const CUtensorMap& lora_act, const CUtensorMap& lora_w, const FusedArgs& a,
+                                 const Nf4Tables& tab, bool pdl, cudaStream_t st);
+
 // ------------------------------------- small-batch register-fed MMA GEMV --
 constexpr int kGemvMmaMaxM = 64;  // tokens: up to eight n8 MMA tiles
 

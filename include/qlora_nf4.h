@@ -309,6 +309,10 @@ const char* qlora_last_error(void);
 #define QLORA_OPT_SKINNY_MAX_SPLITS 6 /* tuning: cap on the reduction splits of
                                         the rank-r matmuls (0 = no cap; a cap
                                         only lowers them, workspaces stay valid) */
+#define QLORA_OPT_FUSED_PAIRS     8  /* 1 (default): with whole output tiles the
+                                        fused matmuls run in CTA pairs sharing
+                                        each dequantised weight tile; 0: one
+                                        CTA per tile, each decoding its own */
 qlora_status qlora_set_option(int option, int64_t value);
 int64_t qlora_get_option(int option);
 

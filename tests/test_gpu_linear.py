@@ -290,3 +290,35 @@ def test_fused_split_tiles_deterministic(q):
     b = gpu_run(q, cfg, t)
     for k in ("Y", "dX", "dA", "dB"):
         assert torch.equal(a[k], b[k]), k
+
+
+# ------------------------------ fused matmuls in CTA pairs (whole tiles) ---
+
+PAIRS = [synth.custom(N=256 * 150 + 8, K=320, M=600, r=16),     # forward: 3 x 151 tiles, odd row tiles
+         synth.custom(N=320, K=256 * 150 + 64, M=520, r=32)]    # dX: 3 x 151 tiles, ragged output columns
+
+
+@pytest.mark.parametrize("cfg", PAIRS, ids=lambda c: c.name)
+def test_fused_pairs_against_oracle(q, cfg):
+    """At least as many output tiles as SMs: the forward (first case) or dX
+    (second) runs in CTA pairs, each CTA decoding half of the shared weight
+    tile into both CTAs' shared memory. Every output against the oracle."""
+    g, errs = full_compare(q, cfg)
+    print({k: f"{v:.2e}" for k, v in errs.items()})
+
+
+@pytest.mark.parametrize("cfg", PAIRS, ids=lambda c: c.name)
+def test_fused_pairs_match_single_cta_bits(q, cfg):
+    """The pair kernel runs the same UMMAs on the same decoded operands as the
+    one-CTA-per-tile kernel: identical bits, including the adapter gradients."""
+    t = inputs(cfg)
+    old = q.get_option(q.OPT_FUSED_PAIRS)
+    try:
+        q.set_option(q.OPT_FUSED_PAIRS, 1)
+        a = gpu_run(q, cfg, t)
+        q.set_option(q.OPT_FUSED_PAIRS, 0)
+        b = gpu_run(q, cfg, t)
+    finally:
+        q.set_option(q.OPT_FUSED_PAIRS, old)
+    for k in ("Y", "dX", "dA", "dB"):
+        assert torch.equal(a[k], b[k]), k
