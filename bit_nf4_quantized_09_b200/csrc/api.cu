@@ -234,23 +234,14 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
 
-// Reduction splits of a skinny matmul: enough CTAs for two per SM of a
-// 148-SM B200 (fixed so workspace sizes do not depend on the device).
+// Reduction splits of a skinny matmul: the CTAs of a row tile form a cluster
+// of S = 1, 2, 4 or 8 that reduces in distributed shared memory; S doubles
+// while the launch stays within about two CTAs per SM of a 148-SM B200 and
+// every split keeps a reduction step. Four 24 KB stages (two CTAs per SM).
 constexpr int64_t kTargetCtas = 296;
 constexpr int kPlanSms = 148;  // the SM count the split plans are tuned for (any count runs them)
-struct Split {
-    int splits;
-    int steps;
-};
-Split split_for(int64_t tiles, int64_t red) {
-    const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
-    // as many splits as fit in one wave of two CTAs per SM, at most 32
-    int64_t s = std::max<int64_t>(
-        1, std::min<int64_t>(std::min<int64_t>(kTargetCtas / std::max<int64_t>(tiles, 1), KT), 32));
-    const int64_t steps = cdiv(KT, s);
-    s = cdiv(KT, steps);
-    return Split{static_cast<int>(s), static_cast<int>(steps)};
-}
+constexpr int kSkinnyStagesUsed = 4;
+int skinny_splits(int64_t tiles, int64_t red);
 
 // ------------------------------------------------------- the low-rank side --
 // The adapter side of a forward or backward call. One adapter (P = 1);
@@ -286,19 +277,18 @@ struct Weights {
 };
 
 // ------------------------------------------------------- workspace layout --
-// Head of every fwd/bwd workspace: the device status word, then the split
-// tickets of the skinny matmuls and the stream-K flags of the fused ones;
+// Head of every fwd/bwd workspace: the device status word, then the tickets
+// of the small-batch kernel and the stream-K flags of the fused matmuls;
 // cleared by one memset at the start of each call (the kernels also leave
 // their tickets at zero).
 struct Layout {
     size_t header = 0;                                   // bytes cleared per call
-    size_t status = 0, ctrT = 0, ctrU = 0, ctrA = 0, ctrB = 0, ctrY = 0, flags = 0;
+    size_t status = 0, ctrY = 0, flags = 0;
     size_t skpart = 0;                                    // fused matmul: partial tiles of stream-K contributors
-    size_t cT = 0, cflat = 0, partT = 0, sT = 0, partY = 0;  // forward
-    size_t partU = 0, sU = 0, partA = 0;                  // backward (partA holds dA and dB partials)
+    size_t cT = 0, cflat = 0, sT = 0, partY = 0;  // forward
+    size_t sU = 0;                                // backward
     size_t total = 0;
     int64_t ldc = 0;
-    Split sT_split{1, 1}, sU_split{1, 1}, grad_split{1, 1};
     GemvMmaPlan reg_gemv{1, 1, 2, 1};
 };
 
@@ -317,18 +307,10 @@ Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
     Layout L;
     const int64_t N = W.N, K = W.K;
     const int R = lo.R();
-    const int NRc = rank_pad(std::min(R, 64));            // chunked rank problems
-    const int NRu = lo.group ? rank_pad(lo.r) : NRc;      // backward down-projection
-    const int nch = lo.chunks(), ndu = lo.down_bwd(), ndb = lo.grad_b();
     L.ldc = (N + 3) / 4 * 4;  // constants row pitch: a multiple of 16 bytes
-    const int64_t mtiles = std::max<int64_t>(1, cdiv(M, 128));
-    const int64_t ktiles = cdiv(K, 128), ntiles = cdiv(N, 128);
+    const int64_t ntiles = cdiv(N, 128);
     L.status = 0;
-    L.ctrT = 256;
-    L.ctrU = L.ctrT + 4 * static_cast<size_t>(nch * mtiles);
-    L.ctrA = L.ctrU + 4 * static_cast<size_t>(ndu * mtiles);
-    L.ctrB = L.ctrA + 4 * static_cast<size_t>(nch * ktiles);
-    L.ctrY = L.ctrB + 4 * static_cast<size_t>(ndb * ntiles);
+    L.ctrY = 256;
     L.flags = L.ctrY + 4 * static_cast<size_t>(ntiles);
     L.header = up256(L.flags + 4 * static_cast<size_t>(kPlanSms));
     size_t off = L.header;
@@ -343,11 +325,8 @@ Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
     L.skpart = take(static_cast<size_t>(fused_partial_ctas(M, fwd ? fwd_tiles_n(W, lo.group) : cdiv(K, 256),
                                                            fwd ? K : N, kPlanSms)) *
                     kFusedBM * kFusedBN * 4);
-    L.sT_split = split_for(mtiles * nch, K);
     L.sT = take(static_cast<size_t>(M) * R * 2);
-    const size_t partT_bytes = static_cast<size_t>(nch) * L.sT_split.splits * M * NRc * 4;
     if (fwd) {
-        L.partT = take(partT_bytes);
         if (M <= kGemvMmaMaxM) {
             // the small-batch kernel may run (its token limit is a runtime option)
             L.reg_gemv = gemv_mma_plan(M, N, K, kPlanSms);
@@ -357,18 +336,7 @@ Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
             if (lo.group) L.cflat = take(static_cast<size_t>(N * K / kBlock) * 4);
         }
     } else {
-        int64_t red_max = N;
-        if (lo.group) {
-            red_max = 0;
-            for (int i = 0; i < W.P; ++i) red_max = std::max(red_max, W.rows(i));
-        }
-        L.sU_split = split_for(mtiles * ndu, red_max);
-        L.grad_split = split_for(nch * ktiles + ndb * ntiles, M);
-        L.partU = take(std::max(static_cast<size_t>(ndu) * L.sU_split.splits * M * NRu * 4, partT_bytes));
-        L.partT = L.partU;
         L.sU = take(static_cast<size_t>(M) * R * 2);
-        const int64_t b_rows = lo.group ? N : ndb * N;
-        L.partA = take(static_cast<size_t>(L.grad_split.splits) * (nch * K + b_rows) * NRc * 4);
     }
     L.total = off;
     return L;
@@ -444,52 +412,40 @@ qlora_status make_rank_map(CUtensorMap* m, const uint16_t* base, int64_t rows, i
                     swizzle_for_rank(NR), what);
 }
 
-// The layout's split, lowered to the tuning cap if one is set.
-Split capped(const Split& sp, int64_t red) {
-    const int64_t cap = g_skinny_max_splits.load();
-    if (cap <= 0 || sp.splits <= cap) return sp;
+int skinny_splits(int64_t tiles, int64_t red) {
     const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
-    const int64_t steps = cdiv(KT, cap);
-    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
+    int64_t cap = g_skinny_max_splits.load();
+    if (cap <= 0 || cap > 8) cap = 8;
+    int64_t s = 1;
+    while (2 * s <= cap && std::max<int64_t>(tiles, 1) * 2 * s <= kTargetCtas && 2 * s <= KT) s *= 2;
+    return static_cast<int>(s);
 }
 
-// A split of a shorter reduction within the layout's partial buffers: at
-// most the layout's number of splits.
-Split split_within(const Split& sp, int64_t red) {
-    const Split c = capped(sp, red);
-    const int64_t KT = std::max<int64_t>(1, cdiv(red, 64));
-    const int64_t steps = cdiv(KT, c.splits);
-    return Split{static_cast<int>(cdiv(KT, steps)), static_cast<int>(steps)};
-}
-
-SkinnyProblem skinny_problem(int64_t rows, int64_t red, const Split& sp, int a_mn, int b_mn, int mode, int ncols,
-                             int64_t out_ld, float* part, int* counter) {
+SkinnyProblem skinny_problem(int64_t rows, int64_t red, int splits, int a_mn, int b_mn, int mode, int ncols,
+                             int64_t out_ld) {
     SkinnyProblem p{};
     p.rows = rows;
     p.red = red;
-    p.splits = sp.splits;
-    p.steps_per_split = sp.steps;
+    p.steps_per_split = static_cast<int>(cdiv(std::max<int64_t>(1, cdiv(red, 64)), splits));
     p.a_mn_major = a_mn;
     p.b_mn_major = b_mn;
     p.mode = mode;
     p.ncols = ncols;
     p.out_ld = out_ld;
     p.scale = 1.0f;
-    p.part = part;
-    p.counter = counter;
     return p;
 }
 
 // sT = bf16(s X A^T) [M, R] in 64-column chunks (one skinny problem each);
 // with row ids, the columns of every adapter but the row's own are zero.
 qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A, const Lora& lo, float scale,
-                      const Split& sp_layout, float* part, int* ctr, uint16_t* sT, int* status, cudaStream_t st) {
+                      uint16_t* sT, int* status, cudaStream_t st) {
     const int R = lo.R(), nch = lo.chunks(), NR = rank_pad(std::min(R, 64));
-    const Split sp = capped(sp_layout, K);
-    const int64_t mtiles = cdiv(M, 128);
     SkinnyMaps maps;
     SkinnyArgs a{};
     a.NR = NR;
+    a.splits = skinny_splits(cdiv(M, 128) * nch, K);
+    a.stages = kSkinnyStagesUsed;
     CUtensorMap tx;
     QLORA_MAP(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "X");
     for (int c = 0; c < nch; ++c) {
@@ -498,8 +454,7 @@ qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A
         QLORA_MAP(&maps.b[c], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A + static_cast<int64_t>(64 * c) * K, K, w, K * 2, 64,
                   NR, CU_TENSOR_MAP_SWIZZLE_128B, "A");
         SkinnyProblem& p = a.p[c];
-        p = skinny_problem(M, K, sp, 0, 0, kSkinnyOutBf16, w, R,
-                           part + static_cast<int64_t>(c) * sp_layout.splits * M * NR, ctr + c * mtiles);
+        p = skinny_problem(M, K, a.splits, 0, 0, kSkinnyOutBf16, w, R);
         p.scale = scale;
         p.out_bf16 = sT + 64 * c;
         p.row_ids = lo.ids;
@@ -517,14 +472,17 @@ qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A
 // above), or for a group one problem per projection, sU_i = s dY_i B_i with
 // dY_i the projection's columns of dY and B_i its rows of B [N, r].
 qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uint16_t* B, const Lora& lo, float scale,
-                      const Split& sp_layout, float* part, int* ctr, uint16_t* sU, int* status, cudaStream_t st) {
+                      uint16_t* sU, int* status, cudaStream_t st) {
     const int R = lo.R(), np = lo.down_bwd();
     const int NR = lo.group ? rank_pad(lo.r) : rank_pad(std::min(R, 64));
-    const int64_t N = W.N, mtiles = cdiv(M, 128);
+    const int64_t N = W.N;
+    int64_t red_max = 0;
+    for (int c = 0; c < np; ++c) red_max = std::max(red_max, lo.group ? W.rows(c) : N);
     SkinnyMaps maps;
     SkinnyArgs a{};
     a.NR = NR;
-    int64_t poff = 0;
+    a.splits = skinny_splits(cdiv(M, 128) * np, red_max);
+    a.stages = kSkinnyStagesUsed;
     for (int c = 0; c < np; ++c) {
         const int64_t n0 = lo.group ? W.off[c] : 0, red = lo.group ? W.rows(c) : N;
         const int w = lo.group ? lo.r : std::min(64, R - 64 * c);
@@ -533,10 +491,8 @@ qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uin
         qlora_status s = lo.group ? make_rank_map(&maps.b[c], B + n0 * lo.r, red, lo.r, lo.r, NR, "B")
                                   : make_rank_map(&maps.b[c], B + 64 * c, N, w, R, NR, "B");
         if (s != QLORA_OK) return s;
-        const Split sp = split_within(sp_layout, red);
         SkinnyProblem& p = a.p[c];
-        p = skinny_problem(M, red, sp, 0, 1, kSkinnyOutBf16, w, R, part + poff, ctr + c * mtiles);
-        poff += static_cast<int64_t>(sp_layout.splits) * M * NR;
+        p = skinny_problem(M, red, a.splits, 0, 1, kSkinnyOutBf16, w, R);
         p.scale = scale;
         p.out_bf16 = sU + (lo.group ? c * lo.r : 64 * c);
         p.row_ids = lo.ids;
@@ -622,7 +578,6 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
     uint8_t* base = static_cast<uint8_t*>(ws);
     int* status = reinterpret_cast<int*>(base + L.status);
     float* cT = reinterpret_cast<float*>(base + L.cT);
-    float* partT = reinterpret_cast<float*>(base + L.partT);
     uint16_t* sT = sT_save ? sT_save : reinterpret_cast<uint16_t*>(base + L.sT);
     const float scale = alpha / static_cast<float>(r);
 
@@ -641,9 +596,7 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
                                                      const_cast<float*>(cflat) + W.off[i] * K / kBlock, sms, st),
                              1, "decode constants");
         }
-        if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
-                          st)) != QLORA_OK)
-            return s;
+        if ((s = down_fwd(X, M, K, A, lo, scale, sT, status, st)) != QLORA_OK) return s;
         CUtensorMap t_codes, t_x;
         QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 128, 256,
                   CU_TENSOR_MAP_SWIZZLE_128B, "codes");
@@ -686,9 +639,7 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
         return QLORA_OK;
     }
     if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
-    if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partT, reinterpret_cast<int*>(base + L.ctrT), sT, status,
-                      st)) != QLORA_OK)
-        return s;
+    if ((s = down_fwd(X, M, K, A, lo, scale, sT, status, st)) != QLORA_OK) return s;
 
     CUtensorMap t_act, t_codes, t_c, t_lact, t_lw;
     QLORA_MAP(&t_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B, "X");
@@ -768,10 +719,8 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     uint8_t* base = static_cast<uint8_t*>(ws);
     int* status = reinterpret_cast<int*>(base + L.status);
     float* cT = reinterpret_cast<float*>(base + L.cT);
-    float* partU = reinterpret_cast<float*>(base + L.partU);
     uint16_t* sU = reinterpret_cast<uint16_t*>(base + L.sU);
     const uint16_t* sT = sT_in ? sT_in : reinterpret_cast<uint16_t*>(base + L.sT);
-    float* partA = reinterpret_cast<float*>(base + L.partA);
     const float scale = alpha / static_cast<float>(r);
     const int NRc = rank_pad(std::min(R, 64));
     const int nch = lo.chunks(), ndb = lo.grad_b();
@@ -780,13 +729,10 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     if (injected_failure()) return QLORA_ERR_CUDA;
     if ((s = decode_constants_t(W, L, cT, st)) != QLORA_OK) return s;
     // sU = s dY B, with B read in place (MN-major)
-    if ((s = down_bwd(dY, M, W, B, lo, scale, L.sU_split, partU, reinterpret_cast<int*>(base + L.ctrU), sU, status,
-                      st)) != QLORA_OK)
-        return s;
+    if ((s = down_bwd(dY, M, W, B, lo, scale, sU, status, st)) != QLORA_OK) return s;
     // sT from the forward, or recomputed
     if (!sT_in) {
-        if ((s = down_fwd(X, M, K, A, lo, scale, L.sT_split, partU, reinterpret_cast<int*>(base + L.ctrT),
-                          reinterpret_cast<uint16_t*>(base + L.sT), status, st)) != QLORA_OK)
+        if ((s = down_fwd(X, M, K, A, lo, scale, reinterpret_cast<uint16_t*>(base + L.sT), status, st)) != QLORA_OK)
             return s;
     }
 
@@ -841,20 +787,19 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     SkinnyMaps maps;
     SkinnyArgs ga{};
     ga.NR = NRc;
-    const Split gsp = capped(L.grad_split, M);
-    const int64_t ktiles = cdiv(K, 128), ntiles = cdiv(N, 128);
+    int64_t grad_tiles = nch * cdiv(K, 128);
+    for (int c = 0; c < ndb; ++c) grad_tiles += cdiv(lo.group ? W.rows(c) : N, 128);
+    ga.splits = skinny_splits(grad_tiles, M);
+    ga.stages = kSkinnyStagesUsed;
     CUtensorMap t_xt;
     QLORA_MAP(&t_xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
     int np = 0;
-    int64_t poff = 0;
     for (int c = 0; c < nch; ++c, ++np) {
         const int w = std::min(64, R - 64 * c);
         maps.a[np] = t_xt;
         if ((s = make_rank_map(&maps.b[np], sU + 64 * c, M, w, R, NRc, "sU")) != QLORA_OK) return s;
-        ga.p[np] = skinny_problem(K, M, gsp, 1, 1, kSkinnyOutF32Transposed, w, K, partA + poff,
-                                  reinterpret_cast<int*>(base + L.ctrA) + c * ktiles);
+        ga.p[np] = skinny_problem(K, M, ga.splits, 1, 1, kSkinnyOutF32Transposed, w, K);
         ga.p[np].out_f32 = dA + static_cast<int64_t>(64 * c) * K;
-        poff += static_cast<int64_t>(L.grad_split.splits) * K * NRc;
     }
     for (int c = 0; c < ndb; ++c, ++np) {
         const int64_t n0 = lo.group ? W.off[c] : 0, rows = lo.group ? W.rows(c) : N;
@@ -863,10 +808,8 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
                   CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
         if ((s = make_rank_map(&maps.b[np], sT + (lo.group ? c * r : 64 * c), M, w, R, NRc, "sT")) != QLORA_OK)
             return s;
-        ga.p[np] = skinny_problem(rows, M, gsp, 1, 1, kSkinnyOutF32, w, dB_cols, partA + poff,
-                                  reinterpret_cast<int*>(base + L.ctrB) + c * ntiles);
+        ga.p[np] = skinny_problem(rows, M, ga.splits, 1, 1, kSkinnyOutF32, w, dB_cols);
         ga.p[np].out_f32 = dB + (lo.group ? n0 * r : 64 * c);
-        poff += static_cast<int64_t>(L.grad_split.splits) * rows * NRc;
     }
     ga.status = status;
     ga.timeout_ns = timeout_ns();

@@ -37,17 +37,6 @@ constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;  // + barriers, + align
 constexpr uint32_t kTmemCols = 512;
 constexpr int kDequantWarps = 8;
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&v)[4]) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
-                 : "memory");
-}
-
 // Dequantise one 64-weight block: 32 code bytes (two 16-byte chunks at c0, c1)
 // into eight 16-byte bf16 chunks at dst + chunk_off(j).
 template <typename ChunkOff>

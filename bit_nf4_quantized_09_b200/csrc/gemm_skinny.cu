@@ -11,13 +11,16 @@
 //         read by TMA straight out of X and dY with the 128-byte swizzle);
 //   B_op  K-major (A [r, K]) or MN-major (B [N, r], sU and sT [M, r] read in
 //         place with a 32/64/128-byte swizzle matching NR).
-// The reduction is split over CTAs; each CTA writes fp32 partials and the last
-// CTA of a row tile (atomic ticket, no waiting) adds them in split order and
-// writes the result, so outputs are deterministic. One launch carries up to
-// eight such problems (grid.z), each with its own pair of operand maps: the
-// 64-column chunks of a rank above 64 (several adapters side by side), the
-// projections of a group, or dA and dB together. A bf16 output may zero, per
-// token row, the columns of the adapters that the row does not use.
+// The reduction is split over the S <= 8 CTAs of a thread-block cluster
+// (grid.y). Each CTA leaves its fp32 accumulator in its own shared memory;
+// after a cluster barrier CTA c sums rows [c 128/S, (c + 1) 128/S) of the
+// tile over the S CTAs in rank order through distributed shared memory and
+// writes them, so outputs are deterministic and no partials reach global
+// memory. One launch carries up to eight such problems (grid.z), each with
+// its own pair of operand maps: the 64-column chunks of a rank above 64
+// (several adapters side by side), the projections of a group, or dA and dB
+// together. A bf16 output may zero, per token row, the columns of the
+// adapters that the row does not use.
 //   warp 0 TMA producer, warp 1 TMEM owner + UMMA issuer, warps 2-5 epilogue.
 #include <algorithm>
 
@@ -31,9 +34,9 @@ namespace {
 constexpr uint32_t kABytes = 128 * 64 * 2;  // 16 KB
 constexpr uint32_t kBBytes = 64 * 64 * 2;   // up to 64 x 64 bf16
 constexpr uint32_t kStage = kABytes + kBBytes;
-constexpr uint32_t kBarOff = kSkinnyStages * kStage;
-constexpr uint32_t kSmem = kBarOff + 256 + 1024;
 constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kRowBytes = 256;  // one fp32 accumulator row of 64 columns in the reduction buffer
+__host__ __device__ constexpr uint32_t smem_bytes(int stages) { return stages * kStage + 256 + 1024; }
 
 // Shared-memory descriptor of an MN-major B tile [64 reduction rows, NR
 // columns] written by TMA with the swizzle whose span is NR * 2 bytes: rows of
@@ -60,18 +63,18 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     const int prob = blockIdx.z;
     const SkinnyProblem P = args.p[prob];
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
-    if (row0 >= P.rows || static_cast<int>(blockIdx.y) >= P.splits) return;  // whole CTA idle
+    if (row0 >= P.rows) return;  // the whole cluster (same row tile) is idle
     const CUtensorMap* ta = &maps.a[prob];
     const CUtensorMap* tb = &maps.b[prob];
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
-    uint64_t* empty = full + kSkinnyStages;
-    uint64_t* acc = empty + kSkinnyStages;
+    const int stages = args.stages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * kStage);
+    uint64_t* empty = full + kSkinnyMaxStages;
+    uint64_t* acc = empty + kSkinnyMaxStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NR = args.NR;
@@ -83,7 +86,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     const uint32_t b_bytes = static_cast<uint32_t>(NR) * 128u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSkinnyStages; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
@@ -106,12 +109,11 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            int last_use[kSkinnyStages];
-            for (int s = 0; s < kSkinnyStages; ++s) last_use[s] = -1;
+            int last = -1;
             for (int i = 0; i < steps; ++i) {
-                const int s = i % kSkinnyStages;
-                const uint32_t u = static_cast<uint32_t>(i / kSkinnyStages);
-                if (i >= kSkinnyStages && !mbar_wait(empty + s, (u - 1) & 1u, tmo, args.status)) {
+                const int s = i % stages;
+                const uint32_t u = static_cast<uint32_t>(i / stages);
+                if (i >= stages && !mbar_wait(empty + s, (u - 1) & 1u, tmo, args.status)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -130,10 +132,11 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                     tma_load_2d(st + kABytes, tb, full + s, k, 0);
                 else
                     tma_load_2d(st + kABytes, tb, full + s, 0, k);
-                last_use[s] = static_cast<int>(u);
+                last = i;
             }
-            for (int s = 0; s < kSkinnyStages; ++s)
-                if (last_use[s] >= 0) mbar_wait(full + s, static_cast<uint32_t>(last_use[s]) & 1u, tmo, nullptr);
+            // every copy in flight has landed before the stages are reused
+            for (int i = max(0, last - stages + 1); i <= last; ++i)
+                mbar_wait(full + i % stages, static_cast<uint32_t>(i / stages) & 1u, tmo, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -141,8 +144,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
             const uint32_t idesc = idesc_bf16(128, NR, P.a_mn_major != 0, P.b_mn_major != 0);
             bool ok = true;
             for (int i = 0; i < steps; ++i) {
-                const int s = i % kSkinnyStages;
-                const uint32_t u = static_cast<uint32_t>(i / kSkinnyStages);
+                const int s = i % stages;
+                const uint32_t u = static_cast<uint32_t>(i / stages);
                 if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a = smem_u32(smem + s * kStage), b = a + kABytes;
@@ -165,13 +168,17 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
         }
         __syncwarp();
     } else {
-        // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1; thread = output row
+        // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1; thread = tile
+        // row t. The accumulator row goes to this CTA's reduction buffer in
+        // the first stages (idle: every UMMA has completed and every copy has
+        // landed): 16-byte chunk c of row t at t * 256 + ((c ^ (t & 7)) << 4),
+        // so eight consecutive rows fill all banks.
         const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc, 0, tmo, args.status));
         tc_fence_after();
         const int q = warp & 3;
-        const int64_t row = row0 + q * 32 + lane;
+        const int t = q * 32 + lane;
         const bool good = ok && !*abort_flag && steps > 0;
-        float v[64];
+        const uint32_t buf = smem_u32(smem) + static_cast<uint32_t>(t) * kRowBytes;
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 16) {
             if (c0 < NR) {
@@ -179,92 +186,69 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                 tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[c0 + i] = good ? __uint_as_float(r[i]) : 0.0f;
-            }
-        }
-        bool last = true;
-        if (P.splits > 1) {
-            if (row < P.rows) {
-                float4* dst = reinterpret_cast<float4*>(P.part + (static_cast<int64_t>(blockIdx.y) * P.rows + row) * NR);
-#pragma unroll
-                for (int c = 0; c < 64; c += 4)
-                    if (c < NR) dst[c / 4] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-            }
-            __threadfence();  // publish this split's partials before taking a ticket
-            epi_bar();
-            if (threadIdx.x == 64) {
-                const int ticket = atomicAdd(P.counter + blockIdx.x, 1);
-                *last_flag = (ticket == P.splits - 1) ? 1 : 0;
-            }
-            epi_bar();
-            last = *last_flag != 0;
-            if (last) {
-                __threadfence();  // see the other splits' partials
-                if (row < P.rows) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = 0.0f;
-                    // splits in order; four splits' slices are loaded at once so
-                    // the loads overlap
-#pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 16) {
-                        if (c0 < NR) {
-                            for (int s0 = 0; s0 < P.splits; s0 += 4) {
-                                float4 x[4][4];
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    const float4* src = reinterpret_cast<const float4*>(
-                                        P.part + (static_cast<int64_t>(s0 + u) * P.rows + row) * NR + c0);
-#pragma unroll
-                                    for (int i = 0; i < 4; ++i)
-                                        x[u][i] = (s0 + u < P.splits) ? __ldcg(src + i)
-                                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                                }
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                                    for (int i = 0; i < 4; ++i) {
-                                        v[c0 + 4 * i] += x[u][i].x;
-                                        v[c0 + 4 * i + 1] += x[u][i].y;
-                                        v[c0 + 4 * i + 2] += x[u][i].z;
-                                        v[c0 + 4 * i + 3] += x[u][i].w;
-                                    }
-                                }
-                            }
-                        }
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w4[4] = {good ? r[4 * i] : 0u, good ? r[4 * i + 1] : 0u, good ? r[4 * i + 2] : 0u,
+                                            good ? r[4 * i + 3] : 0u};
+                    const uint32_t c = static_cast<uint32_t>(c0 / 4 + i);
+                    sts128(buf + ((c ^ static_cast<uint32_t>(t & 7)) << 4), w4);
                 }
-                if (threadIdx.x == 64) P.counter[blockIdx.x] = 0;  // ready for the next call
-            }
-        }
-        if (last && row < P.rows) {
-            const int nc = P.ncols;
-            if (P.mode == kSkinnyOutBf16) {
-                uint16_t* o = P.out_bf16 + row * P.out_ld;
-                // the adapter of this token row (row_ids set): columns of
-                // other adapters are written as zeros
-                const int id = P.row_ids ? __ldg(P.row_ids + row) : 0;
-#pragma unroll
-                for (int j = 0; j < 64; j += 2)
-                    if (j < nc) {
-                        const bool keep = !P.row_ids || (P.ids_col0 + j) / P.ids_r == id;
-                        *reinterpret_cast<uint32_t*>(o + j) =
-                            keep ? pack_bf16x2(__fmul_rn(P.scale, v[j]), __fmul_rn(P.scale, v[j + 1])) : 0u;
-                    }
-            } else if (P.mode == kSkinnyOutF32Transposed) {
-#pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    if (j < nc) P.out_f32[static_cast<int64_t>(j) * P.out_ld + row] = v[j];
-            } else {
-                float4* o = reinterpret_cast<float4*>(P.out_f32 + row * P.out_ld);
-#pragma unroll
-                for (int j = 0; j < 64; j += 4)
-                    if (j < nc) o[j / 4] = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
     }
 
+    // every CTA of the cluster has its accumulator in shared memory
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
+
+    // CTA `rank` sums its slice of rows over the cluster in rank order and
+    // writes it. Items are (row, 4-column chunk) pairs: row-major outputs take
+    // the chunks of a row on neighbouring threads, the transposed output the
+    // rows of a chunk.
+    {
+        const int S = args.splits;
+        const int rank = static_cast<int>(cluster_ctarank());
+        const int rows_per = 128 / S, chunks = NR / 4;
+        const bool by_row = P.mode == kSkinnyOutF32Transposed;
+        const uint32_t buf0 = smem_u32(smem);
+        const int id_rows = P.row_ids != nullptr;
+        for (int it = threadIdx.x; it < rows_per * chunks; it += kSkinnyThreads) {
+            const int rl = by_row ? it % rows_per : it / chunks;
+            const int c = by_row ? it / rows_per : it % chunks;
+            const int t = rank * rows_per + rl;
+            const int64_t row = row0 + t;
+            if (row >= P.rows || 4 * c >= P.ncols) continue;
+            const uint32_t off = static_cast<uint32_t>(t) * kRowBytes + ((static_cast<uint32_t>(c) ^ (t & 7)) << 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < S; ++s) {
+                const float4 x = ld_cluster_f4(mapa_shared(buf0 + off, static_cast<uint32_t>(s)));
+                v.x += x.x;
+                v.y += x.y;
+                v.z += x.z;
+                v.w += x.w;
+            }
+            const int j = 4 * c;
+            if (P.mode == kSkinnyOutBf16) {
+                // the adapter of this token row (row_ids set): columns of
+                // other adapters are written as zeros
+                const int id = id_rows ? __ldg(P.row_ids + row) : 0;
+                const bool keep = !id_rows || (P.ids_col0 + j) / P.ids_r == id;  // 4 columns, one adapter (r >= 8)
+                uint2 o;
+                o.x = keep ? pack_bf16x2(__fmul_rn(P.scale, v.x), __fmul_rn(P.scale, v.y)) : 0u;
+                o.y = keep ? pack_bf16x2(__fmul_rn(P.scale, v.z), __fmul_rn(P.scale, v.w)) : 0u;
+                *reinterpret_cast<uint2*>(P.out_bf16 + row * P.out_ld + j) = o;
+            } else if (P.mode == kSkinnyOutF32Transposed) {
+                P.out_f32[static_cast<int64_t>(j) * P.out_ld + row] = v.x;
+                P.out_f32[static_cast<int64_t>(j + 1) * P.out_ld + row] = v.y;
+                P.out_f32[static_cast<int64_t>(j + 2) * P.out_ld + row] = v.z;
+                P.out_f32[static_cast<int64_t>(j + 3) * P.out_ld + row] = v.w;
+            } else {
+                *reinterpret_cast<float4*>(P.out_f32 + row * P.out_ld + j) = v;
+            }
+        }
+    }
+
+    // no CTA leaves while another may still read its shared memory
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -277,32 +261,35 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
 }  // namespace
 
-size_t skinny_smem_bytes() { return kSmem; }
+size_t skinny_smem_bytes(int stages) { return smem_bytes(stages); }
 
 cudaError_t launch_skinny(const SkinnyMaps& maps, const SkinnyArgs& args, int nproblems, cudaStream_t st, bool pdl) {
     if (nproblems < 1 || nproblems > kSkinnyMaxProblems) return cudaErrorInvalidValue;
+    const int S = args.splits;
+    if (S != 1 && S != 2 && S != 4 && S != 8) return cudaErrorInvalidValue;
+    if (args.stages < 2 || args.stages > kSkinnyMaxStages) return cudaErrorInvalidValue;  // the buffer needs 32 KB
     int64_t max_tiles = 0;
-    int max_splits = 0;
-    for (int p = 0; p < nproblems; ++p) {
-        max_tiles = std::max<int64_t>(max_tiles, (args.p[p].rows + 127) / 128);
-        max_splits = std::max(max_splits, args.p[p].splits);
-    }
+    for (int p = 0; p < nproblems; ++p) max_tiles = std::max<int64_t>(max_tiles, (args.p[p].rows + 127) / 128);
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(max_tiles), static_cast<unsigned>(max_splits),
-                       static_cast<unsigned>(nproblems));
+    cfg.gridDim = dim3(static_cast<unsigned>(max_tiles), static_cast<unsigned>(S), static_cast<unsigned>(nproblems));
     cfg.blockDim = dim3(kSkinnyThreads);
-    cfg.dynamicSmemBytes = kSmem;
+    cfg.dynamicSmemBytes = smem_bytes(args.stages);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, skinny_gemm, maps, args);
 }
 
 cudaError_t skinny_init_device() {
-    return cudaFuncSetAttribute(skinny_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    return cudaFuncSetAttribute(skinny_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem_bytes(kSkinnyMaxStages)));
 }
 
 }  // namespace qlora

@@ -180,9 +180,9 @@ cudaError_t launch_gemv_mma(const CUtensorMap& codes, const CUtensorMap& x, cons
 // the fp32 partials in split order and writes the output. Up to
 // kSkinnyMaxProblems independent problems share one launch (blockIdx.z): the
 // 64-column chunks of a wider rank, or the gradients of several adapters.
-constexpr int kSkinnyStages = 4;
+constexpr int kSkinnyMaxStages = 8;  // 24 KB each
 constexpr int kSkinnyThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
-size_t skinny_smem_bytes();
+size_t skinny_smem_bytes(int stages);
 cudaError_t skinny_init_device();
 
 constexpr int kSkinnyOutBf16 = 0;           // out_bf16[row * out_ld + j] = bf16(scale * D)
@@ -193,16 +193,13 @@ constexpr int kSkinnyMaxProblems = 8;
 struct SkinnyProblem {
     int64_t rows;        // output rows (tiles of 128)
     int64_t red;         // reduction length (steps of 64)
-    int splits;          // reduction splits (grid.y)
-    int steps_per_split;
+    int steps_per_split; // reduction steps of each of the launch's splits
     int a_mn_major;      // A_op rows-contiguous: two 64-wide TMA boxes per step
     int b_mn_major;      // B_op stored [red, NR] (box {NR, 64}, swizzle = NR*2 bytes)
     int mode;            // kSkinnyOut*
     int ncols;           // output columns (<= NR, even; a multiple of 4 for fp32)
     int64_t out_ld;      // output pitch in elements
     float scale;         // bf16 output scale
-    float* part;         // fp32 [splits][rows][NR] partials (splits > 1)
-    int* counter;        // [row tiles] tickets, zero before the launch; left zero
     uint16_t* out_bf16;
     float* out_f32;
     // bf16 output only: with row_ids set, output column j of row `row` is
@@ -215,6 +212,8 @@ struct SkinnyProblem {
 
 struct SkinnyArgs {
     int NR;              // 16, 32 or 64: UMMA N of every problem
+    int splits;          // reduction splits = cluster size along grid.y: 1, 2, 4 or 8
+    int stages;          // pipeline stages, 2 .. kSkinnyMaxStages
     SkinnyProblem p[kSkinnyMaxProblems];
     int* status;
     uint64_t timeout_ns;

@@ -307,8 +307,10 @@ const char* qlora_last_error(void);
 #define QLORA_OPT_LAUNCH_COUNT    5  /* read: kernels launched by this library so
                                         far in this process; set: reset to value */
 #define QLORA_OPT_SKINNY_MAX_SPLITS 6 /* tuning: cap on the reduction splits of
-                                        the rank-r matmuls (0 = no cap; a cap
-                                        only lowers them, workspaces stay valid) */
+                                        the rank-r matmuls, which are the CTAs
+                                        of one cluster: 1, 2, 4 or 8 (0 = no
+                                        cap; other values round down to one of
+                                        these; workspaces do not depend on it) */
 #define QLORA_OPT_FUSED_PAIRS     8  /* 1 (default): with whole output tiles the
                                         fused matmuls run in CTA pairs sharing
                                         each dequantised weight tile; 0: one
