@@ -26,6 +26,7 @@ OP_QUANTIZE, OP_FWD, OP_BWD = 0, 1, 2
 OPT_SMALL_M_MAX, OPT_FAIL_LAUNCHES, OPT_WAIT_TIMEOUT_US, OPT_STALL_PRODUCER, OPT_LAUNCH_COUNT = 1, 2, 3, 4, 5
 OPT_SKINNY_MAX_SPLITS = 6
 OPT_FUSED_PAIRS = 8
+OPT_FUSED_TAIL = 9
 KERNEL_FUSED_FWD, KERNEL_FUSED_DX = 1, 2
 
 

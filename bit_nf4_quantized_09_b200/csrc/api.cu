@@ -57,16 +57,6 @@ qlora_status cuda_fail(cudaError_t e, const char* where) {
         g_launch_count += (nkernels);                   \
     } while (0)
 
-int tree_passes(int64_t nb) {
-    int passes = 1;
-    int64_t n = (nb + 1023) / 1024;
-    if (n == 1) return 2;
-    while (n > 1) {
-        n = (n + 1023) / 1024;
-        ++passes;
-    }
-    return passes;
-}
 
 // Host-side fault injection: consumes one "launch" and reports a failure
 // before anything reaches the GPU.
@@ -241,7 +231,17 @@ bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
 constexpr int64_t kTargetCtas = 296;
 constexpr int kPlanSms = 148;  // the SM count the split plans are tuned for (any count runs them)
 constexpr int kSkinnyStagesUsed = 4;
+constexpr int kSkinnyChunksUsed = 1;
 int skinny_splits(int64_t tiles, int64_t red);
+
+// Whole output tiles (at least as many as SMs) and at least two row tiles:
+// the fused matmuls may run in CTA pairs that share each dequantised weight
+// tile (the workspace then holds partial tiles for a stream-K tail).
+bool pairs_possible(int64_t M, int64_t tiles_n) {
+    const int64_t tiles_m = cdiv(M, kFusedBM);
+    return tiles_m >= 2 && tiles_m * tiles_n >= kPlanSms;
+}
+
 
 // ------------------------------------------------------- the low-rank side --
 // The adapter side of a forward or backward call. One adapter (P = 1);
@@ -322,9 +322,9 @@ Layout layout_for(int op, int64_t M, const Weights& W, const Lora& lo) {
     L.cT = take(static_cast<size_t>(K / kBlock) * L.ldc * 4);
     // the fused matmul's partial tiles, one per CTA, when it splits tiles
     const bool fwd = op == QLORA_OP_FWD;
-    L.skpart = take(static_cast<size_t>(fused_partial_ctas(M, fwd ? fwd_tiles_n(W, lo.group) : cdiv(K, 256),
-                                                           fwd ? K : N, kPlanSms)) *
-                    kFusedBM * kFusedBN * 4);
+    const int64_t tiles_n = fwd ? fwd_tiles_n(W, lo.group) : cdiv(K, 256);
+    const int64_t part_ctas = pairs_possible(M, tiles_n) ? kPlanSms : fused_partial_ctas(M, tiles_n, fwd ? K : N, kPlanSms);
+    L.skpart = take(static_cast<size_t>(part_ctas) * kFusedBM * kFusedBN * 4);
     L.sT = take(static_cast<size_t>(M) * R * 2);
     if (fwd) {
         if (M <= kGemvMmaMaxM) {
@@ -417,16 +417,15 @@ int skinny_splits(int64_t tiles, int64_t red) {
     int64_t cap = g_skinny_max_splits.load();
     if (cap <= 0 || cap > 8) cap = 8;
     int64_t s = 1;
-    while (2 * s <= cap && std::max<int64_t>(tiles, 1) * 2 * s <= kTargetCtas && 2 * s <= KT) s *= 2;
+    while (2 * s <= cap && std::max<int64_t>(tiles, 1) * 2 * s <= kTargetCtas && 2 * s * kSkinnyChunksUsed <= KT)
+        s *= 2;
     return static_cast<int>(s);
 }
 
-SkinnyProblem skinny_problem(int64_t rows, int64_t red, int splits, int a_mn, int b_mn, int mode, int ncols,
-                             int64_t out_ld) {
+SkinnyProblem skinny_problem(int64_t rows, int64_t red, int a_mn, int b_mn, int mode, int ncols, int64_t out_ld) {
     SkinnyProblem p{};
     p.rows = rows;
     p.red = red;
-    p.steps_per_split = static_cast<int>(cdiv(std::max<int64_t>(1, cdiv(red, 64)), splits));
     p.a_mn_major = a_mn;
     p.b_mn_major = b_mn;
     p.mode = mode;
@@ -446,6 +445,7 @@ qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A
     a.NR = NR;
     a.splits = skinny_splits(cdiv(M, 128) * nch, K);
     a.stages = kSkinnyStagesUsed;
+    a.chunks = kSkinnyChunksUsed;
     CUtensorMap tx;
     QLORA_MAP(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, "X");
     for (int c = 0; c < nch; ++c) {
@@ -454,7 +454,7 @@ qlora_status down_fwd(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A
         QLORA_MAP(&maps.b[c], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A + static_cast<int64_t>(64 * c) * K, K, w, K * 2, 64,
                   NR, CU_TENSOR_MAP_SWIZZLE_128B, "A");
         SkinnyProblem& p = a.p[c];
-        p = skinny_problem(M, K, a.splits, 0, 0, kSkinnyOutBf16, w, R);
+        p = skinny_problem(M, K, 0, 0, kSkinnyOutBf16, w, R);
         p.scale = scale;
         p.out_bf16 = sT + 64 * c;
         p.row_ids = lo.ids;
@@ -483,6 +483,7 @@ qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uin
     a.NR = NR;
     a.splits = skinny_splits(cdiv(M, 128) * np, red_max);
     a.stages = kSkinnyStagesUsed;
+    a.chunks = kSkinnyChunksUsed;
     for (int c = 0; c < np; ++c) {
         const int64_t n0 = lo.group ? W.off[c] : 0, red = lo.group ? W.rows(c) : N;
         const int w = lo.group ? lo.r : std::min(64, R - 64 * c);
@@ -492,7 +493,7 @@ qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uin
                                   : make_rank_map(&maps.b[c], B + 64 * c, N, w, R, NR, "B");
         if (s != QLORA_OK) return s;
         SkinnyProblem& p = a.p[c];
-        p = skinny_problem(M, red, a.splits, 0, 1, kSkinnyOutBf16, w, R);
+        p = skinny_problem(M, red, 0, 1, kSkinnyOutBf16, w, R);
         p.scale = scale;
         p.out_bf16 = sU + (lo.group ? c * lo.r : 64 * c);
         p.row_ids = lo.ids;
@@ -507,12 +508,40 @@ qlora_status down_bwd(const uint16_t* dY, int64_t M, const Weights& W, const uin
 }
 
 std::atomic<int64_t> g_fused_pairs{1};
+std::atomic<int64_t> g_fused_tail{0};
 
-// Whole output tiles (at least as many as SMs) and at least two row tiles:
-// the fused matmuls run in CTA pairs that share each dequantised weight tile.
-bool use_pairs(int64_t M, int64_t tiles_n, int sms) {
+// The fused launches of a call. CTA pairs take whole waves of tiles; when
+// their last wave would be short (at most kTailPercent of the SMs busy) its
+// tiles go instead to the one-CTA kernel, split stream-K over every SM and
+// launched as the pair launch's programmatic dependent. Without pairs, one
+// one-CTA launch over all tiles.
+constexpr int64_t kTailPercent = 85;
+struct FusedPlan {
+    int pair_ctas = 0;                      // CTAs of the pair launch (0: none)
+    int64_t tail_first = 0, tail_tiles = 0;  // tiles of the one-CTA launch (pair order; 0 tiles: all)
+    int tail_ctas = 0;                      // CTAs of the one-CTA launch (0: none)
+};
+FusedPlan fused_plan(int64_t M, int64_t tiles_n, int64_t red, int sms) {
+    FusedPlan p;
+    const int cap = std::min(sms, kPlanSms);
     const int64_t tiles_m = cdiv(M, kFusedBM);
-    return g_fused_pairs.load() != 0 && tiles_m >= 2 && tiles_m * tiles_n >= std::min(sms, kPlanSms);
+    if (g_fused_pairs.load() == 0 || tiles_m < 2 || tiles_m * tiles_n < cap) {
+        p.tail_ctas = fused_ctas(M, tiles_n, red, cap);
+        return p;
+    }
+    const int64_t all = 2 * tiles_n * cdiv(tiles_m, 2);
+    const int64_t wave = cap & ~1;
+    const int64_t full = all / wave * wave, rest = all - full;
+    if (g_fused_tail.load() == 0 || full == 0 || rest == 0 || rest * 100 > wave * kTailPercent ||
+        !pairs_possible(M, tiles_n)) {
+        p.pair_ctas = static_cast<int>(all);
+        return p;
+    }
+    p.pair_ctas = static_cast<int>(full);
+    p.tail_first = full;
+    p.tail_tiles = rest;
+    p.tail_ctas = fused_ctas_for(rest, red, cap);
+    return p;
 }
 
 // The projections of a group as column groups of one fused forward; a
@@ -666,12 +695,14 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = static_cast<int>(g_stall_producer.exchange(0));
     if (injected_failure()) return QLORA_ERR_CUDA;
-    // whole tiles in CTA pairs that share each dequantised weight tile
-    const bool pair = use_pairs(M, fused_tiles_n(fa), sms);
-    if (pair) {
-        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 128,
+    // whole tiles in CTA pairs that share each dequantised weight tile, the
+    // tiles of a short last wave stream-K
+    const FusedPlan plan = fused_plan(M, fused_tiles_n(fa), K, sms);
+    CUtensorMap h_codes, h_c;
+    if (plan.pair_ctas) {
+        QLORA_MAP(&h_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 32, 128,
                   CU_TENSOR_MAP_SWIZZLE_32B, "codes");
-        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
+        QLORA_MAP(&h_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 128, 1,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
     }
     cudaEvent_t ev0, ev1;
@@ -679,12 +710,23 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
     // programmatic dependent of the sT launch: the main loop overlaps it
     // (a profiled call keeps plain stream order)
-    if (pair)
-        QLORA_LAUNCH(launch_fused_pair_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
+    if (plan.pair_ctas) {
+        FusedArgs pa = fa;
+        pa.ctas = plan.pair_ctas;
+        QLORA_LAUNCH(launch_fused_pair_fwd(t_act, h_codes, h_c, t_lact, t_lw, pa, tables(), ev0 == nullptr, st), 1,
                      "fused forward (pairs)");
-    else
-        QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), ev0 == nullptr, st), 1,
-                     "fused forward");
+    }
+    if (plan.tail_ctas) {
+        FusedArgs ta = fa;
+        ta.ctas = plan.tail_ctas;
+        ta.tile_first = plan.tail_first;
+        ta.tiles = plan.tail_tiles;
+        ta.pair_order = plan.pair_ctas ? 1 : 0;
+        ta.stall_producer = plan.pair_ctas ? 0 : fa.stall_producer;
+        QLORA_LAUNCH(launch_fused_fwd(t_act, t_codes, t_c, t_lact, t_lw, ta, tables(),
+                                      plan.pair_ctas ? true : ev0 == nullptr, st),
+                     1, "fused forward");
+    }
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
     return QLORA_OK;
 }
@@ -762,23 +804,35 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     fa.timeout_ns = timeout_ns();
     fa.stall_producer = 0;
     if (injected_failure()) return QLORA_ERR_CUDA;
-    const bool pair = use_pairs(M, fused_tiles_n(fa), sms);
-    if (pair) {
-        QLORA_MAP(&t_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 64, 64,
+    const FusedPlan plan = fused_plan(M, fused_tiles_n(fa), N, sms);
+    CUtensorMap h_codes, h_c;
+    if (plan.pair_ctas) {
+        QLORA_MAP(&h_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.w[0].codes, K / 2, N, K / 2, 64, 64,
                   CU_TENSOR_MAP_SWIZZLE_64B, "codes");
-        QLORA_MAP(&t_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 2,
+        QLORA_MAP(&h_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cT, L.ldc, K / kBlock, L.ldc * 4, 64, 2,
                   CU_TENSOR_MAP_SWIZZLE_NONE, "constants");
     }
     cudaEvent_t ev0, ev1;
     take_profile_events(QLORA_KERNEL_FUSED_DX, &ev0, &ev1);
     if (ev0) QLORA_TRY(record_profile_event(ev0, st), "profile event");
-    // plain stream order after the rank-r launches: the adapter gradients,
-    // dX's programmatic dependent, read sU and sT from their first step
-    if (pair)
-        QLORA_LAUNCH(launch_fused_pair_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1,
+    // plain stream order after the rank-r launches (a stream-K tail is the
+    // pair launch's programmatic dependent); the adapter gradients, dX's
+    // programmatic dependent, read sU and sT from their first step
+    if (plan.pair_ctas) {
+        FusedArgs pa = fa;
+        pa.ctas = plan.pair_ctas;
+        QLORA_LAUNCH(launch_fused_pair_dx(t_act, h_codes, h_c, t_lact, t_lw, pa, tables(), false, st), 1,
                      "fused dX (pairs)");
-    else
-        QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, fa, tables(), false, st), 1, "fused dX");
+    }
+    if (plan.tail_ctas) {
+        FusedArgs ta = fa;
+        ta.ctas = plan.tail_ctas;
+        ta.tile_first = plan.tail_first;
+        ta.tiles = plan.tail_tiles;
+        ta.pair_order = plan.pair_ctas ? 1 : 0;
+        QLORA_LAUNCH(launch_fused_dx(t_act, t_codes, t_c, t_lact, t_lw, ta, tables(), plan.pair_ctas != 0, st), 1,
+                     "fused dX");
+    }
     if (ev1) QLORA_TRY(record_profile_event(ev1, st), "profile event");
 
     // dA = sU^T X (as dA^T[K, R] = X^T sU, in 64-column chunks) and dB = dY^T sT
@@ -791,6 +845,7 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
     for (int c = 0; c < ndb; ++c) grad_tiles += cdiv(lo.group ? W.rows(c) : N, 128);
     ga.splits = skinny_splits(grad_tiles, M);
     ga.stages = kSkinnyStagesUsed;
+    ga.chunks = kSkinnyChunksUsed;
     CUtensorMap t_xt;
     QLORA_MAP(&t_xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "X^T");
     int np = 0;
@@ -798,7 +853,7 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
         const int w = std::min(64, R - 64 * c);
         maps.a[np] = t_xt;
         if ((s = make_rank_map(&maps.b[np], sU + 64 * c, M, w, R, NRc, "sU")) != QLORA_OK) return s;
-        ga.p[np] = skinny_problem(K, M, ga.splits, 1, 1, kSkinnyOutF32Transposed, w, K);
+        ga.p[np] = skinny_problem(K, M, 1, 1, kSkinnyOutF32Transposed, w, K);
         ga.p[np].out_f32 = dA + static_cast<int64_t>(64 * c) * K;
     }
     for (int c = 0; c < ndb; ++c, ++np) {
@@ -808,7 +863,7 @@ qlora_status bwd_impl(const uint16_t* dY, const uint16_t* X, int64_t M, const We
                   CU_TENSOR_MAP_SWIZZLE_128B, "dY^T");
         if ((s = make_rank_map(&maps.b[np], sT + (lo.group ? c * r : 64 * c), M, w, R, NRc, "sT")) != QLORA_OK)
             return s;
-        ga.p[np] = skinny_problem(rows, M, ga.splits, 1, 1, kSkinnyOutF32, w, dB_cols);
+        ga.p[np] = skinny_problem(rows, M, 1, 1, kSkinnyOutF32, w, dB_cols);
         ga.p[np].out_f32 = dB + (lo.group ? n0 * r : 64 * c);
     }
     ga.status = status;
@@ -853,7 +908,7 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     if (N <= 0 || K <= 0 || K % kBlock != 0) return 0;
     if (op == QLORA_OP_QUANTIZE) {
         const int64_t nb = N * K / kBlock;
-        return up256(static_cast<size_t>(nb) * 4) + up256(dq_tree_scratch_doubles(nb) * 8);
+        return up256(static_cast<size_t>(nb) * 4) + dq_mean_scratch_bytes(nb);
     }
     if (op != QLORA_OP_FWD && op != QLORA_OP_BWD) return 0;
     if (M < 0 || !rank_ok(r)) return 0;
@@ -898,6 +953,7 @@ qlora_status qlora_set_option(int option, int64_t value) {
             g_skinny_max_splits = value;
             return QLORA_OK;
         case QLORA_OPT_FUSED_PAIRS: g_fused_pairs = value ? 1 : 0; return QLORA_OK;
+        case QLORA_OPT_FUSED_TAIL: g_fused_tail = value ? 1 : 0; return QLORA_OK;
         default: return QLORA_ERR_INVALID_ARG;
     }
 }
@@ -911,6 +967,7 @@ int64_t qlora_get_option(int option) {
         case QLORA_OPT_LAUNCH_COUNT: return g_launch_count.load();
         case QLORA_OPT_SKINNY_MAX_SPLITS: return g_skinny_max_splits.load();
         case QLORA_OPT_FUSED_PAIRS: return g_fused_pairs.load();
+        case QLORA_OPT_FUSED_TAIL: return g_fused_tail.load();
         default: return -1;
     }
 }
@@ -939,6 +996,20 @@ qlora_status qlora_quantize_nf4_bf16(const uint16_t* W, int64_t N, int64_t K, ui
 }
 
 namespace {
+// Quantise: the encoder (which also zeroes the mean kernel's ticket), the
+// mean and the E4M3 group pass.
+qlora_status quantize_dq(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
+                         float* mean, float* absmax, void* mean_scratch, int sms, cudaStream_t st) {
+    const int64_t nb = N * K / kBlock;
+    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, dq_mean_ticket(mean_scratch, nb), tables(), sms, st),
+                 1, "nf4_encode");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_dq_mean(absmax, nb, mean_scratch, mean, st), 1, "double quantisation mean");
+    if (injected_failure()) return QLORA_ERR_CUDA;
+    QLORA_LAUNCH(launch_dq_groups(absmax, nb, mean, qabsmax, s2, st), 1, "double quantisation groups");
+    return QLORA_OK;
+}
+
 qlora_status quantize_any(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, uint8_t* qabsmax, float* s2,
                           float* mean, void* ws, size_t ws_bytes, void* stream) {
     if (!W || !codes || !qabsmax || !s2 || !mean || !ws) return QLORA_ERR_INVALID_ARG;
@@ -954,11 +1025,8 @@ qlora_status quantize_any(const void* W, bool bf16, int64_t N, int64_t K, uint8_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t nb = N * K / kBlock;
     float* absmax = static_cast<float*>(ws);
-    double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + up256(static_cast<size_t>(nb) * 4));
-    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
-    return QLORA_OK;
+    void* tree = static_cast<uint8_t*>(ws) + up256(static_cast<size_t>(nb) * 4);
+    return quantize_dq(W, bf16, N, K, codes, qabsmax, s2, mean, absmax, tree, sms, st);
 }
 }  // namespace
 
@@ -972,8 +1040,9 @@ qlora_status quantize_nodq(const void* W, bool bf16, int64_t N, int64_t K, uint8
     int sms = 0;
     qlora_status s = device_ready(&sms);
     if (s != QLORA_OK) return s;
-    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, tables(), sms, static_cast<cudaStream_t>(stream)), 1,
-                 "nf4_encode");
+    QLORA_LAUNCH(launch_nf4_encode(W, bf16, N, K, codes, absmax, nullptr, tables(), sms,
+                                   static_cast<cudaStream_t>(stream)),
+                 1, "nf4_encode");
     return QLORA_OK;
 }
 }  // namespace
@@ -1169,36 +1238,28 @@ qlora_status qlora_e4m3_encode(const float* x, uint8_t* q, int64_t n, void* stre
 
 // ======================================================== no allocation ==
 // Quantiser scratch for callers that cannot allocate: one file-scope device
-// array, 4 MiB of fp32 block absmax followed by 16 KiB of fp64 partial sums.
-// Host code never touches `g_noalloc_scratch` directly (on the host its name
-// is only a stand-in); each device's real address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// array, 4 MiB of fp32 block absmax followed by the mean's run sums and
+// ticket for 2^20 blocks (2.25 KiB). Host code never touches `g_noalloc_scratch`
+// directly (on the host its name is only a stand-in); the current context's
+// address comes from cudaGetSymbolAddress on every call, so a context
+// recreated after cudaDeviceReset gets its own module's address.
 namespace {
 
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 20;  // 64M weights
 constexpr size_t kNoAllocAbsmaxBytes = static_cast<size_t>(kNoAllocMaxBlocks) * 4;
-constexpr size_t kNoAllocTreeBytes = 16 * 1024;
+// sized at compile time for the largest nb; the mean's scratch does not
+// shrink as nb grows, so it covers every nb <= kNoAllocMaxBlocks
+constexpr size_t kNoAllocTreeBytes = dq_mean_scratch_bytes(kNoAllocMaxBlocks);
 constexpr size_t kNoAllocBytes = kNoAllocAbsmaxBytes + kNoAllocTreeBytes;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64] = {};
-
 qlora_status noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
-        if (!p) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress(static scratch)");
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    if (!p) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress(static scratch)");
+    *out = p;
     return QLORA_OK;
 }
 
@@ -1217,8 +1278,6 @@ extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, in
                        " weights; use qlora_quantize_nf4 with a workspace";
         return QLORA_ERR_EXCEEDS_STATIC_SCRATCH;
     }
-    const int64_t nb = N * K / kBlock;
-    if (dq_tree_scratch_doubles(nb) * 8 > kNoAllocTreeBytes) return QLORA_ERR_EXCEEDS_STATIC_SCRATCH;
     if (injected_failure()) return QLORA_ERR_CUDA;
     int sms = 0;
     qlora_status s = device_ready(&sms);
@@ -1227,9 +1286,6 @@ extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, in
     if ((s = noalloc_scratch(&scratch)) != QLORA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* absmax = static_cast<float*>(scratch);
-    double* tree = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + kNoAllocAbsmaxBytes);
-    QLORA_LAUNCH(launch_nf4_encode(W, false, N, K, codes, absmax, tables(), sms, st), 1, "nf4_encode");
-    if (injected_failure()) return QLORA_ERR_CUDA;
-    QLORA_LAUNCH(launch_double_quant(absmax, nb, tree, qabsmax, s2, mean, st), tree_passes(nb) + 1, "double_quant");
-    return QLORA_OK;
+    void* tree = static_cast<unsigned char*>(scratch) + kNoAllocAbsmaxBytes;
+    return quantize_dq(W, false, N, K, codes, qabsmax, s2, mean, absmax, tree, sms, st);
 }

@@ -122,6 +122,17 @@ __device__ __forceinline__ TileCols tile_cols(const FusedArgs& a, int64_t j) {
     return TileCols{0, 0, 0};
 }
 
+// Row and column tile of tile t of a launch (see FusedArgs::pair_order).
+struct TileRC {
+    int64_t m, n;
+};
+__device__ __forceinline__ TileRC tile_rc(const FusedArgs& a, int tiles_n, int64_t t) {
+    const int64_t g = a.tile_first + t;
+    if (!a.pair_order) return TileRC{g / tiles_n, g % tiles_n};
+    const int64_t p = g >> 1;
+    return TileRC{2 * (p / tiles_n) + (g & 1), p % tiles_n};
+}
+
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -165,7 +176,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
     }
     const int tiles_m = static_cast<int>((args.M + kFusedBM - 1) / kFusedBM);
-    const Sched sc{static_cast<int64_t>(tiles_m) * tiles_n * KT, static_cast<int>(gridDim.x), KT};
+    const int64_t tiles = args.tiles > 0 ? args.tiles : static_cast<int64_t>(tiles_m) * tiles_n;
+    const Sched sc{tiles * KT, static_cast<int>(gridDim.x), KT};
     const int cta = blockIdx.x;
     const int rank_steps = args.rank_cols > 0 ? args.rank_steps : 0;
     const uint64_t tmo = args.timeout_ns;
@@ -207,8 +219,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             SegIter<kSplit> it(sc, cta);
             while (!args.stall_producer && !*abort_flag && it.next()) {
                 ++seg;
-                const int64_t m0 = (it.tile / tiles_n) * kFusedBM;
-                const TileCols tc = tile_cols(args, it.tile % tiles_n);
+                const TileRC rc = tile_rc(args, tiles_n, it.tile);
+                const int64_t m0 = rc.m * kFusedBM;
+                const TileCols tc = tile_cols(args, rc.n);
                 const int64_t n0 = tc.n0;
                 const int nk = it.k_hi - it.k_lo;
                 const int steps = nk + (it.owner() ? rank_steps : 0);
@@ -323,8 +336,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         int g = 0, seg = 0;
         SegIter<kSplit> it(sc, cta);
         while (it.next()) {
-            const int64_t m0 = (it.tile / tiles_n) * kFusedBM;
-            const TileCols tc = tile_cols(args, it.tile % tiles_n);
+            const TileRC rc = tile_rc(args, tiles_n, it.tile);
+            const int64_t m0 = rc.m * kFusedBM;
+            const TileCols tc = tile_cols(args, rc.n);
             const int64_t n0 = tc.n0;
             const int nk = it.k_hi - it.k_lo;
             const int steps = nk + (it.owner() ? rank_steps : 0);
@@ -482,6 +496,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // launched as a programmatic dependent, the grid completes only after its
+    // primary (and so after everything that one waited for); otherwise a no-op
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -818,6 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // as in fused_nf4_gemm
 }
 
 template <bool kTransW>
@@ -833,6 +851,7 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
     cfg.gridDim = dim3(static_cast<unsigned>(a.ctas));
     cfg.blockDim = dim3(kFusedThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
+    const int64_t tiles = a.tiles > 0 ? a.tiles : fused_tiles(a.M, fused_tiles_n(a));
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributePriority;
@@ -841,7 +860,7 @@ cudaError_t launch_fused(const CUtensorMap& act, const CUtensorMap& codes, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    if (static_cast<int64_t>(a.ctas) == fused_tiles(a.M, fused_tiles_n(a)))
+    if (static_cast<int64_t>(a.ctas) == tiles)
         return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, false>, act, codes, cT, lact, lw, a, tab);
     return cudaLaunchKernelEx(&cfg, fused_nf4_gemm<kTransW, true>, act, codes, cT, lact, lw, a, tab);
 }
@@ -854,8 +873,10 @@ cudaError_t launch_pair(const CUtensorMap& act, const CUtensorMap& codes, const 
     cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (e != cudaSuccess) return e;
     const int64_t tiles_m = (a.M + kFusedBM - 1) / kFusedBM;
+    if (a.ctas <= 0 || (a.ctas & 1) || a.ctas > 2 * fused_tiles_n(a) * ((tiles_m + 1) / 2) || a.tile_first != 0)
+        return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * fused_tiles_n(a) * ((tiles_m + 1) / 2)));
+    cfg.gridDim = dim3(static_cast<unsigned>(a.ctas));
     cfg.blockDim = dim3(kFusedThreads);
     cfg.dynamicSmemBytes = kPSmemBytes;
     cfg.stream = st;

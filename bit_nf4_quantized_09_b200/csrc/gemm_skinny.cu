@@ -33,10 +33,12 @@ namespace {
 
 constexpr uint32_t kABytes = 128 * 64 * 2;  // 16 KB
 constexpr uint32_t kBBytes = 64 * 64 * 2;   // up to 64 x 64 bf16
-constexpr uint32_t kStage = kABytes + kBBytes;
+constexpr uint32_t kStage = kABytes + kBBytes;  // per 64-deep chunk of a stage
 constexpr uint32_t kTmemCols = 64;
 constexpr uint32_t kRowBytes = 256;  // one fp32 accumulator row of 64 columns in the reduction buffer
-__host__ __device__ constexpr uint32_t smem_bytes(int stages) { return stages * kStage + 256 + 1024; }
+__host__ __device__ constexpr uint32_t smem_bytes(int stages, int chunks) {
+    return stages * chunks * kStage + 256 + 1024;
+}
 
 // Shared-memory descriptor of an MN-major B tile [64 reduction rows, NR
 // columns] written by TMA with the swizzle whose span is NR * 2 bytes: rows of
@@ -53,8 +55,6 @@ __device__ __forceinline__ uint64_t mn_b_desc(uint32_t addr, int NR) {
     return d;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
 __global__ void __launch_bounds__(kSkinnyThreads, 1)
     skinny_gemm(const __grid_constant__ SkinnyMaps maps, const __grid_constant__ SkinnyArgs args) {
     // a launch that depends on this one programmatically may be scheduled
@@ -69,8 +69,9 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int stages = args.stages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * kStage);
+    const int stages = args.stages, C = args.chunks;
+    const uint32_t stage_bytes = static_cast<uint32_t>(C) * kStage;  // C A chunks, then C B chunks
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
     uint64_t* empty = full + kSkinnyMaxStages;
     uint64_t* acc = empty + kSkinnyMaxStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc + 1);
@@ -78,10 +79,12 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NR = args.NR;
-    const int KT = static_cast<int>((P.red + 63) / 64);
-    const int k_begin = blockIdx.y * P.steps_per_split;
-    const int k_end = min(k_begin + P.steps_per_split, KT);
-    const int steps = max(k_end - k_begin, 0);
+    // the splits interleave: split y takes steps y, y + S, y + 2S, ... (of C
+    // chunks each), so the cluster's CTAs read neighbouring pieces of each row
+    // at the same time
+    const int KT = static_cast<int>((P.red + 64 * C - 1) / (64 * C));
+    const int S = args.splits, y = static_cast<int>(blockIdx.y);
+    const int steps = y < KT ? (KT - y + S - 1) / S : 0;
     const uint64_t tmo = args.timeout_ns;
     const uint32_t b_bytes = static_cast<uint32_t>(NR) * 128u;
 
@@ -118,20 +121,28 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                     break;
                 }
                 if (*abort_flag) break;
-                const int k = (k_begin + i) * 64;
-                uint8_t* st = smem + s * kStage;
-                mbar_arrive_expect_tx(full + s, kABytes + b_bytes);
+                uint8_t* st = smem + s * stage_bytes;
+                mbar_arrive_expect_tx(full + s, static_cast<uint32_t>(C) * (kABytes + b_bytes));
                 const int ar = static_cast<int>(row0);
-                if (!P.a_mn_major) {
-                    tma_load_2d(st, ta, full + s, k, ar);
-                } else {
-                    tma_load_2d(st, ta, full + s, ar, k);
-                    tma_load_2d(st + 8192, ta, full + s, ar + 64, k);
+                // the A chunks first, back to back: C * 128 contiguous bytes of each row in flight together
+                for (int j = 0; j < C; ++j) {
+                    const int k = ((i * S + y) * C + j) * 64;
+                    uint8_t* sa = st + j * kABytes;
+                    if (!P.a_mn_major) {
+                        tma_load_2d(sa, ta, full + s, k, ar);
+                    } else {
+                        tma_load_2d(sa, ta, full + s, ar, k);
+                        tma_load_2d(sa + 8192, ta, full + s, ar + 64, k);
+                    }
                 }
-                if (!P.b_mn_major)
-                    tma_load_2d(st + kABytes, tb, full + s, k, 0);
-                else
-                    tma_load_2d(st + kABytes, tb, full + s, 0, k);
+                for (int j = 0; j < C; ++j) {
+                    const int k = ((i * S + y) * C + j) * 64;
+                    uint8_t* sb = st + C * kABytes + j * kBBytes;
+                    if (!P.b_mn_major)
+                        tma_load_2d(sb, tb, full + s, k, 0);
+                    else
+                        tma_load_2d(sb, tb, full + s, 0, k);
+                }
                 last = i;
             }
             // every copy in flight has landed before the stages are reused
@@ -148,14 +159,17 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
                 const uint32_t u = static_cast<uint32_t>(i / stages);
                 if (!mbar_wait(full + s, u & 1u, tmo, args.status)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t a = smem_u32(smem + s * kStage), b = a + kABytes;
+                const uint32_t st = smem_u32(smem + s * stage_bytes);
+                for (int j = 0; j < C; ++j) {
+                    const uint32_t a = st + j * kABytes, b = st + C * kABytes + j * kBBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t adesc = P.a_mn_major ? sw128_desc(a + kk * 2048, 8192, 1024)
-                                                        : sw128_desc(a + kk * 32, 16, 1024);
-                    const uint64_t bdesc = P.b_mn_major ? mn_b_desc(b + kk * 16 * NR * 2, NR)
-                                                        : sw128_desc(b + kk * 32, 16, 1024);
-                    umma_f16(tmem, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t adesc = P.a_mn_major ? sw128_desc(a + kk * 2048, 8192, 1024)
+                                                            : sw128_desc(a + kk * 32, 16, 1024);
+                        const uint64_t bdesc = P.b_mn_major ? mn_b_desc(b + kk * 16 * NR * 2, NR)
+                                                            : sw128_desc(b + kk * 32, 16, 1024);
+                        umma_f16(tmem, adesc, bdesc, idesc, (i > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 umma_commit(empty + s);
             }
@@ -205,7 +219,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
     // the chunks of a row on neighbouring threads, the transposed output the
     // rows of a chunk.
     {
-        const int S = args.splits;
         const int rank = static_cast<int>(cluster_ctarank());
         const int rows_per = 128 / S, chunks = NR / 4;
         const bool by_row = P.mode == kSkinnyOutF32Transposed;
@@ -261,19 +274,22 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1)
 
 }  // namespace
 
-size_t skinny_smem_bytes(int stages) { return smem_bytes(stages); }
+size_t skinny_smem_bytes(int stages, int chunks) { return smem_bytes(stages, chunks); }
 
 cudaError_t launch_skinny(const SkinnyMaps& maps, const SkinnyArgs& args, int nproblems, cudaStream_t st, bool pdl) {
     if (nproblems < 1 || nproblems > kSkinnyMaxProblems) return cudaErrorInvalidValue;
     const int S = args.splits;
     if (S != 1 && S != 2 && S != 4 && S != 8) return cudaErrorInvalidValue;
-    if (args.stages < 2 || args.stages > kSkinnyMaxStages) return cudaErrorInvalidValue;  // the buffer needs 32 KB
+    // the reduction buffer (32 KB) lies in the stages
+    if (args.chunks != 1 && args.chunks != 2 && args.chunks != 4) return cudaErrorInvalidValue;
+    if (args.stages < 1 || args.stages * args.chunks < 2 || args.stages * args.chunks > kSkinnyMaxStages)
+        return cudaErrorInvalidValue;
     int64_t max_tiles = 0;
     for (int p = 0; p < nproblems; ++p) max_tiles = std::max<int64_t>(max_tiles, (args.p[p].rows + 127) / 128);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(max_tiles), static_cast<unsigned>(S), static_cast<unsigned>(nproblems));
     cfg.blockDim = dim3(kSkinnyThreads);
-    cfg.dynamicSmemBytes = smem_bytes(args.stages);
+    cfg.dynamicSmemBytes = smem_bytes(args.stages, args.chunks);
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -289,7 +305,7 @@ cudaError_t launch_skinny(const SkinnyMaps& maps, const SkinnyArgs& args, int np
 
 cudaError_t skinny_init_device() {
     return cudaFuncSetAttribute(skinny_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem_bytes(kSkinnyMaxStages)));
+                                static_cast<int>(smem_bytes(kSkinnyMaxStages, 1)));
 }
 
 }  // namespace qlora

@@ -20,12 +20,21 @@ struct BlockConstants {
 };
 
 // ----------------------------------------------------------- quantisation --
-// W: fp32 [N, K], or bf16 [N, K] when bf16 is true.
+// W: fp32 [N, K], or bf16 [N, K] when bf16 is true. zero_word: a word the
+// encoder sets to zero (the mean kernel's ticket), or nullptr.
 cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
-                              const Nf4Tables& tab, int num_sms, cudaStream_t st);
-size_t dq_tree_scratch_doubles(int64_t nb);
-cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,
-                                float* mean, cudaStream_t st);
+                              int* zero_word, const Nf4Tables& tab, int num_sms, cudaStream_t st);
+// The double quantisation's mean: the fp64 pairwise tree over the nb
+// constants (zero-padded to a power of two), built from aligned runs of 4096
+// by one launch. Scratch (16-byte aligned): the runs' fp64 sums, then the
+// launch's ticket (dq_mean_ticket), which must be zero before it.
+constexpr size_t dq_mean_scratch_bytes(int64_t nb) { return ((nb + 4095) / 4096 * 8 + 255) / 256 * 256 + 256; }
+int* dq_mean_ticket(void* scratch, int64_t nb);
+cudaError_t launch_dq_mean(const float* absmax, int64_t nb, void* scratch, float* mean, cudaStream_t st);
+// The E4M3 codes and second-level scales of the centred constants (after the
+// encoder has written absmax and the mean).
+cudaError_t launch_dq_groups(const float* absmax, int64_t nb, const float* mean, uint8_t* q, float* s2,
+                             cudaStream_t st);
 // out_map: the bf16 output viewed as [N*K/64 rows, 64], box {64, 128}, SW128.
 constexpr size_t kDequantSmem = 2 * 128 * 128 + 1024;
 cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const BlockConstants& c, int64_t N,
@@ -65,7 +74,15 @@ struct FusedArgs {
     int ngroups;
     int64_t group_end[kMaxGroups];
     int group_rank_x[kMaxGroups];
-    int ctas;           // CTAs (ranges of (tile, step) units): fused_ctas()
+    int ctas;           // CTAs (ranges of (tile, step) units): fused_ctas(); pair launches: 2 * pairs
+    // Tiles of this launch: ids [tile_first, tile_first + tiles) (tiles = 0:
+    // all of them). With pair_order, id 2p + h is row tile 2 (p / tiles_n) + h
+    // of column tile p % tiles_n, the order the CTA-pair launch takes them in,
+    // so a stream-K launch can finish the tiles a shorter pair launch left;
+    // otherwise id t is row tile t / tiles_n of column tile t % tiles_n.
+    int64_t tile_first;
+    int64_t tiles;
+    int pair_order;
     uint16_t* out;      // bf16 [M, out_cols]
     float* part;        // fp32 [fused_partial_ctas()][256][256] partial tiles of contributing CTAs
     int* flags;         // [fused_partial_ctas()] partial-ready flags, zero before the launch
@@ -99,6 +116,12 @@ inline int fused_ctas(int64_t M, int64_t tiles_n, int64_t red, int max_ctas) {
 inline int fused_partial_ctas(int64_t M, int64_t tiles_n, int64_t red, int max_ctas) {
     return fused_tiles(M, tiles_n) >= max_ctas ? 0 : fused_ctas(M, tiles_n, red, max_ctas);
 }
+// CTAs of a stream-K launch over `tiles` tiles (split when fewer than max_ctas).
+inline int fused_ctas_for(int64_t tiles, int64_t red, int max_ctas) {
+    if (tiles >= max_ctas) return static_cast<int>(tiles);
+    const int64_t units = tiles * ((red + kFusedBK - 1) / kFusedBK);
+    return static_cast<int>(units < max_ctas ? units : max_ctas);
+}
 
 // Forward: out = A_op . deq(W)^T + lora_a . lora_b^T, A_op = X [M, K].
 // Maps: act {K, M} box {64, 256} SW128; codes {K/2, N} box {32, 256} SW32;
@@ -121,7 +144,8 @@ cudaError_t launch_fused_dx(const CUtensorMap& act, const CUtensorMap& codes, co
 
 // CTA-pair forms of the two launches (whole tiles, clusters of two CTAs along
 // M that share each dequantised weight tile; each CTA decodes its half). The
-// grid is 2 * (column tiles) * ceil(row tiles / 2).
+// grid is a.ctas: 2 per pair, pairs 0 .. a.ctas / 2 - 1 of the pair order
+// (at most ceil(row tiles / 2) * column tiles).
 // Maps as above except: forward codes box {32, 128}, cT box {128, 1}; dX
 // codes box {64, 64} SW64, cT box {64, 2}.
 cudaError_t launch_fused_pair_fwd(const CUtensorMap& act, const CUtensorMap& codes_half, const CUtensorMap& cT_half,
@@ -180,9 +204,9 @@ cudaError_t launch_gemv_mma(const CUtensorMap& codes, const CUtensorMap& x, cons
 // the fp32 partials in split order and writes the output. Up to
 // kSkinnyMaxProblems independent problems share one launch (blockIdx.z): the
 // 64-column chunks of a wider rank, or the gradients of several adapters.
-constexpr int kSkinnyMaxStages = 8;  // 24 KB each
+constexpr int kSkinnyMaxStages = 8;  // stages x chunks: 24 KB each
 constexpr int kSkinnyThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
-size_t skinny_smem_bytes(int stages);
+size_t skinny_smem_bytes(int stages, int chunks);
 cudaError_t skinny_init_device();
 
 constexpr int kSkinnyOutBf16 = 0;           // out_bf16[row * out_ld + j] = bf16(scale * D)
@@ -193,7 +217,6 @@ constexpr int kSkinnyMaxProblems = 8;
 struct SkinnyProblem {
     int64_t rows;        // output rows (tiles of 128)
     int64_t red;         // reduction length (steps of 64)
-    int steps_per_split; // reduction steps of each of the launch's splits
     int a_mn_major;      // A_op rows-contiguous: two 64-wide TMA boxes per step
     int b_mn_major;      // B_op stored [red, NR] (box {NR, 64}, swizzle = NR*2 bytes)
     int mode;            // kSkinnyOut*
@@ -213,7 +236,8 @@ struct SkinnyProblem {
 struct SkinnyArgs {
     int NR;              // 16, 32 or 64: UMMA N of every problem
     int splits;          // reduction splits = cluster size along grid.y: 1, 2, 4 or 8
-    int stages;          // pipeline stages, 2 .. kSkinnyMaxStages
+    int stages;          // pipeline stages; stages * chunks in 2 .. kSkinnyMaxStages
+    int chunks;          // 64-deep reduction chunks per stage: 1, 2 or 4
     SkinnyProblem p[kSkinnyMaxProblems];
     int* status;
     uint64_t timeout_ns;

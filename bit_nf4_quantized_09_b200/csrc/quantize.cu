@@ -90,8 +90,9 @@ __device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float (&v)[8]) {
 template <bool kBf16>
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const void* __restrict__ W, int64_t nblocks,
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
-                                                         Nf4Tables tab) {
+                                                         Nf4Tables tab, int* __restrict__ zero_word) {
     __shared__ float2 sLut[kCells * kCellCopies];
+    if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;  // the mean kernel's ticket
     for (int j = threadIdx.x; j < kCells; j += blockDim.x) {
         const float lo = (static_cast<float>(j) - 64.5f) * 0.015625f, hi = lo + 0.015625f;  // exact
         int below = 0;
@@ -157,13 +158,10 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const void* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// K2a: fp64 sum of the constants by the stride-doubling pairwise tree.
-// Each CTA of 1024 threads reduces one aligned run of 1024 values; lane l
-// holds value l of its warp and `x += shfl_down(x, s)` for s = 1, 2, 4, 8, 16
-// leaves in lane 0 exactly the tree ((x0 + x1) + (x2 + x3)) + ...; the same
-// step then runs over the 32 warp sums. Runs of a power-of-two length nest, so
-// repeating the pass over the run sums reproduces the tree over all values
-// (zero-padded to a power of two).
+// The fp64 pairwise tree over 1024 values, one per thread: lane l holds value
+// l of its warp and `x += shfl_down(x, s)` for s = 1, 2, 4, 8, 16 leaves in
+// lane 0 exactly the tree ((x0 + x1) + (x2 + x3)) + ...; the same step then
+// runs over the 32 warp sums. The result is valid in thread 0.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ double tree_sum_1024(double x, double* warp_sums) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -180,25 +178,55 @@ __device__ __forceinline__ double tree_sum_1024(double x, double* warp_sums) {
     return y;  // valid in thread 0
 }
 
-__global__ void __launch_bounds__(1024) dq_tree_pass_f32(const float* __restrict__ in, int64_t n,
-                                                          double* __restrict__ out) {
-    __shared__ double ws[32];
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
-    const double x = (i < n) ? static_cast<double>(in[i]) : 0.0;
-    const double s = tree_sum_1024(x, ws);
-    if (threadIdx.x == 0) out[blockIdx.x] = s;
-}
 
-__global__ void __launch_bounds__(1024) dq_tree_pass_f64(const double* __restrict__ in, int64_t n,
-                                                          double* __restrict__ out, int64_t count_for_mean,
-                                                          float* __restrict__ mean_out) {
+// K2a: the mean's fp64 pairwise tree (over the nb constants, zero-padded to a
+// power of two). Its subtrees over aligned runs nest: a CTA of 1024 threads
+// sums one aligned run of 4096 constants, thread i the four 4i .. 4i + 3 as
+// (c0 + c1) + (c2 + c3), then the 1024 values by tree_sum_1024; the last CTA
+// to finish (an atomic ticket that the encoder has set to zero) sums the run
+// sums 1024 at a time, level by level, and writes mean = fp32(sum / nb).
+__global__ void __launch_bounds__(1024) dq_mean_kernel(const float* __restrict__ absmax, int64_t nb,
+                                                        double* __restrict__ run_sums, int* __restrict__ ticket,
+                                                        float* __restrict__ mean) {
     __shared__ double ws[32];
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x;
-    const double x = (i < n) ? in[i] : 0.0;
+    __shared__ int last;
+    const int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x) * 4;
+    float4 f;
+    if (b0 + 3 < nb) {
+        f = __ldcs(reinterpret_cast<const float4*>(absmax + b0));
+    } else {
+        f.x = b0 < nb ? absmax[b0] : 0.0f;
+        f.y = b0 + 1 < nb ? absmax[b0 + 1] : 0.0f;
+        f.z = b0 + 2 < nb ? absmax[b0 + 2] : 0.0f;
+        f.w = 0.0f;  // b0 + 3 >= nb
+    }
+    const double x = (static_cast<double>(f.x) + static_cast<double>(f.y)) +
+                     (static_cast<double>(f.z) + static_cast<double>(f.w));
     const double s = tree_sum_1024(x, ws);
     if (threadIdx.x == 0) {
-        out[blockIdx.x] = s;
-        if (mean_out) *mean_out = __double2float_rn(__ddiv_rn(s, static_cast<double>(count_for_mean)));
+        run_sums[blockIdx.x] = s;
+        __threadfence();  // the run sum, before the ticket
+        last = atomicAdd(ticket, 1) == static_cast<int>(gridDim.x) - 1;
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();  // every run sum, filed before its ticket
+    double total = s;
+    for (int64_t n = gridDim.x; n > 1; n = (n + 1023) / 1024) {
+        // level: node c sums run_sums[1024 c .. 1024 c + 1023] into run_sums[c]
+        for (int64_t c = 0; c * 1024 < n; ++c) {
+            const int64_t i = c * 1024 + threadIdx.x;
+            const double v = i < n ? __ldcg(run_sums + i) : 0.0;
+            total = tree_sum_1024(v, ws);  // thread 0; ends its reads before the barrier below
+            __syncthreads();
+            if (threadIdx.x == 0) run_sums[c] = total;
+            __syncthreads();
+        }
+        __threadfence_block();
+    }
+    if (threadIdx.x == 0) {
+        *mean = __double2float_rn(__ddiv_rn(total, static_cast<double>(nb)));
+        *ticket = 0;
     }
 }
 
@@ -355,20 +383,62 @@ __global__ void __launch_bounds__(256) decode_constants_t_kernel(const uint8_t* 
                                                                   const float* __restrict__ absmax, int64_t N,
                                                                   int64_t KB, int64_t ldc, int64_t cols,
                                                                   float* __restrict__ cT) {
-    __shared__ float tile[32][33];
+    // a CTA takes 64 rows n by 64 block columns kb; thread t decodes the 16
+    // constants of row n0 + t / 4, block columns kb0 + 16 (t % 4) .. + 15
+    // (one 16-byte load of E4M3 codes, or four of fp32 absmax, when the row's
+    // constants are 16-aligned) into a padded shared tile, which leaves as
+    // float4 stores of four consecutive n per block column
+    __shared__ float tile[64][65];
     const float mu = kNoDq ? 0.0f : *mean;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 32, kb0 = static_cast<int64_t>(blockIdx.x) * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-    for (int i = ty; i < 32; i += 8) {
-        const int64_t n = n0 + i, kb = kb0 + tx;
-        float c = 0.0f;
-        if (n < N && kb < KB) c = kNoDq ? absmax[n * KB + kb] : decode_constant(q, s2, mu, n * KB + kb);
-        tile[i][tx] = c;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 64, kb0 = static_cast<int64_t>(blockIdx.x) * 64;
+    const int t = threadIdx.x, nl = t >> 2, k16 = (t & 3) * 16;
+    const int64_t n = n0 + nl;
+    float c[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) c[j] = 0.0f;
+    if (n < N) {
+        const int64_t base = n * KB + kb0 + k16;
+        if ((KB & 15) == 0 && kb0 + k16 < KB) {
+            // 16 whole constants, in one group of 256 (base is a multiple of 16)
+            if (kNoDq) {
+                const float4* src = reinterpret_cast<const float4*>(absmax + base);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = src[i];
+                    c[4 * i] = v.x, c[4 * i + 1] = v.y, c[4 * i + 2] = v.z, c[4 * i + 3] = v.w;
+                }
+            } else {
+                const uint4 w = *reinterpret_cast<const uint4*>(q + base);
+                const float sg = s2[base / kGroup];
+                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    c[i] = __fmaf_rn(e4m3_to_f32(static_cast<uint8_t>(words[i >> 2] >> (8 * (i & 3)))), sg, mu);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int64_t kb = kb0 + k16 + j;
+                if (kb < KB) c[j] = kNoDq ? absmax[n * KB + kb] : decode_constant(q, s2, mu, n * KB + kb);
+            }
+        }
     }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) tile[k16 + j][nl] = c[j];
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int64_t kb = kb0 + i, n = n0 + tx;
-        if (kb < KB && n < cols) cT[kb * ldc + n] = (n < N) ? tile[tx][i] : 0.0f;
+    // cols is a multiple of 4, as are ldc and the rows' offset, so each
+    // float4 lies inside the written range and is 16-byte aligned
+    for (int i = t; i < 64 * 16; i += 256) {
+        const int kl = i >> 4, n4 = (i & 15) * 4;
+        const int64_t kb = kb0 + kl, nn = n0 + n4;
+        if (kb < KB && nn < cols) {
+            float4 v;
+            v.x = nn < N ? tile[kl][n4] : 0.0f;
+            v.y = nn + 1 < N ? tile[kl][n4 + 1] : 0.0f;
+            v.z = nn + 2 < N ? tile[kl][n4 + 2] : 0.0f;
+            v.w = nn + 3 < N ? tile[kl][n4 + 3] : 0.0f;
+            *reinterpret_cast<float4*>(cT + kb * ldc + nn) = v;
+        }
     }
 }
 
@@ -403,56 +473,36 @@ static int grid_for(int64_t work_items, int threads, int max_ctas) {
 }
 
 cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
-                              const Nf4Tables& tab, int num_sms, cudaStream_t st) {
+                              int* zero_word, const Nf4Tables& tab, int num_sms, cudaStream_t st) {
     const int64_t nb = N * K / kBlock;
     const int grid = grid_for(nb * 8, 256, num_sms * 8);
     if (bf16)
-        nf4_encode_kernel<true><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab);
+        nf4_encode_kernel<true><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab,
+                                                       zero_word);
     else
-        nf4_encode_kernel<false><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab);
+        nf4_encode_kernel<false><<<grid, 256, 0, st>>>(W, nb, reinterpret_cast<uint32_t*>(codes), absmax, tab,
+                                                        zero_word);
     return cudaGetLastError();
 }
 
-size_t dq_tree_scratch_doubles(int64_t nb) {
-    // pass outputs, ping-ponged: ceil(nb/1024) + ceil(nb/1024^2) + ...
-    size_t total = 0;
-    int64_t n = nb;
-    do {
-        n = (n + 1023) / 1024;
-        total += static_cast<size_t>(n);
-    } while (n > 1);
-    return total + 1;  // + the slot of the final single-value pass
+int* dq_mean_ticket(void* scratch, int64_t nb) {
+    return reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + dq_mean_scratch_bytes(nb) - 256);
 }
 
-cudaError_t launch_double_quant(const float* absmax, int64_t nb, double* tree_scratch, uint8_t* q, float* s2,
-                                float* mean, cudaStream_t st) {
-    // pass 1 over the fp32 constants, further passes over fp64 run sums
-    int64_t n = (nb + 1023) / 1024;
-    double* cur = tree_scratch;
-    dq_tree_pass_f32<<<static_cast<unsigned>(n), 1024, 0, st>>>(absmax, nb, cur);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (n == 1) {
-        dq_tree_pass_f64<<<1, 1024, 0, st>>>(cur, 1, cur + 1, nb, mean);
-    } else {
-        while (n > 1) {
-            const int64_t m = (n + 1023) / 1024;
-            double* nxt = cur + n;
-            dq_tree_pass_f64<<<static_cast<unsigned>(m), 1024, 0, st>>>(cur, n, nxt, nb,
-                                                                          m == 1 ? mean : nullptr);
-            e = cudaGetLastError();
-            if (e != cudaSuccess) return e;
-            cur = nxt;
-            n = m;
-        }
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+cudaError_t launch_dq_mean(const float* absmax, int64_t nb, void* scratch, float* mean, cudaStream_t st) {
+    const int64_t runs = (nb + 4095) / 4096;
+    if (runs > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    dq_mean_kernel<<<static_cast<unsigned>(runs), 1024, 0, st>>>(absmax, nb, static_cast<double*>(scratch),
+                                                                  dq_mean_ticket(scratch, nb), mean);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dq_groups(const float* absmax, int64_t nb, const float* mean, uint8_t* q, float* s2,
+                             cudaStream_t st) {
     const int64_t ng = (nb + kGroup - 1) / kGroup;
     dq_groups_kernel<<<static_cast<unsigned>((ng * 32 + 255) / 256), 256, 0, st>>>(absmax, nb, mean, q, s2);
     return cudaGetLastError();
 }
-
 cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const BlockConstants& c, int64_t N,
                                int64_t K, const Nf4Tables& tab, int num_sms, cudaStream_t st) {
     const int64_t nb = N * K / kBlock;
@@ -471,7 +521,8 @@ cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes,
 cudaError_t launch_decode_constants_t(const BlockConstants& c, int64_t N, int64_t K, int64_t ldc, int64_t cols,
                                       float* cT, cudaStream_t st) {
     const int64_t KB = K / kBlock;
-    dim3 grid(static_cast<unsigned>((KB + 31) / 32), static_cast<unsigned>((cols + 31) / 32));
+    if ((cols & 3) || (ldc & 3) || (reinterpret_cast<uintptr_t>(cT) & 15)) return cudaErrorInvalidValue;
+    dim3 grid(static_cast<unsigned>((KB + 63) / 64), static_cast<unsigned>((cols + 63) / 64));
     if (c.absmax)
         decode_constants_t_kernel<true><<<grid, 256, 0, st>>>(nullptr, nullptr, nullptr, c.absmax, N, KB, ldc, cols, cT);
     else

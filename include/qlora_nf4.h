@@ -133,19 +133,21 @@ qlora_status qlora_quantize_nf4_bf16(const uint16_t* W, int64_t N, int64_t K,
  * block or synchronise the device in the middle of a step. The pages about
  * QLoRA have no counterpart to this call; it exists only for such callers.
  *   - It takes no workspace and allocates nothing. Its scratch (the fp32
- *     per-block absmax and the fp64 partial sums of the mean) lives in one
- *     static device array of 4 MiB + 16 KiB that every GPU which loads the
- *     library keeps until the process exits.
+ *     per-block absmax, the fp64 partial sums of the mean and a ticket)
+ *     lives in one static device array of 4 MiB + 2.25 KiB that every GPU
+ *     which loads the library keeps until the process exits.
  *   - Limit: N*K <= 67,108,864 weights (at most 1,048,576 blocks of 64, e.g.
  *     8192 x 8192). Larger weights return QLORA_ERR_EXCEEDS_STATIC_SCRATCH
  *     and launch nothing; use qlora_quantize_nf4 with a workspace instead.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
+ *   - Every call looks up the array's address in the current context
+ *     (cudaGetSymbolAddress); the first call on a device, and the first after
+ *     a cudaDeviceReset, also loads the library's module there, so make it
  *     before any stream capture on the device.
  *   - All calls share the one array: calls that overlap on the GPU (for
  *     example on two streams at once) race and corrupt each other's results.
  *     Calls in one stream are ordered and safe; nothing in the array has to
- *     start at zero, every byte read is written earlier in the same call.
+ *     start at zero, every byte read is written earlier in the same call
+ *     (the ticket by the encoder).
  *   - Outputs, argument checks and determinism are those of
  *     qlora_quantize_nf4. */
 qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t N, int64_t K,
@@ -315,6 +317,12 @@ const char* qlora_last_error(void);
                                         fused matmuls run in CTA pairs sharing
                                         each dequantised weight tile; 0: one
                                         CTA per tile, each decoding its own */
+#define QLORA_OPT_FUSED_TAIL      9  /* 1: when the last wave of CTA pairs
+                                        would be short, its tiles run on the
+                                        one-CTA kernel split over every SM
+                                        (stream-K, fp32 partial tiles added in
+                                        a fixed order); 0 (default): whole
+                                        waves of pairs only */
 qlora_status qlora_set_option(int option, int64_t value);
 int64_t qlora_get_option(int option);
 

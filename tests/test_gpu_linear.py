@@ -296,6 +296,10 @@ def test_fused_split_tiles_deterministic(q):
 
 PAIRS = [synth.custom(N=256 * 150 + 8, K=320, M=600, r=16),     # forward: 3 x 151 tiles, odd row tiles
          synth.custom(N=320, K=256 * 150 + 64, M=520, r=32)]    # dX: 3 x 151 tiles, ragged output columns
+# On 148 SMs, with the stream-K tail switched on, both cases run 592 tiles as
+# four whole waves of pairs and the last 12 (of 2 x 151 pair tiles, the row
+# tile past M included) on the one-CTA kernel, every tile split over five CTAs
+# (five reduction steps).
 
 
 @pytest.mark.parametrize("cfg", PAIRS, ids=lambda c: c.name)
@@ -312,13 +316,50 @@ def test_fused_pairs_match_single_cta_bits(q, cfg):
     """The pair kernel runs the same UMMAs on the same decoded operands as the
     one-CTA-per-tile kernel: identical bits, including the adapter gradients."""
     t = inputs(cfg)
-    old = q.get_option(q.OPT_FUSED_PAIRS)
+    old, old_tail = q.get_option(q.OPT_FUSED_PAIRS), q.get_option(q.OPT_FUSED_TAIL)
     try:
+        q.set_option(q.OPT_FUSED_TAIL, 0)  # whole waves of pairs: no tile split
         q.set_option(q.OPT_FUSED_PAIRS, 1)
         a = gpu_run(q, cfg, t)
         q.set_option(q.OPT_FUSED_PAIRS, 0)
         b = gpu_run(q, cfg, t)
     finally:
         q.set_option(q.OPT_FUSED_PAIRS, old)
+        q.set_option(q.OPT_FUSED_TAIL, old_tail)
     for k in ("Y", "dX", "dA", "dB"):
         assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("cfg", PAIRS, ids=lambda c: c.name)
+def test_stream_k_tail_after_pairs(q, cfg):
+    """With the tail on, the short last wave of pairs becomes one more launch
+    (the one-CTA kernel, stream-K); the tiles the pairs ran keep their bits
+    and the tail's tiles, whose partial sums are added in another order, agree
+    with the whole-tile results to fp32 rounding."""
+    t = inputs(cfg)
+    old_tail = q.get_option(q.OPT_FUSED_TAIL)
+    runs, counts = {}, {}
+    try:
+        for tail in (0, 1):
+            q.set_option(q.OPT_FUSED_TAIL, tail)
+            n0 = q.launch_count()
+            runs[tail] = gpu_run(q, cfg, t)
+            counts[tail] = q.launch_count() - n0
+        full_compare(q, cfg, t)  # the tail on: every output against the oracle
+    finally:
+        q.set_option(q.OPT_FUSED_TAIL, old_tail)
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("tile counts are worked out for 148 SMs")
+    assert counts[1] == counts[0] + 1
+    key = "Y" if cfg.K == 320 else "dX"
+    a, b = runs[1][key], runs[0][key]
+    # pair order: tiles 592..603 are pairs 296..301, row tiles 2 and 3 of the
+    # last six column tiles
+    cols = a.shape[1]
+    c0 = 145 * 256
+    assert torch.equal(a[:, :c0], b[:, :c0])
+    assert torch.equal(a[:512, c0:], b[:512, c0:])
+    ref = b[512:, c0:].float()
+    err = (a[512:, c0:].float() - ref).abs().max().item() / max(ref.abs().max().item(), 1e-30)
+    assert err <= 2 ** -7, err
+    assert cols > c0
