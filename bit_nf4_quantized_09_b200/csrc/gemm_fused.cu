@@ -129,8 +129,8 @@ struct TileRC {
 __device__ __forceinline__ TileRC tile_rc(const FusedArgs& a, int tiles_n, int64_t t) {
     const int64_t g = a.tile_first + t;
     if (!a.pair_order) return TileRC{g / tiles_n, g % tiles_n};
-    const int64_t p = g >> 1;
-    return TileRC{2 * (p / tiles_n) + (g & 1), p % tiles_n};
+    const int64_t p = g >> 1, pairs_m = (a.M + 2 * kFusedBM - 1) / (2 * kFusedBM);
+    return TileRC{2 * (p % pairs_m) + (g & 1), p / pairs_m};
 }
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -558,11 +558,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
             start = args.group_end[g];
         }
     }
-    // the pair's column tile and this CTA's row tile (the second row tile of
-    // the last pair may lie past M: its rows are zero-filled and never written)
+    // the pair's column tile and this CTA's row tile, column-major: the row
+    // pairs of one column tile are neighbours, run in the same wave and share
+    // its packed codes through L2 (the second row tile of the last row pair
+    // may lie past M: its rows are zero-filled and never written)
     const int pair = blockIdx.x >> 1;
-    const int64_t m0 = (static_cast<int64_t>(pair / tiles_n) * 2 + rank) * kFusedBM;
-    const TileCols tc = tile_cols(args, pair % tiles_n);
+    const int pairs_m = static_cast<int>((args.M + 2 * kFusedBM - 1) / (2 * kFusedBM));
+    const int64_t m0 = (static_cast<int64_t>(pair % pairs_m) * 2 + rank) * kFusedBM;
+    const TileCols tc = tile_cols(args, pair / pairs_m);
     const int64_t n0 = tc.n0;
     const int rank_steps = args.rank_cols > 0 ? args.rank_steps : 0;
     const int steps = KT + rank_steps;

@@ -76,10 +76,11 @@ struct FusedArgs {
     int group_rank_x[kMaxGroups];
     int ctas;           // CTAs (ranges of (tile, step) units): fused_ctas(); pair launches: 2 * pairs
     // Tiles of this launch: ids [tile_first, tile_first + tiles) (tiles = 0:
-    // all of them). With pair_order, id 2p + h is row tile 2 (p / tiles_n) + h
-    // of column tile p % tiles_n, the order the CTA-pair launch takes them in,
-    // so a stream-K launch can finish the tiles a shorter pair launch left;
-    // otherwise id t is row tile t / tiles_n of column tile t % tiles_n.
+    // all of them). With pair_order, id 2p + h is row tile 2 (p % pairs_m) + h
+    // of column tile p / pairs_m (pairs_m = ceil(row tiles / 2)), the order the
+    // CTA-pair launch takes them in, so a stream-K launch can finish the tiles
+    // a shorter pair launch left; otherwise id t is row tile t / tiles_n of
+    // column tile t % tiles_n.
     int64_t tile_first;
     int64_t tiles;
     int pair_order;
