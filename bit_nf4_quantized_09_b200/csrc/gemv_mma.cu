@@ -104,32 +104,34 @@ __device__ __forceinline__ uint32_t lut(uint32_t lane_base, uint32_t w, uint32_t
     return lds32(lane_base + e * 128u);
 }
 
-// sum_{j < cols} sT[j] * B[j] over bf16 operands, fp32 products and sums in
-// order (cols a multiple of 8, both rows 16-byte aligned); the loads of each
-// 32 columns are issued before their first product.
-__device__ __forceinline__ float rank_dot(const uint16_t* sT, const uint16_t* b, int cols) {
-    float acc = 0.0f;
-    for (int c0 = 0; c0 < cols; c0 += 32) {
-        uint4 tv[4], bv[4];
+// The rank-r term of two 8-row halves of a warp's 16 rows, added to the
+// warp's accumulators: for each 16-column rank step, A fragment = the rows'
+// B entries (row g in slots 0 and 2, row g + 8 in slots 1 and 3), X fragment =
+// the tokens' sT entries at the rows' sT columns; columns from `cols` on read
+// as zero. `use_a` / `use_b` keep one half (the other's A slots zero) when the
+// two halves read different sT columns (projections of a group).
+template <int MT>
+__device__ __forceinline__ void rank_mma(const GemvMmaArgs& a, float (&acc)[MT][4], int64_t rowA, int64_t rowB,
+                                         int col, bool use_a, bool use_b, int g, int q) {
+    const int cols = a.rank_cols, M = static_cast<int>(a.M);
+    const uint16_t* bA = a.B + rowA * a.B_ld;
+    const uint16_t* bB = a.B + rowB * a.B_ld;
+    for (int k0 = 0; k0 < cols; k0 += 16) {
+        const int j0 = k0 + 2 * q, j1 = j0 + 8;
+        uint32_t af[4];
+        af[0] = use_a && j0 < cols ? __ldg(reinterpret_cast<const uint32_t*>(bA + j0)) : 0u;
+        af[1] = use_b && j0 < cols ? __ldg(reinterpret_cast<const uint32_t*>(bB + j0)) : 0u;
+        af[2] = use_a && j1 < cols ? __ldg(reinterpret_cast<const uint32_t*>(bA + j1)) : 0u;
+        af[3] = use_b && j1 < cols ? __ldg(reinterpret_cast<const uint32_t*>(bB + j1)) : 0u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool in = c0 + 8 * i < cols;
-            tv[i] = in ? __ldg(reinterpret_cast<const uint4*>(sT + c0) + i) : make_uint4(0u, 0u, 0u, 0u);
-            bv[i] = in ? __ldg(reinterpret_cast<const uint4*>(b + c0) + i) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (c0 + 8 * i >= cols) break;
-            const uint32_t tw[4] = {tv[i].x, tv[i].y, tv[i].z, tv[i].w};
-            const uint32_t bw[4] = {bv[i].x, bv[i].y, bv[i].z, bv[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc = __fmaf_rn(__uint_as_float(tw[j] << 16), __uint_as_float(bw[j] << 16), acc);
-                acc = __fmaf_rn(__uint_as_float(tw[j] & 0xFFFF0000u), __uint_as_float(bw[j] & 0xFFFF0000u), acc);
-            }
+        for (int t = 0; t < MT; ++t) {
+            const int m = min(8 * t + g, M - 1);  // tokens past M: copies, never written
+            const uint16_t* xs = a.sT + static_cast<int64_t>(m) * a.sT_ld + col;
+            const uint32_t x0 = j0 < cols ? __ldg(reinterpret_cast<const uint32_t*>(xs + j0)) : 0u;
+            const uint32_t x1 = j1 < cols ? __ldg(reinterpret_cast<const uint32_t*>(xs + j1)) : 0u;
+            mma_bf16(acc[t], af, x0, x1);
         }
     }
-    return acc;
 }
 
 // Column of sT holding the rank-r input of output row n.
@@ -335,6 +337,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
 
+        // the rank-r term of the warp's rows, added by the CTA whose segment
+        // ends at the tile's last block column (exactly one per tile); the
+        // rows' two 8-row halves each lie inside one projection of a group
+        auto add_rank = [&](int seg) {
+            griddep_wait();  // sT from the preceding launch
+            const int64_t ra = static_cast<int64_t>(t0 + seg) * kRowsCta + warp * 16 + g;
+            const int64_t rA = ra < N ? ra : N - 1, rB = ra + 8 < N ? ra + 8 : N - 1;
+            const int cA = rank_col(a, rA), cB = rank_col(a, rB);  // uniform over the warp
+            if (cA == cB) {
+                rank_mma<MT>(a, acc, rA, rB, cA, true, true, g, q);
+            } else {
+                rank_mma<MT>(a, acc, rA, rB, cA, true, false, g, q);
+                rank_mma<MT>(a, acc, rA, rB, cB, false, true, g, q);
+            }
+        };
+
         bool ok = true;
         for (int k = 0; k < nst && ok; ++k) {
             const int s = k % S;
@@ -385,8 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + s);
-            if (k == nst0 - 1) flush(0);
-            else if (k == nst - 1) flush(1);
+            if (k == nst0 - 1) {
+                if (blo0 + len0 == KB) add_rank(0);
+                flush(0);
+            } else if (k == nst - 1) {
+                if (len1 == KB) add_rank(1);
+                flush(1);
+            }
         }
         if (!ok) abort_flag = 1;
     }
@@ -406,27 +429,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nseg; ++j) {
         if (!last_of[j]) continue;
         __threadfence();  // see the other CTAs' partials
-        griddep_wait();   // sT from the preceding launch
         const int tile = t0 + j;
         const int n0 = tile * kRowsCta;
         const int np = sc.parts(tile);
-        for (int i = threadIdx.x; i < M * kRowsCta; i += kThreads) {
-            const int m = i / kRowsCta, n = n0 + i % kRowsCta;
+        // four consecutive rows of one token per item; every partial of an
+        // item is loaded before the first add (N is a multiple of 8)
+        for (int i = threadIdx.x; i < M * (kRowsCta / 4); i += kThreads) {
+            const int m = i / (kRowsCta / 4), n = n0 + 4 * (i % (kRowsCta / 4));
             if (n >= N) continue;
-            // every load of this output goes out before the first use: the
-            // rank-r operands, then the partials in CTA order, 16 at a time
-            const float lr = rank_dot(a.sT + static_cast<int64_t>(m) * a.sT_ld + rank_col(a, n),
-                                      a.B + static_cast<int64_t>(n) * a.B_ld, a.rank_cols);
-            float s = 0.0f;
-            for (int s0 = 0; s0 < np; s0 += 16) {
-                float v[16];
+            float4 s4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int s0 = 0; s0 < np; s0 += 8) {
+                float4 v[8];
 #pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    v[u] = s0 + u < np ? __ldcg(a.part + (static_cast<int64_t>(s0 + u) * M + m) * N + n) : 0.0f;
+                for (int u = 0; u < 8; ++u)
+                    v[u] = s0 + u < np
+                               ? __ldcg(reinterpret_cast<const float4*>(a.part + (static_cast<int64_t>(s0 + u) * M + m) * N + n))
+                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) s += v[u];
+                for (int u = 0; u < 8; ++u) {
+                    s4.x += v[u].x;
+                    s4.y += v[u].y;
+                    s4.z += v[u].z;
+                    s4.w += v[u].w;
+                }
             }
-            a.Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(s + lr, 0.0f) & 0xFFFFu);
+            *reinterpret_cast<uint2*>(a.Y + static_cast<int64_t>(m) * N + n) =
+                make_uint2(pack_bf16x2(s4.x, s4.y), pack_bf16x2(s4.z, s4.w));
         }
         if (threadIdx.x == 0) a.counter[tile] = 0;  // ready for the next call
     }
