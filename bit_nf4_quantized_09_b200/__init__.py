@@ -267,6 +267,10 @@ def merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
     v = w.c_view()
     _check(lib().qlora_merge_lora(ctypes.byref(v), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                                   _stream(out.device)), "qlora_merge_lora")
+    if _check_device_status:
+        st = call_status(out.device)
+        if st != QLORA_OK:
+            raise QLoraError(st, "qlora_merge_lora", "device status after the call")
     return out
 
 
@@ -461,6 +465,14 @@ def linear_bwd_group(dY: torch.Tensor, X: torch.Tensor, group: list, A: torch.Te
 def device_status(ws: torch.Tensor) -> int:
     out = _int(0)
     _check(lib().qlora_device_status(_ptr(ws), ctypes.byref(out), _stream(ws.device)), "qlora_device_status")
+    return out.value
+
+
+def call_status(device=None) -> int:
+    """Status word of the calls without a workspace (the adapter merge), read
+    and cleared: QLORA_OK, or QLORA_ERR_DEVICE_TIMEOUT after a wait ran out."""
+    out = _int(0)
+    _check(lib().qlora_device_status(None, ctypes.byref(out), _stream(device)), "qlora_device_status")
     return out.value
 
 

@@ -146,7 +146,7 @@ qlora_status device_ready(int* sms_out) {
                            std::to_string(minor) + ")";
             d.status = QLORA_ERR_UNSUPPORTED_DEVICE;
         } else if ((e = fused_init_device()) != cudaSuccess || (e = skinny_init_device()) != cudaSuccess ||
-                   (e = gemv_mma_init_device()) != cudaSuccess) {
+                   (e = gemv_mma_init_device()) != cudaSuccess || (e = merge_tc_init_device()) != cudaSuccess) {
             d.status = cuda_fail(e, "cudaFuncSetAttribute");
         } else if (!g_encode) {
             void* fn = nullptr;
@@ -889,6 +889,10 @@ Weights single_weight(const qlora_nf4_weight* w) {
 
 }  // namespace
 
+// The device word that records bounded waits that ran out in calls without a
+// workspace (defined with the no-allocation quantiser's scratch below).
+qlora_status call_status_word(int** out);
+
 // =================================================================== ABI ==
 
 extern "C" {
@@ -1067,6 +1071,8 @@ qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const uint16_t* A, cons
     if (injected_failure()) return QLORA_ERR_CUDA;
     int sms = 0;
     if ((s = device_ready(&sms)) != QLORA_OK) return s;
+    int* status = nullptr;
+    if ((s = call_status_word(&status)) != QLORA_OK) return s;
     MergeArgs a{};
     a.codes = w->codes;
     a.c = constants_of(w);
@@ -1076,7 +1082,19 @@ qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const uint16_t* A, cons
     a.N = w->N;
     a.K = w->K;
     a.W_out = W_out;
-    QLORA_LAUNCH(launch_merge_lora(a, r, tables(), sms, static_cast<cudaStream_t>(stream)), 1, "merge_lora");
+    a.status = status;
+    a.timeout_ns = timeout_ns();
+    const int64_t N = w->N, K = w->K;
+    CUtensorMap mb, ma, mc;
+    QLORA_MAP(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, r, N, static_cast<uint64_t>(r) * 2, 64, 128,
+              CU_TENSOR_MAP_SWIZZLE_128B, "B");
+    QLORA_MAP(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, r, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, "A");
+    QLORA_MAP(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+              "codes");
+    CUtensorMap mo;
+    QLORA_MAP(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_out, K, N, K * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B, "W_out");
+    QLORA_LAUNCH(launch_merge_tc(mb, ma, mc, mo, a, r, tables(), sms, static_cast<cudaStream_t>(stream)), 1,
+                 "merge_lora");
     return QLORA_OK;
 }
 
@@ -1205,11 +1223,21 @@ qlora_status qlora_linear_bwd_group(const uint16_t* dY, const uint16_t* X, int64
 }
 
 qlora_status qlora_device_status(const void* ws, int* status_host, void* stream) {
-    if (!ws || !status_host) return QLORA_ERR_INVALID_ARG;
+    if (!status_host) return QLORA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int v = 0;
-    QLORA_TRY(cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st), "read status");
-    QLORA_TRY(cudaStreamSynchronize(st), "sync");
+    if (ws) {
+        QLORA_TRY(cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st), "read status");
+        QLORA_TRY(cudaStreamSynchronize(st), "sync");
+    } else {
+        // calls without a workspace: the library's own word, cleared once read
+        int* w = nullptr;
+        const qlora_status s = call_status_word(&w);
+        if (s != QLORA_OK) return s;
+        QLORA_TRY(cudaMemcpyAsync(&v, w, sizeof(int), cudaMemcpyDeviceToHost, st), "read status");
+        QLORA_TRY(cudaMemsetAsync(w, 0, sizeof(int), st), "clear status");
+        QLORA_TRY(cudaStreamSynchronize(st), "sync");
+    }
     *status_host = (v & kStatusTimeout) ? QLORA_ERR_DEVICE_TIMEOUT : (v ? QLORA_ERR_CUDA : QLORA_OK);
     return QLORA_OK;
 }
@@ -1237,6 +1265,20 @@ qlora_status qlora_e4m3_encode(const float* x, uint8_t* q, int64_t n, void* stre
 }  // extern "C"
 
 // ======================================================== no allocation ==
+// The status word of calls without a workspace (the adapter merge): one
+// file-scope device int, read and cleared by qlora_device_status(NULL, ...).
+namespace {
+static __device__ int g_call_status;
+}  // namespace
+
+qlora_status call_status_word(int** out) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_call_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    *out = static_cast<int*>(p);
+    return QLORA_OK;
+}
+
 // Quantiser scratch for callers that cannot allocate: one file-scope device
 // array, 4 MiB of fp32 block absmax followed by the mean's run sums and
 // ticket for 2^20 blocks (2.25 KiB). Host code never touches `g_noalloc_scratch`

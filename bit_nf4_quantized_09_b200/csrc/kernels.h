@@ -269,9 +269,17 @@ struct MergeArgs {
     float scale;           // alpha / r
     int64_t N, K;
     uint16_t* W_out;       // bf16 [N, K]
+    int* status;           // device status word (a bounded wait that ran out)
+    uint64_t timeout_ns;
 };
 
-// W_out = bf16(deq(W) + scale . B . A); r in {8, 16, 32, 64}.
-cudaError_t launch_merge_lora(const MergeArgs& a, int r, const Nf4Tables& tab, int num_sms, cudaStream_t st);
+// W_out = bf16(deq(W) + scale . B . A); r in {8, 16, 32, 64}, on tcgen05.
+// Maps: b_map = B [N, r] bf16 box {64, 128} SW128; a_map = A [r, K] bf16 box
+// {64, 64} SW128; codes_map = codes [N, K/2] uint8 box {128, 128} SW128;
+// out_map = W_out [N, K] bf16 box {64, 32} SW128.
+cudaError_t launch_merge_tc(const CUtensorMap& b_map, const CUtensorMap& a_map, const CUtensorMap& codes_map,
+                            const CUtensorMap& out_map, const MergeArgs& a, int r, const Nf4Tables& tab, int num_sms,
+                            cudaStream_t st);
+cudaError_t merge_tc_init_device();
 
 }  // namespace qlora

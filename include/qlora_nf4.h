@@ -179,7 +179,9 @@ qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, vo
  * exact bf16 products accumulated in fp32 (order unspecified): an entry is
  * off the exact merge by at most one bf16 step plus that fp32 error.
  * A: bf16 [r, K]; B: bf16 [N, r]; W_out: bf16 [N, K] (device, caller-owned);
- * r in {8, 16, 32, 64}. No workspace. Errors as for qlora_linear_fwd. To
+ * r in {8, 16, 32, 64}. No workspace: a device wait that ran out is recorded
+ * in the status word read by qlora_device_status(NULL, ...); other errors as
+ * for qlora_linear_fwd. To
  * store the merged weight in 4 bits again, quantise W_out with
  * qlora_quantize_nf4_bf16 (the update may be lost, as the explainer warns). */
 qlora_status qlora_merge_lora(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
@@ -280,7 +282,9 @@ qlora_status qlora_linear_bwd_group(const uint16_t* dY, const uint16_t* X, int64
 qlora_status qlora_nf4_tables(float* levels_host, float* thresholds_host);
 
 /* Read the device status word at the head of a fwd/bwd workspace (0 = ok,
- * otherwise a QLORA_ERR_DEVICE_* code). Synchronises `stream`. */
+ * otherwise a QLORA_ERR_DEVICE_* code). With ws = NULL it reads, and clears,
+ * the library's own status word of the calls that take no workspace
+ * (qlora_merge_lora) on the current device. Synchronises `stream`. */
 qlora_status qlora_device_status(const void* ws, int* status_host, void* stream);
 
 /* Human-readable name of a status code, and the text of the last CUDA error
