@@ -1281,7 +1281,7 @@ qlora_status call_status_word(int** out) {
 
 // Quantiser scratch for callers that cannot allocate: one file-scope device
 // array, 4 MiB of fp32 block absmax followed by the mean's run sums and
-// ticket for 2^20 blocks (2.25 KiB). Host code never touches `g_noalloc_scratch`
+// ticket for 2^20 blocks (768 B). Host code never touches `g_noalloc_scratch`
 // directly (on the host its name is only a stand-in); the current context's
 // address comes from cudaGetSymbolAddress on every call, so a context
 // recreated after cudaDeviceReset gets its own module's address.

@@ -25,10 +25,14 @@ struct BlockConstants {
 cudaError_t launch_nf4_encode(const void* W, bool bf16, int64_t N, int64_t K, uint8_t* codes, float* absmax,
                               int* zero_word, const Nf4Tables& tab, int num_sms, cudaStream_t st);
 // The double quantisation's mean: the fp64 pairwise tree over the nb
-// constants (zero-padded to a power of two), built from aligned runs of 4096
-// by one launch. Scratch (16-byte aligned): the runs' fp64 sums, then the
-// launch's ticket (dq_mean_ticket), which must be zero before it.
-constexpr size_t dq_mean_scratch_bytes(int64_t nb) { return ((nb + 4095) / 4096 * 8 + 255) / 256 * 256 + 256; }
+// constants (zero-padded to a power of two), built from aligned runs of
+// kMeanRun by one launch. Scratch (16-byte aligned): the runs' fp64 sums, then
+// the launch's ticket (dq_mean_ticket), which must be zero before it.
+constexpr int kMeanPerThread = 16;
+constexpr int64_t kMeanRun = 1024 * kMeanPerThread;  // 16384 constants per CTA
+constexpr size_t dq_mean_scratch_bytes(int64_t nb) {
+    return ((nb + kMeanRun - 1) / kMeanRun * 8 + 255) / 256 * 256 + 256;
+}
 int* dq_mean_ticket(void* scratch, int64_t nb);
 cudaError_t launch_dq_mean(const float* absmax, int64_t nb, void* scratch, float* mean, cudaStream_t st);
 // The E4M3 codes and second-level scales of the centred constants (after the

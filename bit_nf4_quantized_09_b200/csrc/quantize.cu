@@ -91,6 +91,7 @@ template <bool kBf16>
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const void* __restrict__ W, int64_t nblocks,
                                                          uint32_t* __restrict__ codes, float* __restrict__ absmax,
                                                          Nf4Tables tab, int* __restrict__ zero_word) {
+    asm volatile("griddepcontrol.launch_dependents;");  // the mean launch may be scheduled; it waits for this grid
     __shared__ float2 sLut[kCells * kCellCopies];
     if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;  // the mean kernel's ticket
     for (int j = threadIdx.x; j < kCells; j += blockDim.x) {
@@ -181,27 +182,35 @@ __device__ __forceinline__ double tree_sum_1024(double x, double* warp_sums) {
 
 // K2a: the mean's fp64 pairwise tree (over the nb constants, zero-padded to a
 // power of two). Its subtrees over aligned runs nest: a CTA of 1024 threads
-// sums one aligned run of 4096 constants, thread i the four 4i .. 4i + 3 as
-// (c0 + c1) + (c2 + c3), then the 1024 values by tree_sum_1024; the last CTA
-// to finish (an atomic ticket that the encoder has set to zero) sums the run
-// sums 1024 at a time, level by level, and writes mean = fp32(sum / nb).
+// sums one aligned run of 16384 constants, thread i its 16 consecutive ones in
+// tree order (((c0 + c1) + (c2 + c3)) + ...), then the 1024 values by
+// tree_sum_1024; the last CTA to finish (an atomic ticket that the encoder has
+// set to zero) sums the run sums 1024 at a time, level by level, and writes
+// mean = fp32(sum / nb).
 __global__ void __launch_bounds__(1024) dq_mean_kernel(const float* __restrict__ absmax, int64_t nb,
                                                         double* __restrict__ run_sums, int* __restrict__ ticket,
                                                         float* __restrict__ mean) {
     __shared__ double ws[32];
     __shared__ int last;
-    const int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x) * 4;
-    float4 f;
-    if (b0 + 3 < nb) {
-        f = __ldcs(reinterpret_cast<const float4*>(absmax + b0));
-    } else {
-        f.x = b0 < nb ? absmax[b0] : 0.0f;
-        f.y = b0 + 1 < nb ? absmax[b0 + 1] : 0.0f;
-        f.z = b0 + 2 < nb ? absmax[b0 + 2] : 0.0f;
-        f.w = 0.0f;  // b0 + 3 >= nb
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // absmax and the zeroed ticket of the encoder
+    const int64_t b0 = (static_cast<int64_t>(blockIdx.x) * 1024 + threadIdx.x) * kMeanPerThread;
+    double q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t bj = b0 + 4 * j;
+        float4 f;
+        if (bj + 3 < nb) {
+            f = __ldcg(reinterpret_cast<const float4*>(absmax + bj));  // kept in L2 for the group pass
+        } else {
+            f.x = bj < nb ? absmax[bj] : 0.0f;
+            f.y = bj + 1 < nb ? absmax[bj + 1] : 0.0f;
+            f.z = bj + 2 < nb ? absmax[bj + 2] : 0.0f;
+            f.w = 0.0f;  // bj + 3 >= nb
+        }
+        q[j] = (static_cast<double>(f.x) + static_cast<double>(f.y)) + (static_cast<double>(f.z) + static_cast<double>(f.w));
     }
-    const double x = (static_cast<double>(f.x) + static_cast<double>(f.y)) +
-                     (static_cast<double>(f.z) + static_cast<double>(f.w));
+    const double x = (q[0] + q[1]) + (q[2] + q[3]);  // the thread's 16 consecutive constants in tree order
     const double s = tree_sum_1024(x, ws);
     if (threadIdx.x == 0) {
         run_sums[blockIdx.x] = s;
@@ -237,6 +246,7 @@ __global__ void __launch_bounds__(1024) dq_mean_kernel(const float* __restrict__
 __global__ void __launch_bounds__(256) dq_groups_kernel(const float* __restrict__ c, int64_t nb,
                                                          const float* __restrict__ mean, uint8_t* __restrict__ q,
                                                          float* __restrict__ s2) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the mean of the preceding launch
     const int lane = threadIdx.x & 31;
     const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t ng = (nb + kGroup - 1) / kGroup;
@@ -489,19 +499,35 @@ int* dq_mean_ticket(void* scratch, int64_t nb) {
     return reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) + dq_mean_scratch_bytes(nb) - 256);
 }
 
+// programmatic dependent launches: each waits (griddepcontrol.wait) for its
+// predecessor before it reads, so only the launch latency overlaps
+static cudaLaunchConfig_t pdl_config(unsigned grid, unsigned block, cudaStream_t st, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
 cudaError_t launch_dq_mean(const float* absmax, int64_t nb, void* scratch, float* mean, cudaStream_t st) {
-    const int64_t runs = (nb + 4095) / 4096;
+    const int64_t runs = (nb + kMeanRun - 1) / kMeanRun;
     if (runs > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    dq_mean_kernel<<<static_cast<unsigned>(runs), 1024, 0, st>>>(absmax, nb, static_cast<double*>(scratch),
-                                                                  dq_mean_ticket(scratch, nb), mean);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pdl_config(static_cast<unsigned>(runs), 1024, st, attr);
+    return cudaLaunchKernelEx(&cfg, dq_mean_kernel, absmax, nb, static_cast<double*>(scratch),
+                              dq_mean_ticket(scratch, nb), mean);
 }
 
 cudaError_t launch_dq_groups(const float* absmax, int64_t nb, const float* mean, uint8_t* q, float* s2,
                              cudaStream_t st) {
     const int64_t ng = (nb + kGroup - 1) / kGroup;
-    dq_groups_kernel<<<static_cast<unsigned>((ng * 32 + 255) / 256), 256, 0, st>>>(absmax, nb, mean, q, s2);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = pdl_config(static_cast<unsigned>((ng * 32 + 255) / 256), 256, st, attr);
+    return cudaLaunchKernelEx(&cfg, dq_groups_kernel, absmax, nb, static_cast<const float*>(mean), q, s2);
 }
 cudaError_t launch_nf4_dequant(const CUtensorMap& out_map, const uint8_t* codes, const BlockConstants& c, int64_t N,
                                int64_t K, const Nf4Tables& tab, int num_sms, cudaStream_t st) {

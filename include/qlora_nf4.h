@@ -134,7 +134,7 @@ qlora_status qlora_quantize_nf4_bf16(const uint16_t* W, int64_t N, int64_t K,
  * QLoRA have no counterpart to this call; it exists only for such callers.
  *   - It takes no workspace and allocates nothing. Its scratch (the fp32
  *     per-block absmax, the fp64 partial sums of the mean and a ticket)
- *     lives in one static device array of 4 MiB + 2.25 KiB that every GPU
+ *     lives in one static device array of 4 MiB + 768 B that every GPU
  *     which loads the library keeps until the process exits.
  *   - Limit: N*K <= 67,108,864 weights (at most 1,048,576 blocks of 64, e.g.
  *     8192 x 8192). Larger weights return QLORA_ERR_EXCEEDS_STATIC_SCRATCH
