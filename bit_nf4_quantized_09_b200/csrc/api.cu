@@ -40,6 +40,10 @@ void take_profile_events(int kernel, cudaEvent_t* start, cudaEvent_t* stop) {
 
 qlora_status cuda_fail(cudaError_t e, const char* where) {
     g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+    // a launch refused for its configuration also sets the thread's last
+    // error; read it here so that later launches checked through
+    // cudaGetLastError do not report it again
+    (void)cudaGetLastError();
     return QLORA_ERR_CUDA;
 }
 
@@ -650,6 +654,9 @@ qlora_status fwd_impl(const uint16_t* X, int64_t M, const Weights& W, const uint
         ga.ctas = L.reg_gemv.ctas;
         ga.units = L.reg_gemv.units;
         ga.stages = L.reg_gemv.stages;
+        ga.const_vec = (K / kBlock) % 4 == 0 &&
+                       (ga.absmax ? reinterpret_cast<uintptr_t>(ga.absmax) % 16 == 0
+                                  : reinterpret_cast<uintptr_t>(ga.qabsmax) % 4 == 0);
         ga.part = reinterpret_cast<float*>(base + L.partY);
         ga.counter = reinterpret_cast<int*>(base + L.ctrY);
         ga.sT = sT;

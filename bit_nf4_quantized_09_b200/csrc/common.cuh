@@ -214,6 +214,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// mbar_wait for a waiter that can take a little latency (a producer a few
+// stages ahead of its consumers): between polls the warp sleeps, 32 ns at
+// first, doubling up to 512 ns, so that it takes no issue slots from the
+// warps that compute. Bounded the same way.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, int* status) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    uint32_t ns = 32;
+    while (!mbar_try_wait(a, parity)) {
+        if (global_timer_ns() - t0 > timeout_ns) {
+            if (status) atomicOr(status, kStatusTimeout);
+            return false;
+        }
+        __nanosleep(ns);
+        ns = ns < 512 ? 2 * ns : 512;
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // Thread-block clusters (two CTAs of one GPU sharing shared memory)
 // ---------------------------------------------------------------------------

@@ -21,27 +21,36 @@
 // Decoding. A code byte holds two consecutive weights (the first in the high
 // nibble), so one 256-entry table of bf16 pairs turns a byte into the 32-bit
 // operand register of two weights. The table lives in shared memory with one
-// copy per lane (entry e of lane l at word 32 e + l): every lookup of a warp
-// hits 32 distinct banks.
+// copy per lane (entry e of lane l at byte 256 e + 4 l): every lookup of a
+// warp hits 32 distinct banks, and the offset 256 e + 4 l is a single byte
+// permute of the code word and 4 l, so a lookup costs two instructions. The
+// other 128 bytes of each 256-byte entry hold the stages' block constants.
 //
 // Data movement. A producer warp stages, per pipeline step of four block
-// columns, the packed codes of the CTA's 256 weight rows (one 128 x 256-byte
-// TMA box: 128 contiguous bytes of every row, so each DRAM access is a whole
+// columns (aligned: the step's first column is a multiple of four), the
+// packed codes of the CTA's 256 weight rows (one 128 x 256-byte TMA box: 128 contiguous bytes of every row, so each DRAM access is a whole
 // line; 128-byte swizzle) and the matching X columns of every token (one
 // 64 x M box per block column, 128-byte swizzle) into a ring of stages guarded by
 // mbarriers; every wait is bounded. Four producer warps take the steps in
 // turn: each issues its step's copies and decodes the step's block constants
 // c' (E4M3 code, second-level scale and mean, or the fp32 constant; every
-// load issued before the first use) into the stage, so four steps' load
+// load issued before the first use) beside the table, so four steps' load
 // latencies overlap and a consumer reads the four constants of a row with
-// one 16-byte load.
+// one 16-byte load. Since steps are aligned, a row's four constants of a step
+// are one aligned 4-byte word (or float4) when K/64 is a multiple of four, so
+// each row costs one load, not four scattered ones.
 //
 // Fragment layout. Lane (g, q) of a consumer warp that owns 16 weight rows
-// reads the 8 code bytes 8q .. 8q + 7 of rows g and g + 8 of each block.
+// reads the 8 code bytes 8q .. 8q + 7 of each block of two of them, its
+// fragment rows g and g + 8 (warp rows frag_row(g) and frag_row(g) + 8, an
+// order chosen so that the code loads meet no bank conflict).
 // Inside MMA step s (0..3) of a block its A-operand slots 2q, 2q + 1 hold
 // weights 16q + 4s, +1 (code byte 8q + 2s) and slots 2q + 8, 2q + 9 hold
 // weights 16q + 4s + 2, +3 (byte 8q + 2s + 1); its X fragment uses the same
-// order, X[m][16q .. 16q + 15] of the block (two swizzled 16-byte chunks).
+// order, X[m][16q .. 16q + 15] of the block (two swizzled 16-byte chunks),
+// loaded only by lanes of existing tokens (with one token, 4 lanes of 32:
+// every quarter-warp phase of a 16-byte load costs a shared-memory
+// wavefront, so loads of columns that are never written are left out).
 //
 // Work split. A CTA of 16 consumer warps owns 256 weight rows; the (row tile,
 // block column) units are dealt out in equal contiguous ranges, one per CTA,
@@ -66,16 +75,17 @@ constexpr int kProdWarps = 4;                 // producer warps: TMA (one lane) 
 constexpr int kThreads = (kWarps + kProdWarps) * 32;
 constexpr int kRowsCta = kWarps * 16;         // 256 weight rows
 constexpr int kStep = 4;                      // block columns per pipeline step
-constexpr int kMaxStages = 6;
-constexpr uint32_t kLutBytes = 256 * 32 * 4;  // 256 entries x 32 lane copies
+constexpr int kMaxStages = 6;  // at most 8: the constants of 8 stages fill the table's free halves
+// The pair table: entry e at byte 256 e, its 32 lane copies in the first 128
+// bytes; the second 128 bytes of the entries hold the stages' block constants.
+constexpr uint32_t kLutBytes = 256 * 256;
 constexpr uint32_t kCodeStage = 32 * kStep * kRowsCta;  // 128 contiguous bytes of each of the 256 rows
 
 __host__ __device__ constexpr uint32_t x_box_bytes(int64_t M) {
     return static_cast<uint32_t>((M * 128 + 1023) / 1024 * 1024);  // 1024-aligned for the 128-byte swizzle
 }
-constexpr uint32_t kConstBytes = kRowsCta * kStep * 4;  // c' of the step: [256 rows][4 blocks] fp32
 __host__ __device__ constexpr uint32_t stage_bytes(int64_t M) {
-    return kCodeStage + kStep * x_box_bytes(M) + kConstBytes;
+    return kCodeStage + kStep * x_box_bytes(M);
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
@@ -98,10 +108,17 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory"); }
 
-// The bf16 pair of code byte k of w, from this lane's copy of the table.
-__device__ __forceinline__ uint32_t lut(uint32_t lane_base, uint32_t w, uint32_t k) {
-    const uint32_t e = __byte_perm(w, 0u, 0x4440u + k);
-    return lds32(lane_base + e * 128u);
+// The bf16 pair of code byte k of w, from this lane's copy of the table at
+// `base`: one byte permute forms the offset 256 e + 4 lane (e in byte 1,
+// lane4 = 4 lane in byte 0) and the load adds the table's address.
+__device__ __forceinline__ uint32_t lut(uint32_t base, uint32_t lane4, uint32_t w, uint32_t k) {
+    return lds32(base + __byte_perm(w, lane4, 0x5504u + (k << 4)));
+}
+
+// Address of the block constants (4 x fp32) of weight row r (0..255) of
+// stage s, in the free half of table entry 32 s + r / 8.
+__device__ __forceinline__ uint32_t const_addr(uint32_t base, int s, int r) {
+    return base + static_cast<uint32_t>(32 * s + (r >> 3)) * 256u + 128u + static_cast<uint32_t>(r & 7) * 16u;
 }
 
 // The rank-r term of two 8-row halves of a warp's 16 rows, added to the
@@ -155,27 +172,39 @@ struct Sched {
     __device__ int parts(int tile) const { return cta_of(min((tile + 1) * KB, U) - 1) - cta_of(tile * KB) + 1; }
 };
 
-// Pipeline step k of a CTA's range: its segment, first block column and the
-// number of its block columns inside the segment (steps never straddle two
-// segments; the last step of a segment may be short).
+// Pipeline steps are the aligned groups of kStep block columns (first column
+// a multiple of kStep) that meet a segment's column range; step k of a CTA's
+// range: its segment, first block column and the blocks [b0, b1) of the step
+// inside the segment (the first and last step of a segment may be partial).
 struct Step {
-    int seg, col0, nb;
+    int seg, col0, b0, b1;
 };
+__device__ __forceinline__ int steps_in(int lo, int hi) { return (hi + kStep - 1) / kStep - lo / kStep; }
 __device__ __forceinline__ Step step_of(int k, int nst0, int blo0, int len0, int len1) {
     Step s;
     s.seg = k >= nst0 ? 1 : 0;
-    const int kk = s.seg ? k - nst0 : k;
-    s.col0 = (s.seg ? 0 : blo0) + kStep * kk;
-    s.nb = min(kStep, (s.seg ? len1 : len0) - kStep * kk);
+    const int lo = s.seg ? 0 : blo0, hi = s.seg ? len1 : blo0 + len0;
+    s.col0 = (lo / kStep + (s.seg ? k - nst0 : k)) * kStep;
+    s.b0 = max(lo - s.col0, 0);
+    s.b1 = min(hi - s.col0, kStep);
     return s;
 }
+
+// Warp-local weight row of MMA fragment row g (0..7; g + 8 maps to this + 8).
+// Lanes 0-15 (g < 4) then read rows 0, 2, 4, 6 and lanes 16-31 rows 1, 3, 5, 7,
+// whose 128-byte-swizzled chunk pairs are disjoint: a half-warp's 8-byte code
+// loads meet no bank twice.
+__device__ __forceinline__ int frag_row(int g) { return ((g & 3) << 1) | (g >> 2); }
 
 template <int MT, bool kNoDq>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_mma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                     const GemvMmaArgs a, const Nf4Tables tab) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // the table first (16-byte alignment suffices), then the stages on a
+    // 1024-byte boundary for the 128-byte swizzle
+    uint8_t* stages_mem =
+        reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw + kLutBytes) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
     __shared__ int last_of[2];
     __shared__ float levels[16];
@@ -193,11 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int blo0 = u0 - t0 * KB;
     const int len0 = min(u1, (t0 + 1) * KB) - u0;
     const int len1 = u1 - u0 - len0;
-    const int nst0 = (len0 + kStep - 1) / kStep, nst = nst0 + (len1 + kStep - 1) / kStep;
+    const int nst0 = steps_in(blo0, blo0 + len0), nst = nst0 + (len1 > 0 ? steps_in(0, len1) : 0);
     const int S = a.stages;
     const uint32_t xbox = x_box_bytes(M), stage = stage_bytes(M);
-    const uint32_t lut_base = smem_u32(smem);
-    const uint32_t st_base = lut_base + kLutBytes;
+    const uint32_t lut_base = smem_u32(smem_raw);
+    const uint32_t st_base = smem_u32(stages_mem);
     const uint64_t tmo = a.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -226,14 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = pw; k < nst; k += kProdWarps) {
             const int s = k % S;
             const uint32_t u = static_cast<uint32_t>(k / S);
-            if (k >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(empty + s, (u - 1) & 1u, tmo, a.status))) {
+            if (k >= S && !__all_sync(0xFFFFFFFFu, mbar_wait_sleep(empty + s, (u - 1) & 1u, tmo, a.status))) {
                 abort_flag = 1;
                 break;
             }
             if (abort_flag) break;
             const Step sp = step_of(k, nst0, blo0, len0, len1);
             const int row0 = (t0 + sp.seg) * kRowsCta;
-            uint8_t* st = smem + kLutBytes + s * stage;
+            uint8_t* st = stages_mem + s * stage;
             if (lane == 0) {
                 mbar_expect_tx(full + s, tx);
                 // whole steps even past a segment's end: the extra columns are
@@ -247,7 +276,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the step's constants: lane l decodes rows l, l + 32, ... (clamped
             // to valid rows and columns; unused ones are never read); every
             // load is issued before the first use
-            float4* cst = reinterpret_cast<float4*>(st + kCodeStage + kStep * xbox);
+            if (a.const_vec) {
+                // the step's four constants of a row are one aligned word (E4M3)
+                // or float4, and with double quantisation lie in one group of 256
+                constexpr int kVBatch = 4;  // rows whose loads are in flight together
+#pragma unroll 1
+                for (int j0 = 0; j0 < kRowsPerLane; j0 += kVBatch) {
+                    uint32_t qw[kVBatch];
+                    float sv[kVBatch];
+                    float4 av[kVBatch];
+#pragma unroll
+                    for (int j = 0; j < kVBatch; ++j) {
+                        const int64_t ib =
+                            static_cast<int64_t>(min(row0 + lane + 32 * (j0 + j), N - 1)) * KB + sp.col0;
+                        if (kNoDq) {
+                            av[j] = __ldg(reinterpret_cast<const float4*>(a.absmax + ib));
+                        } else {
+                            qw[j] = __ldg(reinterpret_cast<const uint32_t*>(a.qabsmax + ib));
+                            sv[j] = __ldg(a.s2 + (ib >> 8));
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < kVBatch; ++j) {
+                        if (!kNoDq)
+                            av[j] = make_float4(__fmaf_rn(e4m3_to_f32(qw[j]), sv[j], mean),
+                                                __fmaf_rn(e4m3_to_f32(qw[j] >> 8), sv[j], mean),
+                                                __fmaf_rn(e4m3_to_f32(qw[j] >> 16), sv[j], mean),
+                                                __fmaf_rn(e4m3_to_f32(qw[j] >> 24), sv[j], mean));
+                    {
+                        const float4 v = av[j];
+                        sts128(const_addr(lut_base, s, lane + 32 * (j0 + j)), __float_as_uint(v.x), __float_as_uint(v.y),
+                               __float_as_uint(v.z), __float_as_uint(v.w));
+                    }
+                    }
+                }
+            } else {
             constexpr int kBatch = 4;  // rows whose loads are in flight together
 #pragma unroll 1
             for (int j0 = 0; j0 < kRowsPerLane; j0 += kBatch) {
@@ -273,8 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int b = 0; b < kStep; ++b)
                         c4[b] = kNoDq ? sv[j][b] : __fmaf_rn(e4m3_to_f32(qv[j][b]), sv[j][b], mean);
-                    cst[lane + 32 * (j0 + j)] = make_float4(c4[0], c4[1], c4[2], c4[3]);
+                    sts128(const_addr(lut_base, s, lane + 32 * (j0 + j)), __float_as_uint(c4[0]), __float_as_uint(c4[1]),
+                           __float_as_uint(c4[2]), __float_as_uint(c4[3]));
                 }
+            }
             }
             mbar_arrive(full + s);  // release this lane's constants (the copies complete the phase)
         }
@@ -286,22 +351,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------ consumers --
         const int g = lane >> 2, q = lane & 3;
-        const uint32_t lane_lut = lut_base + 4u * static_cast<uint32_t>(lane);
+        const uint32_t lane4 = 4u * static_cast<uint32_t>(lane);
         // the table: entry e = bf16(level[e >> 4]) | bf16(level[e & 15]) << 16,
         // four lane copies per 16-byte store
         for (int i = threadIdx.x; i < 256 * 8; i += kWarps * 32) {
             const int e = i >> 3;
             const uint32_t v = pack_bf16x2(levels[e >> 4], levels[e & 15]);
-            sts128(lut_base + static_cast<uint32_t>(e) * 128u + static_cast<uint32_t>(i & 7) * 16u, v, v, v, v);
+            sts128(lut_base + static_cast<uint32_t>(e) * 256u + static_cast<uint32_t>(i & 7) * 16u, v, v, v, v);
         }
         consumer_bar();
 
         float acc[MT][4];
 #pragma unroll
         for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
-        // X fragment rows in a stage's box: token g + 8t (clamped to the last
-        // token: the MMA columns past M hold copies whose sums are never
-        // written), chunks 2q and 2q + 1 of its 128-byte row, swizzled
+        // X fragment rows in a stage's box: token g + 8t, chunks 2q and 2q + 1
+        // of its 128-byte row, swizzled; lanes of tokens past M load nothing
+        // and feed zeros (their MMA columns are never written)
         uint32_t xoff[MT][2];
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
@@ -309,19 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             xoff[t][0] = m * 128u + (((2u * q) ^ (m & 7u)) << 4);
             xoff[t][1] = m * 128u + (((2u * q + 1u) ^ (m & 7u)) << 4);
         }
-        // this lane's code bytes in a stage's box: rows g and g + 8 of the warp
-        // (a row past N is decoded from zero-filled codes and its sums dropped);
-        // the 8 bytes of block b sit in 16-byte chunk 2b + q/2 of the row's 128,
-        // stored at chunk (2b + q/2) ^ (row & 7)
-        const uint32_t crow_sw = static_cast<uint32_t>(g & 7);
-        const uint32_t coff = static_cast<uint32_t>(warp * 16 + g) * 128u + 8u * (q & 1);
-        const uint32_t crow = static_cast<uint32_t>(warp * 16 + g);  // its row of the constants
+        // this lane's code bytes in a stage's box: warp rows frag_row(g) and
+        // frag_row(g) + 8 (a row past N is decoded from zero-filled codes and
+        // its sums dropped); the 8 bytes of block b sit in 16-byte chunk
+        // 2b + q/2 of the row's 128, stored at chunk (2b + q/2) ^ (row & 7)
+        const int fr = frag_row(g);
+        const uint32_t crow_sw = static_cast<uint32_t>(fr & 7);
+        const uint32_t coff = static_cast<uint32_t>(warp * 16 + fr) * 128u + 8u * (q & 1);
+        const uint32_t crow = static_cast<uint32_t>(warp * 16 + fr);  // its row of the constants
         auto flush = [&](int seg) {
-            // segment done: its partial sums, acc[t][0..1] = (row g, tokens
-            // 8t + 2q, +1) and acc[t][2..3] = (row g + 8, the same tokens)
+            // segment done: its partial sums, acc[t][0..1] = (row fr, tokens
+            // 8t + 2q, +1) and acc[t][2..3] = (row fr + 8, the same tokens)
             const int tile = t0 + seg;
             const int sl = sc.slot(tile, c);
-            const int rowA = tile * kRowsCta + warp * 16 + g, rowB = rowA + 8;
+            const int rowA = tile * kRowsCta + warp * 16 + fr, rowB = rowA + 8;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
 #pragma unroll
@@ -342,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rows' two 8-row halves each lie inside one projection of a group
         auto add_rank = [&](int seg) {
             griddep_wait();  // sT from the preceding launch
-            const int64_t ra = static_cast<int64_t>(t0 + seg) * kRowsCta + warp * 16 + g;
+            const int64_t ra = static_cast<int64_t>(t0 + seg) * kRowsCta + warp * 16 + fr;
             const int64_t rA = ra < N ? ra : N - 1, rB = ra + 8 < N ? ra + 8 : N - 1;
             const int cA = rank_col(a, rA), cB = rank_col(a, rB);  // uniform over the warp
             if (cA == cB) {
@@ -362,15 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const uint32_t stc = st_base + static_cast<uint32_t>(s) * stage;
             // the step's block constants of rows g and g + 8
-            const uint4 ca4 = lds128(stc + kCodeStage + kStep * xbox + crow * 16u);
-            const uint4 cb4 = lds128(stc + kCodeStage + kStep * xbox + crow * 16u + 128u);
+            const uint4 ca4 = lds128(const_addr(lut_base, s, static_cast<int>(crow)));
+            const uint4 cb4 = lds128(const_addr(lut_base, s, static_cast<int>(crow) + 8));
             const float cA[kStep] = {__uint_as_float(ca4.x), __uint_as_float(ca4.y), __uint_as_float(ca4.z),
                                      __uint_as_float(ca4.w)};
             const float cB[kStep] = {__uint_as_float(cb4.x), __uint_as_float(cb4.y), __uint_as_float(cb4.z),
                                      __uint_as_float(cb4.w)};
 #pragma unroll
             for (int b = 0; b < kStep; ++b) {
-                if (b >= sp.nb) break;
+                if (b < sp.b0 || b >= sp.b1) continue;
                 const uint32_t ch = ((2u * b + (q >> 1)) ^ crow_sw) << 4;
                 const uint2 wa = lds64(stc + coff + ch), wb = lds64(stc + coff + ch + 1024u);
                 // A fragments of the block's four MMA steps (unscaled levels)
@@ -379,26 +445,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int st4 = 0; st4 < 4; ++st4) {
                     const uint32_t xa = st4 < 2 ? wa.x : wa.y, xb = st4 < 2 ? wb.x : wb.y;
                     const uint32_t kk = (st4 & 1) * 2;
-                    af[st4][0] = lut(lane_lut, xa, kk);
-                    af[st4][1] = lut(lane_lut, xb, kk);
-                    af[st4][2] = lut(lane_lut, xa, kk + 1);
-                    af[st4][3] = lut(lane_lut, xb, kk + 1);
+                    af[st4][0] = lut(lut_base, lane4, xa, kk);
+                    af[st4][1] = lut(lut_base, lane4, xb, kk);
+                    af[st4][2] = lut(lut_base, lane4, xa, kk + 1);
+                    af[st4][3] = lut(lut_base, lane4, xb, kk + 1);
                 }
                 const uint32_t xb0 = stc + kCodeStage + b * xbox;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    const uint4 x0 = lds128(xb0 + xoff[t][0]), x1 = lds128(xb0 + xoff[t][1]);
+                    uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+                    if (t < MT / 2 || g + 8 * t < M) {  // tiles below MT / 2 are full
+                        x0 = lds128(xb0 + xoff[t][0]);
+                        x1 = lds128(xb0 + xoff[t][1]);
+                    }
                     const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    // two independent two-step chains per block
-                    float t0v[4] = {0.0f, 0.0f, 0.0f, 0.0f}, t1v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    mma_bf16(t0v, af[0], xw[0], xw[1]);
-                    mma_bf16(t1v, af[2], xw[4], xw[5]);
-                    mma_bf16(t0v, af[1], xw[2], xw[3]);
-                    mma_bf16(t1v, af[3], xw[6], xw[7]);
-                    acc[t][0] = __fmaf_rn(t0v[0] + t1v[0], cA[b], acc[t][0]);
-                    acc[t][1] = __fmaf_rn(t0v[1] + t1v[1], cA[b], acc[t][1]);
-                    acc[t][2] = __fmaf_rn(t0v[2] + t1v[2], cB[b], acc[t][2]);
-                    acc[t][3] = __fmaf_rn(t0v[3] + t1v[3], cB[b], acc[t][3]);
+                    // the block's four MMA steps in one chain, then one FMA per
+                    // accumulator with the block constants
+                    float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    mma_bf16(tv, af[0], xw[0], xw[1]);
+                    mma_bf16(tv, af[1], xw[2], xw[3]);
+                    mma_bf16(tv, af[2], xw[4], xw[5]);
+                    mma_bf16(tv, af[3], xw[6], xw[7]);
+                    acc[t][0] = __fmaf_rn(tv[0], cA[b], acc[t][0]);
+                    acc[t][1] = __fmaf_rn(tv[1], cA[b], acc[t][1]);
+                    acc[t][2] = __fmaf_rn(tv[2], cB[b], acc[t][2]);
+                    acc[t][3] = __fmaf_rn(tv[3], cB[b], acc[t][3]);
                 }
             }
             __syncwarp();
@@ -465,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr size_t kSmemLimit = 226 * 1024;
 
 size_t smem_bytes(int64_t M, int stages) { return kLutBytes + static_cast<size_t>(stages) * stage_bytes(M) + 1024; }
+static_assert(kMaxStages <= 8, "block constants of at most 8 stages fit in the table's free halves");
 
 template <int MT, bool kNoDq>
 cudaError_t launch_mt(const CUtensorMap& codes, const CUtensorMap& x, const GemvMmaArgs& a, const Nf4Tables& tab,

@@ -180,6 +180,7 @@ struct GemvMmaArgs {
     int ctas;                // grid size (from the plan)
     int64_t units;           // (row tiles) * (K/64 block columns)
     int stages;              // shared-memory pipeline stages (from the plan)
+    int const_vec;           // K/64 % 4 == 0 and the constants aligned (qabsmax 4 B, absmax 16 B): one vector load per row and step
     float* part;             // fp32 [max_parts][M][N] partial sums
     int* counter;            // [row tiles] tickets, zero before the launch; left zero
     const uint16_t* sT;      // bf16 [M, sT_ld], read only in the epilogue

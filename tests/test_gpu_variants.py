@@ -121,10 +121,13 @@ def test_nodq_forward_backward(q, cfg):
     check("dB", f64(dB), dBr)
 
 
-def test_nodq_small_batch_four_token_tiles(q):
-    """A weight without double quantisation through the small-batch kernel
-    with 24 tokens (four n8 token tiles; forced past its default limit)."""
-    cfg = synth.custom(N=1024, K=576, M=24, r=16)
+@pytest.mark.parametrize("cfg", [synth.custom(N=1024, K=576, M=24, r=16), synth.custom(N=776, K=2048, M=5, r=8)],
+                         ids=lambda c: c.name)
+def test_nodq_small_batch_four_token_tiles(q, cfg):
+    """A weight without double quantisation through the small-batch kernel:
+    24 tokens (four n8 token tiles; forced past its default limit) with K/64
+    odd (one constant load per block), and 5 tokens with K/64 a multiple of
+    four (one float4 of constants per row and step)."""
     W, X, A, B = synth.weight(cfg), synth.activations(cfg), synth.lora_a(cfg), synth.lora_b(cfg)
     w = quantize(q, W, True)
     old = q.get_option(q.OPT_SMALL_M_MAX)
