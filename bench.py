@@ -437,7 +437,9 @@ def other_rows(q, dev):
             q.linear_fwd(Xc, wcs[i % ncopy], Ac, Bc, c.alpha, Y=Yc, sT=sTc, ws=wsc)
         torch.cuda.synchronize()
         assert_device_ok(q, [wsc], c.name)
-        tk = statistics.median(e[0].elapsed_time(e[1]) for e in evs[3:])
+        # mean, not median: single-launch event times come in steps of about
+        # 2 us here, and the mean of many launches resolves below that step
+        tk = statistics.mean(e[0].elapsed_time(e[1]) for e in evs[3:])
         gb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384) + 2 * c.M * (c.N + c.K) + 2 * c.r * (c.N + c.K)
         wb = c.N * c.K * (0.5 + 1 / 64 + 4 / 16384)
         sweep[c.name] = {"us": tf * 1e3, "GBs": gb / tf / 1e6, "frac_hbm": gb / tf / 1e6 / pk_hbm,

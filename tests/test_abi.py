@@ -123,6 +123,10 @@ def test_host_validation_without_gpu(q):
     assert bwd(dA=None) == -1
     assert bwd(dA=P + 4) == -3
     assert bwd(wsb=bws - 256) == -5
+    # the status reader needs somewhere to put the word, with or without a
+    # workspace (NULL reads the library's own word)
+    assert L.qlora_device_status(P, None, None) == -1
+    assert L.qlora_device_status(None, None, None) == -1
 
 
 def test_host_validation_storage_without_dq_and_merge(q):
