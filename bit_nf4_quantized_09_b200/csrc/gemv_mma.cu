@@ -40,9 +40,10 @@
 // are one aligned 4-byte word (or float4) when K/64 is a multiple of four, so
 // each row costs one load, not four scattered ones.
 //
-// Fragment layout. Lane (g, q) of a consumer warp that owns 16 weight rows
-// reads the 8 code bytes 8q .. 8q + 7 of each block of two of them, its
-// fragment rows g and g + 8 (warp rows frag_row(g) and frag_row(g) + 8, an
+// Fragment layout. A consumer warp owns 32 weight rows as two 16-row MMA
+// tiles, which share every X fragment it loads. In each tile, lane (g, q)
+// reads the 8 code bytes 8q .. 8q + 7 of each block of two rows, its
+// fragment rows g and g + 8 (tile rows frag_row(g) and frag_row(g) + 8, an
 // order chosen so that the code loads meet no bank conflict).
 // Inside MMA step s (0..3) of a block its A-operand slots 2q, 2q + 1 hold
 // weights 16q + 4s, +1 (code byte 8q + 2s) and slots 2q + 8, 2q + 9 hold
@@ -52,7 +53,7 @@
 // every quarter-warp phase of a 16-byte load costs a shared-memory
 // wavefront, so loads of columns that are never written are left out).
 //
-// Work split. A CTA of 16 consumer warps owns 256 weight rows; the (row tile,
+// Work split. A CTA of 8 consumer warps owns 256 weight rows; the (row tile,
 // block column) units are dealt out in equal contiguous ranges, one per CTA,
 // one CTA per SM (stream-K), so no wave is left part-empty; a range may cross
 // into the next row tile. Every CTA that touches a tile writes its fp32
@@ -70,10 +71,11 @@ namespace qlora {
 
 namespace {
 
-constexpr int kWarps = 16;                    // consumer warps
+constexpr int kTilesW = 2;                    // 16-row MMA tiles per consumer warp (sharing its X fragments)
+constexpr int kWarps = 16 / kTilesW;          // consumer warps
 constexpr int kProdWarps = 4;                 // producer warps: TMA (one lane) and the block constants
 constexpr int kThreads = (kWarps + kProdWarps) * 32;
-constexpr int kRowsCta = kWarps * 16;         // 256 weight rows
+constexpr int kRowsCta = kWarps * 16 * kTilesW;  // 256 weight rows
 constexpr int kStep = 4;                      // block columns per pipeline step
 constexpr int kMaxStages = 6;  // at most 8: the constants of 8 stages fill the table's free halves
 // The pair table: entry e at byte 256 e, its 32 lane copies in the first 128
@@ -361,9 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         consumer_bar();
 
-        float acc[MT][4];
+        float acc[kTilesW][MT][4];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+        for (int h = 0; h < kTilesW; ++h)
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc[h][t][0] = acc[h][t][1] = acc[h][t][2] = acc[h][t][3] = 0.0f;
         // X fragment rows in a stage's box: token g + 8t, chunks 2q and 2q + 1
         // of its 128-byte row, swizzled; lanes of tokens past M load nothing
         // and feed zeros (their MMA columns are never written)
@@ -374,48 +378,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             xoff[t][0] = m * 128u + (((2u * q) ^ (m & 7u)) << 4);
             xoff[t][1] = m * 128u + (((2u * q + 1u) ^ (m & 7u)) << 4);
         }
-        // this lane's code bytes in a stage's box: warp rows frag_row(g) and
-        // frag_row(g) + 8 (a row past N is decoded from zero-filled codes and
-        // its sums dropped); the 8 bytes of block b sit in 16-byte chunk
-        // 2b + q/2 of the row's 128, stored at chunk (2b + q/2) ^ (row & 7)
+        // this lane's code bytes in a stage's box: in MMA tile h of the warp,
+        // rows frag_row(g) and frag_row(g) + 8 (a row past N is decoded from
+        // zero-filled codes and its sums dropped); the 8 bytes of block b sit
+        // in 16-byte chunk 2b + q/2 of the row's 128, stored at chunk
+        // (2b + q/2) ^ (row & 7)
         const int fr = frag_row(g);
+        const int wrow = warp * 16 * kTilesW + fr;  // CTA row of tile 0's fragment row g; tile h adds 16 h
         const uint32_t crow_sw = static_cast<uint32_t>(fr & 7);
-        const uint32_t coff = static_cast<uint32_t>(warp * 16 + fr) * 128u + 8u * (q & 1);
-        const uint32_t crow = static_cast<uint32_t>(warp * 16 + fr);  // its row of the constants
+        const uint32_t coff = static_cast<uint32_t>(wrow) * 128u + 8u * (q & 1);
         auto flush = [&](int seg) {
-            // segment done: its partial sums, acc[t][0..1] = (row fr, tokens
-            // 8t + 2q, +1) and acc[t][2..3] = (row fr + 8, the same tokens)
+            // segment done: its partial sums, acc[h][t][0..1] = (row wrow +
+            // 16 h, tokens 8t + 2q, +1) and acc[h][t][2..3] = (that row + 8,
+            // the same tokens)
             const int tile = t0 + seg;
             const int sl = sc.slot(tile, c);
-            const int rowA = tile * kRowsCta + warp * 16 + fr, rowB = rowA + 8;
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
+            for (int h = 0; h < kTilesW; ++h) {
+                const int rowA = tile * kRowsCta + wrow + 16 * h, rowB = rowA + 8;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tok = 8 * t + 2 * q + e;
-                    if (tok < M) {
-                        float* pt = a.part + (static_cast<int64_t>(sl) * M + tok) * N;
-                        if (rowA < N) pt[rowA] = acc[t][e];
-                        if (rowB < N) pt[rowB] = acc[t][2 + e];
+                for (int t = 0; t < MT; ++t) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int tok = 8 * t + 2 * q + e;
+                        if (tok < M) {
+                            float* pt = a.part + (static_cast<int64_t>(sl) * M + tok) * N;
+                            if (rowA < N) pt[rowA] = acc[h][t][e];
+                            if (rowB < N) pt[rowB] = acc[h][t][2 + e];
+                        }
                     }
+                    acc[h][t][0] = acc[h][t][1] = acc[h][t][2] = acc[h][t][3] = 0.0f;
                 }
-                acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
             }
         };
 
         // the rank-r term of the warp's rows, added by the CTA whose segment
-        // ends at the tile's last block column (exactly one per tile); the
-        // rows' two 8-row halves each lie inside one projection of a group
+        // ends at the tile's last block column (exactly one per tile); each
+        // MMA tile's two 8-row halves lie inside one projection of a group
         auto add_rank = [&](int seg) {
             griddep_wait();  // sT from the preceding launch
-            const int64_t ra = static_cast<int64_t>(t0 + seg) * kRowsCta + warp * 16 + fr;
-            const int64_t rA = ra < N ? ra : N - 1, rB = ra + 8 < N ? ra + 8 : N - 1;
-            const int cA = rank_col(a, rA), cB = rank_col(a, rB);  // uniform over the warp
-            if (cA == cB) {
-                rank_mma<MT>(a, acc, rA, rB, cA, true, true, g, q);
-            } else {
-                rank_mma<MT>(a, acc, rA, rB, cA, true, false, g, q);
-                rank_mma<MT>(a, acc, rA, rB, cB, false, true, g, q);
+#pragma unroll
+            for (int h = 0; h < kTilesW; ++h) {
+                const int64_t ra = static_cast<int64_t>(t0 + seg) * kRowsCta + wrow + 16 * h;
+                const int64_t rA = ra < N ? ra : N - 1, rB = ra + 8 < N ? ra + 8 : N - 1;
+                const int cA = rank_col(a, rA), cB = rank_col(a, rB);  // uniform over the warp
+                if (cA == cB) {
+                    rank_mma<MT>(a, acc[h], rA, rB, cA, true, true, g, q);
+                } else {
+                    rank_mma<MT>(a, acc[h], rA, rB, cA, true, false, g, q);
+                    rank_mma<MT>(a, acc[h], rA, rB, cB, false, true, g, q);
+                }
             }
         };
 
@@ -427,28 +439,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(full + s, u & 1u, tmo, a.status));
             if (!ok) break;
             const uint32_t stc = st_base + static_cast<uint32_t>(s) * stage;
-            // the step's block constants of rows g and g + 8
-            const uint4 ca4 = lds128(const_addr(lut_base, s, static_cast<int>(crow)));
-            const uint4 cb4 = lds128(const_addr(lut_base, s, static_cast<int>(crow) + 8));
-            const float cA[kStep] = {__uint_as_float(ca4.x), __uint_as_float(ca4.y), __uint_as_float(ca4.z),
-                                     __uint_as_float(ca4.w)};
-            const float cB[kStep] = {__uint_as_float(cb4.x), __uint_as_float(cb4.y), __uint_as_float(cb4.z),
-                                     __uint_as_float(cb4.w)};
+            // the step's block constants of each tile's rows fr and fr + 8
+            float cA[kTilesW][kStep], cB[kTilesW][kStep];
+#pragma unroll
+            for (int h = 0; h < kTilesW; ++h) {
+                const uint4 ca4 = lds128(const_addr(lut_base, s, wrow + 16 * h));
+                const uint4 cb4 = lds128(const_addr(lut_base, s, wrow + 16 * h + 8));
+                cA[h][0] = __uint_as_float(ca4.x);
+                cA[h][1] = __uint_as_float(ca4.y);
+                cA[h][2] = __uint_as_float(ca4.z);
+                cA[h][3] = __uint_as_float(ca4.w);
+                cB[h][0] = __uint_as_float(cb4.x);
+                cB[h][1] = __uint_as_float(cb4.y);
+                cB[h][2] = __uint_as_float(cb4.z);
+                cB[h][3] = __uint_as_float(cb4.w);
+            }
 #pragma unroll
             for (int b = 0; b < kStep; ++b) {
                 if (b < sp.b0 || b >= sp.b1) continue;
                 const uint32_t ch = ((2u * b + (q >> 1)) ^ crow_sw) << 4;
-                const uint2 wa = lds64(stc + coff + ch), wb = lds64(stc + coff + ch + 1024u);
-                // A fragments of the block's four MMA steps (unscaled levels)
-                uint32_t af[4][4];
+                // A fragments of the block's four MMA steps of each tile
+                // (unscaled levels)
+                uint32_t af[kTilesW][4][4];
 #pragma unroll
-                for (int st4 = 0; st4 < 4; ++st4) {
-                    const uint32_t xa = st4 < 2 ? wa.x : wa.y, xb = st4 < 2 ? wb.x : wb.y;
-                    const uint32_t kk = (st4 & 1) * 2;
-                    af[st4][0] = lut(lut_base, lane4, xa, kk);
-                    af[st4][1] = lut(lut_base, lane4, xb, kk);
-                    af[st4][2] = lut(lut_base, lane4, xa, kk + 1);
-                    af[st4][3] = lut(lut_base, lane4, xb, kk + 1);
+                for (int h = 0; h < kTilesW; ++h) {
+                    const uint32_t ca = stc + coff + static_cast<uint32_t>(h) * 2048u + ch;
+                    const uint2 wa = lds64(ca), wb = lds64(ca + 1024u);
+#pragma unroll
+                    for (int st4 = 0; st4 < 4; ++st4) {
+                        const uint32_t xa = st4 < 2 ? wa.x : wa.y, xb = st4 < 2 ? wb.x : wb.y;
+                        const uint32_t kk = (st4 & 1) * 2;
+                        af[h][st4][0] = lut(lut_base, lane4, xa, kk);
+                        af[h][st4][1] = lut(lut_base, lane4, xb, kk);
+                        af[h][st4][2] = lut(lut_base, lane4, xa, kk + 1);
+                        af[h][st4][3] = lut(lut_base, lane4, xb, kk + 1);
+                    }
                 }
                 const uint32_t xb0 = stc + kCodeStage + b * xbox;
 #pragma unroll
@@ -459,17 +484,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x1 = lds128(xb0 + xoff[t][1]);
                     }
                     const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    // the block's four MMA steps in one chain, then one FMA per
-                    // accumulator with the block constants
-                    float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    mma_bf16(tv, af[0], xw[0], xw[1]);
-                    mma_bf16(tv, af[1], xw[2], xw[3]);
-                    mma_bf16(tv, af[2], xw[4], xw[5]);
-                    mma_bf16(tv, af[3], xw[6], xw[7]);
-                    acc[t][0] = __fmaf_rn(tv[0], cA[b], acc[t][0]);
-                    acc[t][1] = __fmaf_rn(tv[1], cA[b], acc[t][1]);
-                    acc[t][2] = __fmaf_rn(tv[2], cB[b], acc[t][2]);
-                    acc[t][3] = __fmaf_rn(tv[3], cB[b], acc[t][3]);
+                    // per tile, the block's four MMA steps in one chain, then
+                    // one FMA per accumulator with the block constants
+#pragma unroll
+                    for (int h = 0; h < kTilesW; ++h) {
+                        float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        mma_bf16(tv, af[h][0], xw[0], xw[1]);
+                        mma_bf16(tv, af[h][1], xw[2], xw[3]);
+                        mma_bf16(tv, af[h][2], xw[4], xw[5]);
+                        mma_bf16(tv, af[h][3], xw[6], xw[7]);
+                        acc[h][t][0] = __fmaf_rn(tv[0], cA[h][b], acc[h][t][0]);
+                        acc[h][t][1] = __fmaf_rn(tv[1], cA[h][b], acc[h][t][1]);
+                        acc[h][t][2] = __fmaf_rn(tv[2], cB[h][b], acc[h][t][2]);
+                        acc[h][t][3] = __fmaf_rn(tv[3], cB[h][b], acc[h][t][3]);
+                    }
                 }
             }
             __syncwarp();
@@ -537,6 +565,7 @@ constexpr size_t kSmemLimit = 226 * 1024;
 
 size_t smem_bytes(int64_t M, int stages) { return kLutBytes + static_cast<size_t>(stages) * stage_bytes(M) + 1024; }
 static_assert(kMaxStages <= 8, "block constants of at most 8 stages fit in the table's free halves");
+static_assert(kRowsCta == 256, "the codes tensor map's box is 256 rows");
 
 template <int MT, bool kNoDq>
 cudaError_t launch_mt(const CUtensorMap& codes, const CUtensorMap& x, const GemvMmaArgs& a, const Nf4Tables& tab,
