@@ -4,9 +4,8 @@
 // bound by streaming the packed weight (about half a byte per weight);
 // "ta-paperlens QLoRA explainer", 落とし穴, names this small-batch regime as
 // the one where 4-bit weights pay off. The kernel is shaped so that the
-// decode and its bookkeeping cost fewer instructions than the stream allows:
-// per two weights one byte permute, one integer multiply-add and one
-// shared-memory load.
+// decode and its bookkeeping stay a few instructions per weight: per two
+// weights one byte permute and one shared-memory load from a table.
 //
 // Factored dequantisation. Within a 64-weight block every weight is
 // level[code] * c'_b, so for output row n
@@ -28,9 +27,10 @@
 //
 // Data movement. A producer warp stages, per pipeline step of four block
 // columns (aligned: the step's first column is a multiple of four), the
-// packed codes of the CTA's 256 weight rows (one 128 x 256-byte TMA box: 128 contiguous bytes of every row, so each DRAM access is a whole
-// line; 128-byte swizzle) and the matching X columns of every token (one
-// 64 x M box per block column, 128-byte swizzle) into a ring of stages guarded by
+// packed codes of the CTA's 256 weight rows (one 128 x 256-byte TMA box:
+// 128 contiguous bytes of every row, so each DRAM access is a whole line;
+// 128-byte swizzle) and the matching X columns of every token (one 64 x M
+// box per block column, 128-byte swizzle) into a ring of stages guarded by
 // mbarriers; every wait is bounded. Four producer warps take the steps in
 // turn: each issues its step's copies and decodes the step's block constants
 // c' (E4M3 code, second-level scale and mean, or the fp32 constant; every
