@@ -37,15 +37,44 @@ namespace qlora {
 // IEEE division instead (so no remainder of a value near a threshold can be
 // subnormal), and values far below every threshold code to the zero level
 // either way.
+// The quotient's three roundings and the cell index's fma run on pairs of
+// weights in the packed fp32x2 instructions of sm_100 (each half an IEEE
+// fp32 operation with round-to-nearest, so every result is bit for bit the
+// scalar one), halving their issue slots.
 // Loads of the next block run ahead of the current block's arithmetic.
 // ---------------------------------------------------------------------------
 constexpr int kCells = 129;
 constexpr int kCellCopies = 16;
 
-__device__ __forceinline__ uint32_t nf4_code(float q, const float2* sLut, int copy) {
-    const int j = __float_as_int(__fmaf_rn(q, 64.0f, 12582976.0f)) - 0x4B400000;  // RN(64 q + 64), 0..128
+// The code of q, given jbits = the bits of fma(q, 64, 1.5 * 2^23 + 64).
+__device__ __forceinline__ uint32_t nf4_code_j(float q, uint32_t jbits, const float2* sLut, int copy) {
+    const int j = static_cast<int>(jbits - 0x4B400000u);  // RN(64 q + 64), 0..128
     const float2 e = sLut[j * kCellCopies + copy];  // {threshold in the cell (2 if none), thresholds below}
     return static_cast<uint32_t>(__float_as_int(e.y)) + (q > e.x ? 1u : 0u);
+}
+
+__device__ __forceinline__ uint32_t nf4_code(float q, const float2* sLut, int copy) {
+    return nf4_code_j(q, __float_as_uint(__fmaf_rn(q, 64.0f, 12582976.0f)), sLut, copy);
+}
+
+// Packed fp32 pairs: lo in bits 0..31, hi in bits 32..63.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
 // One thread's eight consecutive weights of a block, as loaded: two float4
@@ -137,12 +166,22 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const void* __restrict_
             word = 0x77777777u;  // all-zero block: every element is the exact-zero level
         } else if (c >= 0x1p-96f) {
             const float y = __frcp_rn(c);
+            const uint64_t y2 = f2_pack(y, y), nc2 = f2_pack(-c, -c);
+            const uint64_t k64 = f2_pack(64.0f, 64.0f), kmagic = f2_pack(12582976.0f, 12582976.0f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float q0 = __fmul_rn(v[i], y);
-                const float rem = __fmaf_rn(-c, q0, v[i]);
-                const float q = __fmaf_rn(rem, y, q0);
-                word |= nf4_code(q, sLut, copy) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+            for (int i = 0; i < 8; i += 2) {
+                // weights i and i + 1: q = RN(v / c) and the cell fma, in pairs
+                const uint64_t v2 = f2_pack(v[i], v[i + 1]);
+                const uint64_t q0 = f2_mul(v2, y2);
+                const uint64_t rem = f2_fma(nc2, q0, v2);
+                const uint64_t q = f2_fma(rem, y2, q0);
+                const uint64_t jb = f2_fma(q, k64, kmagic);
+                float qa, qb, ja, jbf;
+                f2_unpack(q, qa, qb);
+                f2_unpack(jb, ja, jbf);
+                const uint32_t ca = nf4_code_j(qa, __float_as_uint(ja), sLut, copy);
+                const uint32_t cb = nf4_code_j(qb, __float_as_uint(jbf), sLut, copy);
+                word |= ((ca << 4) | cb) << (4 * i);  // element i in the high nibble of byte i / 2
             }
         } else {
 #pragma unroll
