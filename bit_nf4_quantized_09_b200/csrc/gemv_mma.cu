@@ -22,8 +22,9 @@
 // operand register of two weights. The table lives in shared memory with one
 // copy per lane (entry e of lane l at byte 256 e + 4 l): every lookup of a
 // warp hits 32 distinct banks, and the offset 256 e + 4 l is a single byte
-// permute of the code word and 4 l, so a lookup costs two instructions. The
-// other 128 bytes of each 256-byte entry hold the stages' block constants.
+// permute of the code word and 4 l, so a lookup is that permute and a
+// shared-memory load at the offset from the table's address. The other 128
+// bytes of each 256-byte entry hold the stages' block constants.
 //
 // Data movement. A producer warp stages, per pipeline step of four block
 // columns (aligned: the step's first column is a multiple of four), the
